@@ -1,0 +1,428 @@
+"""Benchmark of the int4 mixture-of-experts FFN layer (libmoe_int4) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload scout_decode]
+
+One step = one full layer forward (routing, bucketing, routed SwiGLU experts,
+shared expert, weighted combine) over one batch of synthetic tokens already
+resident in HBM.  For N > 1 (launched by torch.distributed.run) every rank
+runs an independent replica of the workload (the layer does not shard), and
+the reported throughput is all ranks' tokens over the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (the plain numpy restatement of the
+layer) on rank 0 on a bounded sample of the same workload; other ranks exit.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE layer tokens/s; % of HBM roofline (decode) / BF16-FP8 TC peak (prefill)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_text(s: synth.LayerShape) -> str:
+    w = "int4 g128" if s.fmt == "int4" else "fp8 e4m3 rows"
+    gate = "sigmoid" if s.k == 1 else "softmax over top-%d" % s.k
+    return ("%s: T=%d tokens, d_model=%d, expert d_ff=%d, E=%d routed experts (%s), top-%d %s gate, "
+            "bf16 shared expert d_ff=%d%s" % (s.name, s.T, s.D, s.F, s.E, w, s.k, gate, s.F_shared,
+                                               ", Zipf router bias" if s.skewed else ""))
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed loop runs
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--id=" + uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception as e:  # no nvidia-smi: report no clocks
+            log("clock sampling unavailable:", e)
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if not self.proc or not self.lines:
+            return None
+        inside = [l for t, l in self.lines if t0 <= t <= t1] or [l for _, l in self.lines]
+        sm, mx, reasons = [], None, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in inside:
+            parts = [p.strip() for p in l.split(",")]
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names[1:], parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
+    import int4_quantized_expert_b200 as moe
+    E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
+    wr = synth.router_weight(seed, E, D).to(dev)
+    bias = synth.router_bias(shape)
+    bias = None if bias is None else torch.from_numpy(bias).to(dev)
+    sg, su, sd = (t.to(dev) for t in synth.shared_weights(seed, D, Fs))
+    alloc = lambda n, kk: (torch.empty(E, n, kk // 2, dtype=torch.uint8, device=dev),
+                           torch.empty(E, n, kk // 128, dtype=torch.float32, device=dev))
+    gate, up, down = alloc(F, D), alloc(F, D), alloc(D, F)
+    for e, g, u, d in synth.iter_expert_weights(seed, range(E), D, F):
+        for w, (c, s) in ((g, gate), (u, up), (d, down)):
+            moe.quantize_int4(torch.from_numpy(w).to(dev), out=(c[e], s[e]))
+    torch.cuda.synchronize()
+    layer = moe.MoELayer(E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr, router_bias=bias, gate=gate,
+                         up=up, down=down, shared=(sg, su, sd), T_max=shape.T)
+    x = synth.tokens(seed, shape.T, D).to(dev)
+    return layer, x, (wr, bias)
+
+
+def kernel_bytes(shape: synth.LayerShape, n_touched: int) -> dict:
+    """Algorithmic HBM bytes per launch of each decode-path kernel: every
+    weight byte of a touched expert and of the shared expert read once, every
+    activation read and written once."""
+    T, D, F, Fs, E, k = shape.T, shape.D, shape.F, shape.F_shared, shape.E, shape.k
+    S = T * k
+    codes_gu = 2 * F * D // 2
+    scales_gu = 2 * F * (D // 128) * 4
+    codes_d = D * F // 2
+    scales_d = D * (F // 128) * 4
+    return {
+        "route_topk": T * D * 2 + E * D * 2 + T * D * 2 + S * 8,
+        "bucket": S * 4 * 3 + (E + 1) * 8,
+        "decode_plan": (E + 1) * 8,
+        "decode_gate_up": n_touched * (codes_gu + scales_gu) + 2 * Fs * D * 2 + T * D * 2 + (S * F + T * Fs) * 2,
+        "decode_down": n_touched * (codes_d + scales_d) + D * Fs * 2 + (S * F + T * Fs) * 2 + (S + T) * D * 4,
+        "combine": (S + T) * D * 4 + T * D * 2,
+    }
+
+
+def run_ours(args, rank: int, world: int, dev: torch.device):
+    import int4_quantized_expert_b200 as moe
+    shape = synth.SHAPES[args.workload]
+    layer, x, (wr, bias) = build_layer(shape, args.seed + 0, dev)
+    r = moe.route(x, wr, bias, shape.k)
+    n_touched = int((r["counts"] > 0).sum().item())
+    names = layer.launch_names(shape.T)
+    out = torch.empty(shape.T, shape.D, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)    # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def new_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        for e in evs:
+            e.record(stream)          # create the underlying cudaEvent_t
+        return evs
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer.forward(x, out)
+    torch.cuda.synchronize()
+    assert layer.device_status() == moe.Status.OK
+
+    events = [new_events() for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()                 # L2 flushed between steps (outside the step's events)
+        layer.forward_timed(x, out, events[i])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler else None
+    if sampler:
+        sampler.stop()
+    status = layer.device_status()
+    if status != moe.Status.OK:
+        raise RuntimeError("device status %d after the timed loop" % status)
+
+    per_kernel = np.zeros(len(names))
+    step_ms = np.zeros(args.steps)
+    for i, evs in enumerate(events):
+        for j in range(len(names)):
+            per_kernel[j] += evs[j].elapsed_time(evs[j + 1])
+        step_ms[i] = evs[0].elapsed_time(evs[-1])
+    per_kernel /= args.steps
+    ms = float(step_ms.mean())
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end through the host-buffer entry point (copies inside the timed region)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    n_e2e = max(3, min(args.steps, 200))
+    for _ in range(3):
+        layer.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for _ in range(n_e2e):
+        flush.zero_()
+        e0.record(stream)
+        layer.forward_host(xh, oh)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    kb = kernel_bytes(shape, n_touched)
+    dom = int(np.argmax(per_kernel))
+    dom_name = names[dom]
+    peak, peak_src = peaks()
+    achieved = kb[dom_name] / (per_kernel[dom] * 1e-3) / 1e9
+    layer_bytes = sum(kb.values())
+
+    result = {
+        "metric": METRIC,
+        "value": world * shape.T / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
+        "config": {
+            "workload": workload_text(shape),
+            "weights": "routed int4 g128 (fp32 scales, zero point 0); router and shared bf16",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "experts_touched": n_touched,
+            "l2": "flushed between steps (256 MB write); weights 1.3 GB exceed L2",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": dom_name,
+            "achieved": achieved,
+            "peak": peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": None,
+            "algorithmic_bytes": kb[dom_name],
+        },
+        "layer": {
+            "algorithmic_bytes": layer_bytes,
+            "achieved_gbs": layer_bytes / (ms * 1e-3) / 1e9,
+            "frac_of_peak": layer_bytes / (ms * 1e-3) / 1e9 / peak,
+            "per_kernel_ms": {n: float(v) for n, v in zip(names, per_kernel)},
+        },
+        "e2e": {
+            "value": world * shape.T / (e2e_ms * 1e-3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": shape.T * shape.D * 2,
+            "d2h_bytes_per_step": shape.T * shape.D * 2,
+            "ms_per_step": e2e_ms,
+        },
+        "gpu_launches": len(names) * args.steps,
+        "clocks": clocks,
+    }
+    return result, shape
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------
+def oracle_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_layer(shape: synth.LayerShape, seed: int, f_sub: int, token: int, x):
+    """The oracle's layer restricted to the first f_sub hidden units of every
+    expert (and of the shared expert): a layer of the same kind whose work per
+    token is f_sub / F of the full one.  Weights are quantized before timing."""
+    from oracle import ffn as offn, quant as oq, route as oroute
+    wr = synth.router_weight(seed, shape.E, shape.D)
+    bias = synth.router_bias(shape)
+    ids = oroute.route(x[token:token + 1], wr, bias, shape.k)["ids"][0]
+    sg, su, sd = synth.shared_weights(seed, shape.D, shape.F_shared)
+    fs_sub = max(128, f_sub * shape.F_shared // shape.F // 128 * 128)
+    experts = {}
+    for e in ids:
+        g, u, d = synth.expert_weights(seed, int(e), shape.D, shape.F)
+        experts[int(e)] = tuple(oq.int4_row_quantize(np.ascontiguousarray(w))
+                                for w in (g[:f_sub], u[:f_sub], d[:, :f_sub]))
+    return offn.Layer(shape.fmt, shape.k, wr, bias, experts.__getitem__,
+                      (sg[:fs_sub], su[:fs_sub], sd[:, :fs_sub].contiguous())), fs_sub
+
+
+def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: int, n_warm: int):
+    """Runs the oracle for one token per step on a hidden-width slice sized so
+    a step takes about budget_s; returns (tokens/s, sample text, per-step s)."""
+    from oracle import ffn as offn
+    x = synth.tokens(seed, shape.T, shape.D)
+    probe_f = 128
+    lay, fs = oracle_sample_layer(shape, seed, probe_f, 0, x)
+    t = time.perf_counter()
+    offn.moe_forward(lay, x, tokens=[0])
+    c128 = max(time.perf_counter() - t, 1e-4)
+    f_sub = int(min(shape.F, max(128, (budget_s / c128) * 128 // 128 * 128)))
+    lay, fs = oracle_sample_layer(shape, seed, f_sub, 0, x)
+    for _ in range(n_warm):
+        offn.moe_forward(lay, x, tokens=[0])
+    t = time.perf_counter()
+    for _ in range(n_steps):
+        offn.moe_forward(lay, x, tokens=[0])
+    el = (time.perf_counter() - t) / max(n_steps, 1)
+    frac = f_sub / shape.F
+    sample = ("1 token of %s per step, its routed expert(s) and the shared expert restricted to the first "
+              "%d of %d (shared %d of %d) hidden units, i.e. %.4f of a token's FFN work; routing over all %d "
+              "tokens; tokens/s scaled by that fraction" % (shape.name, f_sub, shape.F, fs, shape.F_shared,
+                                                           frac, shape.T))
+    return frac / el, sample, el
+
+
+def run_reference(args):
+    shape = synth.SHAPES[args.workload]
+    budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
+    v, sample, per_step = time_oracle(shape, args.seed, budget, args.steps, args.warmup)
+    cores = oracle_cores()
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": "tokens/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
+        "config": {"workload": workload_text(shape), "weights": "routed int4 g128; router and shared bf16",
+                   "parallelism": "CPU oracle on the host cores"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="scout_decode", choices=["tiny", "scout_decode"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    result, shape = run_ours(args, rank, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = time_oracle(shape, args.seed, budget_s=10.0, n_steps=2, n_warm=0)
+        result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle_cores(),
+                                  "kind": "oracle", "sample": sample}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,331 @@
+// extern "C" entry points of libmoe_int4: argument checks, workspace layout,
+// and the stream-ordered launch sequence of each operation.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "ffn_decode.cuh"
+
+namespace moe {
+moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, uint8_t* codes, float* scales,
+                                cudaStream_t stream);
+moe_status launch_quantize_fp8_rows(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                                    int64_t num_valid, float scale_ub, uint8_t* q, float* scales,
+                                    cudaStream_t stream);
+moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
+                        int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
+                        int32_t* inv_perm, bf16* x_frag, int32_t* zero_words, int n_zero, cudaStream_t stream,
+                        cudaEvent_t between = nullptr);
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxT = 1 << 20;
+constexpr int kMaxDim = 16384;
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool valid_dim(int32_t v) { return v >= 128 && v <= kMaxDim && v % 128 == 0; }
+
+moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
+    if (T < 1 || T > kMaxT) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!valid_dim(D)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (E < 1 || E > 256 || k < 1 || k > E || k > 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+// Workspace regions, each 256-byte aligned.
+struct WsLayout {
+    size_t status, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t x_frag, h_r, h_s, y_r, y_s, x_in, out, total;
+};
+
+WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
+    WsLayout w;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    const int64_t S = T * L.k;
+    w.status = take(64);
+    w.counters = take(64);
+    w.ids = take(S * 4);
+    w.gates = take(S * 4);
+    w.counts = take(size_t(L.E) * 4);
+    w.offsets = take(size_t(L.E + 1) * 4);
+    w.perm = take(S * 4);
+    w.inv_perm = take(S * 4);
+    w.chunks = take(size_t(decode_max_chunks(int(T), L.k, L.E)) * sizeof(ChunkEntry));
+    w.nchunks = take(16);
+    w.x_frag = take(T * L.D * 2);
+    w.h_r = take(S * L.F * 2);
+    w.h_s = take(T * L.F_shared * 2);
+    w.y_r = take(S * L.D * 4);
+    w.y_s = take(T * L.D * 4);
+    w.x_in = take(T * L.D * 2);
+    w.out = take(T * L.D * 2);
+    w.total = off;
+    return w;
+}
+
+moe_status check_layer(const moe_layer_desc* L) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    if (L->E < 1 || L->E > 256 || L->k < 1 || L->k > L->E || L->k > 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!valid_dim(L->D) || !valid_dim(L->F) || !valid_dim(L->F_shared)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->format != MOE_WEIGHTS_INT4_G128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {L->w_router, L->w_gate, L->s_gate, L->w_up, L->s_up, L->w_down, L->s_down,
+                          L->ws_gate, L->ws_up, L->ws_down};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (L->router_bias && !aligned16(L->router_bias)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Optional per-launch timing: event i is recorded before the i-th kernel of
+// the layer, the last one after the final kernel.
+struct Marks {
+    void* const* ev = nullptr;
+    int32_t n = 0;
+    int32_t i = 0;
+    void mark(cudaStream_t st) {
+        if (ev && i < n) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
+        ++i;
+    }
+};
+
+const char* const kDecodeLaunches[] = {"route_topk", "bucket", "decode_plan", "decode_gate_up",
+                                       "decode_down", "combine"};
+constexpr int32_t kDecodeLaunchCount = 6;
+
+template <typename T>
+T* at(void* base, size_t off) {
+    return reinterpret_cast<T*>(static_cast<unsigned char*>(base) + off);
+}
+
+moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
+                           const WsLayout& W, cudaStream_t st, Marks& mk) {
+    int32_t* status = at<int32_t>(ws, W.status);
+    int32_t* counters = at<int32_t>(ws, W.counters);
+    int32_t* perm = at<int32_t>(ws, W.perm);
+    int32_t* inv = at<int32_t>(ws, W.inv_perm);
+    float* gates = at<float>(ws, W.gates);
+    bf16* x_frag = at<bf16>(ws, W.x_frag);
+    bf16* h_r = at<bf16>(ws, W.h_r);
+    bf16* h_s = at<bf16>(ws, W.h_s);
+    float* y_r = at<float>(ws, W.y_r);
+    float* y_s = at<float>(ws, W.y_s);
+    ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
+    int32_t* nch = at<int32_t>(ws, W.nchunks);
+
+    mk.mark(st);
+    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+                                at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
+                                at<int32_t>(ws, W.offsets), perm, inv, x_frag, nullptr, 0, st,
+                                (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
+    ++mk.i;
+    if (s != MOE_OK) return s;
+    mk.mark(st);
+    s = launch_decode_plan(at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), T, L.E, chunks, nch, nch + 1,
+                           counters, st);
+    if (s != MOE_OK) return s;
+
+    DecodeMaps m1, m2;
+    const uint64_t E = uint64_t(L.E);
+    bool ok = make_tmap_2d(&m1.r0, L.w_gate, false, L.D / 2, E * L.F, 128, 32, true) &&
+              make_tmap_2d(&m1.r1, L.w_up, false, L.D / 2, E * L.F, 128, 32, true) &&
+              make_tmap_2d(&m1.s0, L.ws_gate, true, L.D, L.F_shared, 64, 32, true) &&
+              make_tmap_2d(&m1.s1, L.ws_up, true, L.D, L.F_shared, 64, 32, true) &&
+              make_tmap_2d(&m2.r0, L.w_down, false, L.F / 2, E * L.D, 128, 32, true) &&
+              make_tmap_2d(&m2.s0, L.ws_down, true, L.F_shared, L.D, 64, 32, true);
+    if (!ok) return MOE_ERR_CUDA;
+    m2.r1 = m2.r0;
+    m2.s1 = m2.s0;
+
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.n_rows_r = L.F;
+    p.n_rows_s = L.F_shared;
+    p.K_r = L.D;
+    p.K_s = L.D;
+    p.k_top = L.k;
+    p.scale_buf_floats = 2 * 32 * (L.D / kGroup);
+    p.chunks = chunks;
+    p.n_chunks = nch;
+    p.n_shared_chunks = nch + 1;
+    p.perm = perm;
+    p.gates = gates;
+    p.b_r = x_frag;
+    p.ldb_r = L.D;
+    p.b_s = x_frag;
+    p.ldb_s = L.D;
+    p.sc0 = L.s_gate;
+    p.sc1 = L.s_up;
+    p.h_r = h_r;
+    p.h_s = h_s;
+    p.task_counter = counters;
+    p.status = status;
+    mk.mark(st);
+    s = launch_decode_ffn(0, m1, p, st);
+    if (s != MOE_OK) return s;
+
+    p.n_rows_r = L.D;
+    p.n_rows_s = L.D;
+    p.K_r = L.F;
+    p.K_s = L.F_shared;
+    p.scale_buf_floats = 32 * (L.F / kGroup);
+    p.b_r = h_r;
+    p.ldb_r = L.F;
+    p.b_s = h_s;
+    p.ldb_s = L.F_shared;
+    p.sc0 = L.s_down;
+    p.sc1 = nullptr;
+    p.y_r = y_r;
+    p.y_s = y_s;
+    p.task_counter = counters + 1;
+    mk.mark(st);
+    s = launch_decode_ffn(1, m2, p, st);
+    if (s != MOE_OK) return s;
+    mk.mark(st);
+    s = launch_combine(y_s, y_r, inv, T, L.D, L.k, out, st);
+    mk.mark(st);
+    return s;
+}
+
+moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t T, void* out, void* workspace,
+                            size_t workspace_bytes, cudaStream_t st, Marks mk = Marks()) {
+    moe_status s = check_layer(layer);
+    if (s != MOE_OK) return s;
+    s = check_route_shape(T, layer->D, layer->E, layer->k);
+    if (s != MOE_OK) return s;
+    if (!x || !out || !workspace || !aligned16(x) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout W = ws_layout(*layer, T);
+    if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (decode_smem_bytes(2 * 32 * (layer->D / kGroup)) > 227 * 1024 ||
+        decode_smem_bytes(32 * (layer->F / kGroup)) > 227 * 1024)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (layer->path == MOE_PATH_PREFILL) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return ffn_decode_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t moe_abi_version(void) { return 1; }
+
+moe_status moe_quantize_int4(const float* w, int64_t rows, int64_t cols, int32_t group_size, uint8_t* codes,
+                             float* scales, void* stream) {
+    if (group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows < 0 || cols <= 0 || cols % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0) return MOE_OK;
+    if (!w || !codes || !scales || !aligned16(w) || !aligned16(codes) || !aligned16(scales))
+        return MOE_ERR_INVALID_ARG;
+    return launch_quantize_int4(w, rows, cols, codes, scales, as_stream(stream));
+}
+
+moe_status moe_quantize_fp8_rows(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                                 int64_t num_valid_rows, float scale_ub, uint8_t* q, float* scales,
+                                 void* stream) {
+    if (x_dtype != MOE_DTYPE_BF16 && x_dtype != MOE_DTYPE_FP32) return MOE_ERR_INVALID_ARG;
+    if (rows < 0 || cols <= 0 || cols % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (num_valid_rows < 0 || num_valid_rows > rows) return MOE_ERR_INVALID_ARG;
+    if (!(scale_ub > 0.0f)) return MOE_ERR_INVALID_ARG;   // also rejects NaN
+    if (rows == 0) return MOE_OK;
+    if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+    return launch_quantize_fp8_rows(x, x_dtype, rows, cols, num_valid_rows, scale_ub, q, scales,
+                                    as_stream(stream));
+}
+
+moe_status moe_route(const void* x, int32_t T, int32_t D, const void* w_router, const float* router_bias,
+                     int32_t E, int32_t k, int32_t* topk_ids, float* topk_gates, int32_t* expert_counts,
+                     int32_t* expert_offsets, int32_t* perm, void* stream) {
+    moe_status s = check_route_shape(T, D, E, k);
+    if (s != MOE_OK) return s;
+    const void* ptrs[] = {x, w_router, topk_ids, topk_gates, expert_counts, expert_offsets, perm};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (router_bias && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
+    return launch_route(static_cast<const bf16*>(x), T, D, static_cast<const bf16*>(w_router), router_bias, E, k,
+                        topk_ids, topk_gates, expert_counts, expert_offsets, perm, nullptr, nullptr, nullptr, 0,
+                        as_stream(stream));
+}
+
+size_t moe_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max) {
+    if (check_layer(layer) != MOE_OK || T_max < 1 || T_max > kMaxT) return 0;
+    return ws_layout(*layer, T_max).total;
+}
+
+moe_status moe_ffn_forward(const moe_layer_desc* layer, const void* x, int32_t T, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    return ffn_forward_impl(layer, x, T, out, workspace, workspace_bytes, as_stream(stream));
+}
+
+moe_status moe_ffn_forward_host(const moe_layer_desc* layer, const void* x_host, int32_t T, void* out_host,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    moe_status s = check_layer(layer);
+    if (s != MOE_OK) return s;
+    s = check_route_shape(T, layer->D, layer->E, layer->k);
+    if (s != MOE_OK) return s;
+    if (!x_host || !out_host || !workspace) return MOE_ERR_INVALID_ARG;
+    const WsLayout W = ws_layout(*layer, T);
+    if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = as_stream(stream);
+    const size_t bytes = size_t(T) * layer->D * 2;
+    void* xd = at<void>(workspace, W.x_in);
+    void* od = at<void>(workspace, W.out);
+    if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+    s = ffn_forward_impl(layer, xd, T, od, workspace, workspace_bytes, st);
+    if (s != MOE_OK) return s;
+    if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream, void* const* events,
+                                 int32_t n_events) {
+    if (!events || n_events < kDecodeLaunchCount + 1) return MOE_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_events; ++i)
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+    Marks mk;
+    mk.ev = events;
+    mk.n = n_events;
+    return ffn_forward_impl(layer, x, T, out, workspace, workspace_bytes, as_stream(stream), mk);
+}
+
+int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, const char** names, int32_t max_names) {
+    if (check_layer(layer) != MOE_OK || T < 1) return 0;
+    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
+    return kDecodeLaunchCount;
+}
+
+moe_status moe_ffn_device_status(const void* workspace, void* stream) {
+    if (!workspace) return MOE_ERR_INVALID_ARG;
+    int32_t v = 0;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    return v == DEV_OK ? MOE_OK : MOE_ERR_TIMEOUT;
+}
+
+}  // extern "C"

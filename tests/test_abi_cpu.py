@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import int4_quantized_expert_b200 as moe
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe_int4.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(moe.LIB_PATH):
+        from int4_quantized_expert_b200 import build
+        build.build()
+    return moe.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    assert lib.moe_status_string(0) == b"ok"
+    assert lib.moe_status_string(3) == b"workspace too small"
+    assert lib.moe_status_string(99) == b"unknown status"
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    S = moe.Status
+    fake = 1 << 20           # an aligned non-null address that is never dereferenced
+    assert lib.moe_quantize_int4(fake, 4, 256, 64, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_int4(fake, 4, 100, 128, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_int4(None, 4, 256, 128, fake, fake, None) == S.INVALID_ARG
+    assert lib.moe_quantize_int4(fake + 4, 4, 256, 128, fake, fake, None) == S.INVALID_ARG
+    assert lib.moe_quantize_int4(None, 0, 256, 128, None, None, None) == S.OK   # empty: no-op
+    assert lib.moe_quantize_fp8_rows(fake, 7, 4, 16, 4, 1.0, fake, fake, None) == S.INVALID_ARG
+    assert lib.moe_quantize_fp8_rows(fake, 0, 4, 12, 4, 1.0, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_fp8_rows(fake, 0, 4, 16, 5, 1.0, fake, fake, None) == S.INVALID_ARG
+    assert lib.moe_quantize_fp8_rows(fake, 0, 4, 16, 4, 0.0, fake, fake, None) == S.INVALID_ARG
+    assert lib.moe_quantize_fp8_rows(fake, 0, 4, 16, 4, float("nan"), fake, fake, None) == S.INVALID_ARG
+
+
+def test_route_rejects_bad_shapes(lib):
+    S = moe.Status
+    f = 1 << 20
+    args = lambda T, D, E, k: (f, T, D, f, None, E, k, f, f, f, f, f, None)
+    assert lib.moe_route(*args(0, 256, 4, 1)) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_route(*args(8, 200, 4, 1)) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_route(*args(8, 256, 4, 5)) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_route(*args(8, 256, 300, 1)) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_route(*args(8, 256, 16, 9)) == S.UNSUPPORTED_SHAPE
+    a = list(args(8, 256, 4, 1))
+    a[7] = None
+    assert lib.moe_route(*a) == S.INVALID_ARG
+
+
+def _desc(**kw):
+    d = moe.LayerDesc()
+    d.E, d.k, d.D, d.F, d.F_shared = 4, 1, 256, 512, 512
+    d.format, d.group_size, d.path = moe.FMT_INT4, 128, moe.PATH_AUTO
+    f = 1 << 20
+    for name in ("w_router", "w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down",
+                 "ws_gate", "ws_up", "ws_down"):
+        setattr(d, name, f)
+    d.act_scale_ub = float("inf")
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_size_and_layer_checks(lib):
+    d = _desc()
+    n16 = lib.moe_ffn_workspace_size(ctypes.byref(d), 16)
+    n64 = lib.moe_ffn_workspace_size(ctypes.byref(d), 64)
+    assert 0 < n16 < n64 and n16 % 256 == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(D=200)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(k=5)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=64)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(w_up=None)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(d), 0) == 0
+
+
+def test_forward_rejects_small_workspace_and_bad_pointers(lib):
+    S = moe.Status
+    d = _desc()
+    f = 1 << 20
+    need = lib.moe_ffn_workspace_size(ctypes.byref(d), 16)
+    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f, need - 256, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f + 16, need, None) == S.INVALID_ARG  # ws not 256-aligned
+    assert lib.moe_ffn_forward(ctypes.byref(d), None, 16, f, f, need, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward(ctypes.byref(d), f, 0, f, f, need, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_ffn_forward(None, f, 16, f, f, need, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward_host(ctypes.byref(d), f, 16, f, f, need - 256, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_ffn_device_status(None, None) == S.INVALID_ARG
+    ev = (ctypes.c_void_p * 2)(f, f)
+    assert lib.moe_ffn_forward_timed(ctypes.byref(d), f, 16, f, f, need, None, ev, 2) == S.INVALID_ARG
+
+
+def test_launch_names(lib):
+    d = _desc()
+    n = lib.moe_ffn_launch_names(ctypes.byref(d), 16, None, 0)
+    arr = (ctypes.c_char_p * n)()
+    assert lib.moe_ffn_launch_names(ctypes.byref(d), 16, arr, n) == n
+    names = [arr[i].decode() for i in range(n)]
+    assert names[0] == "route_topk" and len(set(names)) == n
+    assert lib.moe_ffn_launch_names(ctypes.byref(_desc(D=100)), 16, None, 0) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        moe.quantize_int4(torch.zeros(2, 128))

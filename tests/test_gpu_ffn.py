@@ -1,0 +1,82 @@
+"""The whole layer on the GPU vs the oracle:
+max |gpu - oracle| <= 1e-2 * max |oracle| (bf16 output, fp32 accumulation)."""
+import numpy as np
+import pytest
+import torch
+
+import int4_quantized_expert_b200 as moe
+import synth
+from oracle import ffn as offn
+from tests._layers import build, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+def _run(b, path=moe.PATH_AUTO, tokens=None):
+    b.gpu.set_path(path)
+    out = b.gpu(b.x.cuda())
+    assert b.gpu.device_status() == moe.Status.OK
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = offn.moe_forward(b.oracle, b.x, tokens=tokens)
+    sel = ref["tokens"]
+    return got[sel], ref["out"]
+
+
+@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_DECODE])
+def test_tiny(path):
+    b = build(synth.SHAPES["tiny"])
+    got, ref = _run(b, path)
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("T,D,F,Fs,E,k", [
+    (1, 256, 512, 512, 4, 1),        # one token
+    (37, 384, 640, 384, 5, 2),       # ragged: 3 groups along D, 2 token chunks + 5
+    (16, 128, 256, 128, 1, 1),       # a single expert
+    (50, 256, 384, 256, 6, 3),
+    (16, 512, 1024, 768, 16, 1),
+])
+def test_ragged_decode(T, D, F, Fs, E, k):
+    b = build(synth.LayerShape("r", T, D, F, E, k, Fs))
+    got, ref = _run(b, moe.PATH_DECODE)
+    assert rel_err(got, ref) <= TOL
+
+
+def test_all_tokens_on_one_expert_and_empty_experts():
+    shape = synth.LayerShape("one", 40, 256, 512, 4, 1, 256)
+    b = build(shape, margin=False)
+    wr = torch.zeros(4, 256, dtype=torch.bfloat16)
+    wr[2] = 0.02
+    b.gpu.tensors[0].copy_(wr.cuda())
+    b.oracle.w_router = wr
+    b.x = torch.ones(40, 256, dtype=torch.bfloat16) * torch.linspace(0.5, 1.5, 40).to(torch.bfloat16)[:, None]
+    got, ref = _run(b, moe.PATH_DECODE)
+    assert rel_err(got, ref) <= TOL
+
+
+def test_repeat_calls_identical():
+    b = build(synth.SHAPES["tiny"])
+    o1 = b.gpu(b.x.cuda()).clone()
+    o2 = b.gpu(b.x.cuda())
+    assert torch.equal(o1, o2)
+
+
+def test_host_buffers_match_device_call():
+    b = build(synth.SHAPES["tiny"])
+    dev = b.gpu(b.x.cuda()).cpu()
+    xh = b.x.clone().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    b.gpu.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, dev)
+
+
+@pytest.mark.slow
+def test_scout_decode_full_size():
+    """The decode workload at full size (T=16, D=5120, F=8192, 16 experts),
+    every token checked against the oracle."""
+    b = build(synth.SHAPES["scout_decode"])
+    got, ref = _run(b)
+    assert rel_err(got, ref) <= TOL

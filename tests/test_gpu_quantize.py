@@ -1,0 +1,74 @@
+"""GPU quantizers vs the oracle: int4 codes/scales and e4m3 bytes/scales must be
+bit-exact (both sides take every rounding decision in fp32)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import int4_quantized_expert_b200 as moe
+import synth
+from oracle import quant as oq
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (3, 384), (37, 512), (256, 5120), (130, 8192)])
+def test_int4_bit_exact(rows, cols):
+    g = synth.stream(11, rows * 7 + cols)
+    w = (g.standard_normal((rows, cols), dtype=np.float32) * np.float32(0.02))
+    w[0, :128] = 0.0                                      # all-zero group
+    if rows > 2:
+        w[1, :128] = np.linspace(-1, 1, 128, dtype=np.float32)   # exact .5 quotients
+        w[2, 5] = 1e4                                     # one huge value
+    codes, scales = moe.quantize_int4(torch.from_numpy(w).cuda())
+    q_ref, s_ref = oq.int4_row_quantize(w)
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy(), oq.pack_int4(q_ref))
+
+
+def test_int4_worked_group_on_gpu():
+    group = np.zeros((1, 128), np.float32)
+    group[0, :6] = [0.3125, 0.4375, -0.0625, 1.0, -1.0, 0.1875]
+    codes, scales = moe.quantize_int4(torch.from_numpy(group).cuda())
+    q = oq.unpack_int4(codes.cpu().numpy())
+    assert q[0, :6].tolist() == [2, 4, 0, 7, -8, 2] and scales.item() == 0.125
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rows,cols,nv,ub", [(1, 8, 1, math.inf), (33, 5120, 30, math.inf),
+                                               (64, 8192, 64, 2.0), (5, 40, 3, 0.5)])
+def test_fp8_rows_bit_exact(dtype, rows, cols, nv, ub):
+    g = synth.stream(12, rows * 3 + cols)
+    x = g.standard_normal((rows, cols), dtype=np.float32) * np.float32(3.0)
+    x[0, :4] = [0.0, -1e-9, 1e-30, -0.0]              # signed zero and underflow
+    xt = torch.from_numpy(x).to(dtype)
+    q, s = moe.quantize_fp8_rows(xt.cuda(), num_valid_rows=nv, scale_ub=ub)
+    q_ref, s_ref = oq.fp8_row_quantize(xt.float().numpy(), num_valid_rows=nv, scale_ub=ub)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.slow
+def test_int4_full_size_sampled_experts():
+    """int4_row_quantize of a 16-expert Scout-shaped layer at full size (one
+    launch over all 2.01 G weights, as timed standalone), checked on sampled
+    experts' down projections and gate rows."""
+    shape = synth.SHAPES["skewed"]
+    E, D, F = shape.E, shape.D, shape.F
+    w = torch.empty(E * 3, F * D, dtype=torch.float32, device="cuda")   # 8.05 GB
+    for e, g, u, d in synth.iter_expert_weights(0, range(E), D, F):
+        w[3 * e].copy_(torch.from_numpy(g).view(-1))
+        w[3 * e + 1].copy_(torch.from_numpy(u).view(-1))
+        w[3 * e + 2].copy_(torch.from_numpy(d).view(-1))
+    rows = E * 3 * F          # gate/up rows have K = D; down rows K = F differ, so view by [rows, D]
+    codes, scales = moe.quantize_int4(w.view(-1, D))
+    del w
+    for e in (0, 7, 15):
+        g, u, d = synth.expert_weights(0, e, D, F)
+        for which, mat in ((0, g), (2, d)):
+            q_ref, s_ref = oq.int4_row_quantize(mat.reshape(-1, D))
+            n = mat.size // D
+            base = (3 * e + which) * n
+            assert np.array_equal(scales[base:base + n].cpu().numpy(), s_ref)
+            assert np.array_equal(codes[base:base + n].cpu().numpy(), oq.pack_int4(q_ref))
