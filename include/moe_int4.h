@@ -215,6 +215,30 @@ MOE_API int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, con
                                      int32_t max_names);
 
 /*
+ * moe_ffn_forward_noalloc -- the layer forward of moe_ffn_forward, for
+ * callers that cannot allocate device memory and so cannot pass a workspace:
+ * for example a plugin behind a fixed interface that hands over only its
+ * input and output buffers, or a runtime that has reserved all device memory
+ * for its own pool, where an extra cudaMalloc would fail or would stall the
+ * device.  The web pages have no counterpart; this is an interface
+ * convenience only.
+ *   x    device, bf16 [T, D];  out  device, bf16 [T, D]
+ * The library's own scratch is a fixed 8 MiB device array, reserved on every
+ * device that loads the library until the process exits.  A call whose
+ * scratch need (moe_ffn_workspace_size(layer, T)) exceeds 8 MiB returns
+ * MOE_ERR_WORKSPACE_TOO_SMALL and launches nothing; use moe_ffn_forward then.
+ * No cudaMalloc, cudaFree or other allocation is made.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls on a device share the one array: calls that may overlap on the
+ * GPU (different streams, or different host threads) race and corrupt each
+ * other's results -- serialize them.  Leftover contents from an earlier call
+ * are harmless; what must start at zero is cleared by every call.
+ */
+MOE_API moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
+                                           void* stream);
+
+/*
  * moe_ffn_device_status -- SYNCHRONIZES `stream`, then reads the device
  * status word that the kernels of the last moe_ffn_forward on this workspace
  * set.  Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait gave up; the

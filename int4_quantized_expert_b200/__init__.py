@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_forward_timed.restype = ctypes.c_int
         L.moe_ffn_launch_names.argtypes = [ctypes.POINTER(LayerDesc), i32, ctypes.POINTER(ctypes.c_char_p), i32]
         L.moe_ffn_launch_names.restype = i32
+        L.moe_ffn_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp]
+        L.moe_ffn_forward_noalloc.restype = ctypes.c_int
         L.moe_ffn_device_status.argtypes = [vp, vp]
         L.moe_ffn_device_status.restype = ctypes.c_int
         _lib = L

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "ffn_decode.cuh"
 
@@ -329,3 +331,54 @@ moe_status moe_ffn_device_status(const void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Layer forward without caller-provided scratch.
+//
+// The scratch lives in one file-scope device array of kNoAllocScratchBytes.
+// Every device that loads this library reserves it for the life of the
+// process, so it is kept small: it covers the layer's intermediate buffers for
+// decode-sized batches only.  Host code cannot use the array's name as a
+// device address (it names a host-side shadow), so the first call on each
+// device asks the runtime for the real address, with that device current,
+// and remembers it.  Calls share the array and it keeps whatever the previous
+// call left; the layer path already clears what must start at zero (the
+// device status word and the task counters) on every call.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+moe_status noalloc_scratch_address(void** addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
+                                              void* stream) {
+    moe_status s = check_layer(layer);
+    if (s != MOE_OK) return s;
+    s = check_route_shape(T, layer->D, layer->E, layer->k);
+    if (s != MOE_OK) return s;
+    if (ws_layout(*layer, T).total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    void* scratch = nullptr;
+    s = noalloc_scratch_address(&scratch);
+    if (s != MOE_OK) return s;
+    return ffn_forward_impl(layer, x, T, out, scratch, kNoAllocScratchBytes, as_stream(stream));
+}
