@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "moe_int4.h"
@@ -27,9 +28,11 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // ---------------------------------------------------------------------------
 // Read-only global loads that do not allocate in L1 (weights are streamed once)
 // ---------------------------------------------------------------------------
+// (Not volatile: they read memory no thread of the kernel writes, so the
+// compiler may schedule them freely.)
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
@@ -37,14 +40,14 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // Read-only global load that may be cached in L1 (small operands reused by many warps)
 __device__ __forceinline__ uint4 ldg_cached(const void* p) {
     uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
 
 __device__ __forceinline__ float ldg_f32(const float* p) {
     float v;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    asm("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
 
@@ -89,12 +92,33 @@ __device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t w_xor88) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+
+// The same shape with fp16 inputs: d = a * b + c (c separate from d).
+__device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1, float c0, float c1, float c2, float c3) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    mma_f16_16816(d, a0, a1, a2, a3, b0, b1, d[0], d[1], d[2], d[3]);
+}
+
+// int4 codes -> exact fp16 integers, two per instruction.  0x6400 is 1024.0
+// in fp16, whose mantissa step is 1; a nibble placed in mantissa bits 0..3
+// with its top bit flipped (two's-complement q -> q + 8) reads 1032 + q, and
+// one in bits 4..7 reads 1024 + 16 (q + 8) = 1152 + 16 q.
+__device__ __forceinline__ uint32_t f16_lo_nibbles(uint32_t w) { return (w & 0x000F000Fu) ^ 0x64086408u; }
+__device__ __forceinline__ uint32_t f16_hi_nibbles(uint32_t w) { return (w & 0x00F000F0u) ^ 0x64806480u; }
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
@@ -146,11 +170,15 @@ __device__ __forceinline__ int32_t ld_volatile(const int32_t* p) {
 
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // at once if another wait of this launch already timed out (status set).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+// With backoff_ns > 0 the thread sleeps between polls, leaving the issue
+// slots of its SM sub-partition to the warps doing the arithmetic.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
+                                          uint32_t backoff_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     if (status && ld_volatile(status) != DEV_OK) return false;
     const long long t0 = clock64();
     for (uint32_t i = 1;; ++i) {
+        if (backoff_ns) __nanosleep(backoff_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 1023u) == 0 && status && ld_volatile(status) != DEV_OK) return false;
         if (clock64() - t0 > kWaitCycles) {

@@ -34,7 +34,13 @@ namespace moe {
 constexpr int DC_ROWS = 32;                 // output rows per task
 constexpr int DC_KPH = 4;                   // K phases
 constexpr int DC_CONSUMERS = 8;             // 2 row blocks x 4 K phases
-constexpr int DC_THREADS = (DC_CONSUMERS + 1) * 32;
+// Three warpgroups: warpgroup 0 holds the producer (warp 0, one thread) and
+// gives most of its registers to warpgroups 1 and 2, the 8 consumer warps:
+// 128 x 40 + 256 x 232 = 384 x 168, the registers the block launches with.
+constexpr int DC_THREADS = 384;
+constexpr int DC_PRODUCER_REGS = 40;
+constexpr int DC_CONSUMER_REGS = 232;
+static_assert(128 * DC_PRODUCER_REGS + 256 * DC_CONSUMER_REGS <= DC_THREADS * 168, "register split");
 constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 32 rows x 128 B
 constexpr int DC_STAGE = 2 * DC_CHUNK;      // 8 KB
 constexpr int DC_NSTAGES = 16;              // ring: 128 KB in flight
@@ -73,8 +79,150 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
     return tile + r * 128 + ((j ^ (r & 7)) << 4);
 }
 
+
 // position of element i (0..7) of an 8-block in the x0 x4 x1 x5 x2 x6 x3 x7 layout
 __device__ __forceinline__ int frag_pos8(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
+
+// The int4 part of a decode task: the warp's stages q, q + 4, ... of groups
+// of 128 K, NT token tiles.  Returns false if a wait timed out.
+//
+// Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
+// shift and four LOP3s give (k0,k4) and (k2,k6) as 1032 + q and (k1,k5),
+// (k3,k7) as 1152 + 16 q.  The B rows (fp16 tokens, scaled per row by a power
+// of two) store odd positions divided by 16 and every 8-block in the order
+// x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x plus a per-group
+// offset that the partial sum starts from (negc, passed as the MMA's C).
+// Token rows that do not exist point at a zero row, so every load is
+// unconditional; the fragments of the next group are loaded one group ahead.
+template <int MODE, int NT>
+__device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
+                                             const float* sc, uint32_t it_base, int q, int lane, int row_a,
+                                             int row_b, const bf16* const (&brow)[DC_NT],
+                                             const float* const (&crow)[DC_NT][2], float (&acc0)[DC_NT][4],
+                                             float (&acc1)[DC_NT][4], int32_t* status) {
+    constexpr int GPS = MODE == 0 ? 2 : 4;   // groups per stage
+    const int c = lane & 3;
+    const int ng = ti.K / kGroup;
+    // byte offsets of this thread's 16-byte chunks in a swizzled 32 x 128 B tile:
+    // chunk 4 gi + c of rows row_a and row_b, for the tile's two groups gi
+    uint32_t off_a[2], off_b[2];
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+        off_a[gi] = row_a * 128 + (((4 * gi + c) ^ (row_a & 7)) << 4);
+        off_b[gi] = row_b * 128 + (((4 * gi + c) ^ (row_b & 7)) << 4);
+    }
+    const float* sga_p = sc + row_a * ng;
+    const float* sgb_p = sc + row_b * ng;
+    const float* sua_p = sc + (DC_ROWS + row_a) * ng;
+    const float* sub_p = sc + (DC_ROWS + row_b) * ng;
+    const bf16* xp[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) xp[nt] = brow[nt] + 32 * c;
+
+    uint4 xA[NT][4], xB[NT][4];
+    float cA[NT][2], cB[NT][2];
+    auto load = [&](int G, uint4 (&xv)[NT][4], float (&cv)[NT][2]) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[nt][i] = ldg_cached(xp[nt] + G * kGroup + 8 * i);
+            cv[nt][0] = ldg_f32(crow[nt][0] + G);
+            cv[nt][1] = ldg_f32(crow[nt][1] + G);
+        }
+    };
+    auto group = [&](const unsigned char* st, int G, int gi, const unsigned char* tile, int Gn,
+                     uint4 (&xc)[NT][4], float (&cc)[NT][2], uint4 (&xn)[NT][4], float (&cn)[NT][2]) {
+        load(Gn, xn, cn);   // Gn is clamped to a valid group; a final redundant load is harmless
+        const uint4 wa = lds128(tile + off_a[gi]);
+        const uint4 wb = lds128(tile + off_b[gi]);
+        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
+        if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
+        const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
+        const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
+        // two accumulation chains per matrix (even / odd words); the even one
+        // starts from the group offset, the odd one from zero
+        float pg[2][NT][4], pu[2][NT][4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
+            const uint32_t ea0 = f16_lo_nibbles(WA[jj]), ea1 = f16_lo_nibbles(WB[jj]);
+            const uint32_t ea2 = f16_lo_nibbles(wa8), ea3 = f16_lo_nibbles(wb8);
+            const uint32_t oa0 = f16_hi_nibbles(WA[jj]), oa1 = f16_hi_nibbles(WB[jj]);
+            const uint32_t oa2 = f16_hi_nibbles(wa8), oa3 = f16_hi_nibbles(wb8);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float* d = pg[jj & 1][nt];
+                if (jj == 0) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y,
+                                           cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
+                else if (jj == 1) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
+                else mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y);
+                mma_f16_16816(d, oa0, oa1, oa2, oa3, xc[nt][jj].z, xc[nt][jj].w);
+            }
+            if (MODE == 0) {
+                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                const uint32_t eu0 = f16_lo_nibbles(VA[jj]), eu1 = f16_lo_nibbles(VB[jj]);
+                const uint32_t eu2 = f16_lo_nibbles(va8), eu3 = f16_lo_nibbles(vb8);
+                const uint32_t ou0 = f16_hi_nibbles(VA[jj]), ou1 = f16_hi_nibbles(VB[jj]);
+                const uint32_t ou2 = f16_hi_nibbles(va8), ou3 = f16_hi_nibbles(vb8);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float* d = pu[jj & 1][nt];
+                    if (jj == 0) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y,
+                                               cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
+                    else if (jj == 1) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
+                    else mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y);
+                    mma_f16_16816(d, ou0, ou1, ou2, ou3, xc[nt][jj].z, xc[nt][jj].w);
+                }
+            }
+        }
+        const float sga = sga_p[G], sgb = sgb_p[G];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            acc0[nt][0] = fmaf(pg[0][nt][0] + pg[1][nt][0], sga, acc0[nt][0]);
+            acc0[nt][1] = fmaf(pg[0][nt][1] + pg[1][nt][1], sga, acc0[nt][1]);
+            acc0[nt][2] = fmaf(pg[0][nt][2] + pg[1][nt][2], sgb, acc0[nt][2]);
+            acc0[nt][3] = fmaf(pg[0][nt][3] + pg[1][nt][3], sgb, acc0[nt][3]);
+        }
+        if (MODE == 0) {
+            const float sua = sua_p[G], sub = sub_p[G];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                acc1[nt][0] = fmaf(pu[0][nt][0] + pu[1][nt][0], sua, acc1[nt][0]);
+                acc1[nt][1] = fmaf(pu[0][nt][1] + pu[1][nt][1], sua, acc1[nt][1]);
+                acc1[nt][2] = fmaf(pu[0][nt][2] + pu[1][nt][2], sub, acc1[nt][2]);
+                acc1[nt][3] = fmaf(pu[0][nt][3] + pu[1][nt][3], sub, acc1[nt][3]);
+            }
+        }
+    };
+
+    bool ok = true;
+    if (q < ti.n_stages) load(q * GPS, xA, cA);
+    for (int s = q; s < ti.n_stages; s += DC_KPH) {
+        const uint32_t it = it_base + s;
+        const uint32_t slot = it % DC_NSTAGES;
+        if (!mbar_wait(&sm->full[slot], (it / DC_NSTAGES) & 1, status)) { ok = false; break; }
+        const unsigned char* st = ring + slot * DC_STAGE;
+        const int G0 = s * GPS;
+        const int g_next_stage = min((s + DC_KPH) * GPS, ng - 1);
+        // groups alternate between the A and B fragment buffers; a stage holds
+        // an even number of groups, so every stage starts on A
+#pragma unroll
+        for (int gl = 0; gl < GPS; gl += 2) {
+            if (G0 + gl >= ng) break;
+            // MODE 0: both groups in tile 0 (gate) and tile 1 (up);
+            // MODE 1: groups 0,1 in tile 0 and 2,3 in tile 1 of the one matrix
+            const unsigned char* tile = st + (MODE == 0 ? 0 : (gl >> 1) * DC_CHUNK);
+            group(st, G0 + gl, 0, tile, (gl + 1 < GPS) ? min(G0 + gl + 1, ng - 1) : g_next_stage,
+                  xA, cA, xB, cB);
+            if (G0 + gl + 1 >= ng) break;
+            group(st, G0 + gl + 1, 1, tile, (gl + 2 < GPS) ? min(G0 + gl + 2, ng - 1) : g_next_stage,
+                  xB, cB, xA, cA);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->empty[slot]);
+    }
+    return ok;
+}
 
 template <int MODE>   // 0 = gate/up with SwiGLU, 1 = down
 __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
@@ -104,16 +252,17 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const int n_chunks = *p.n_chunks, n_sh = *p.n_shared_chunks;
     const int n_tasks = n_sh * nbs + (n_chunks - n_sh) * nbr;
 
-    if (warp == DC_CONSUMERS) {
+    if (warp < 4) {
         // ------------------------------ producer ------------------------------
-        if (lane == 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(DC_PRODUCER_REGS));
+        if (warp == 0 && lane == 0) {
             prefetch_tmap(&tm_r0); prefetch_tmap(&tm_r1); prefetch_tmap(&tm_s0); prefetch_tmap(&tm_s1);
             uint32_t it = 0;
             bool ok = true;
             for (uint32_t tn = 0; ok; ++tn) {
                 const int t = atomicAdd(p.task_counter, 1);
                 const int b = tn & 1;
-                if (!mbar_wait(&sm->sempty[b], ((tn >> 1) & 1) ^ 1, p.status)) break;
+                if (!mbar_wait(&sm->sempty[b], ((tn >> 1) & 1) ^ 1, p.status, 128)) break;
                 TaskInfo ti;
                 ti.pad = 0;
                 if (t >= n_tasks) {
@@ -151,7 +300,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const int kbytes = ti.kind ? 128 : 64;   // tile x extent in elements (uint8 codes / bf16)
                 for (int s = 0; s < ti.n_stages; ++s, ++it) {
                     const uint32_t slot = it % DC_NSTAGES;
-                    if (!mbar_wait(&sm->empty[slot], ((it / DC_NSTAGES) & 1) ^ 1, p.status)) { ok = false; break; }
+                    if (!mbar_wait(&sm->empty[slot], ((it / DC_NSTAGES) & 1) ^ 1, p.status, 128)) { ok = false; break; }
                     unsigned char* st = ring + slot * DC_STAGE;
                     if (MODE == 0) {
                         mbar_arrive_expect_tx(&sm->full[slot], DC_STAGE);
@@ -176,7 +325,9 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     }
 
     // ------------------------------ consumers ------------------------------
-    const int rb = warp & 1, q = warp >> 1;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(DC_CONSUMER_REGS));
+    const int ci = warp - 4;
+    const int rb = ci & 1, q = ci >> 1;
     const int g = lane >> 2, c = lane & 3;
     const int row_a = 16 * rb + sigma8(g), row_b = row_a + 8;
     uint32_t it_base = 0;
@@ -188,16 +339,32 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         const float* sc = sbuf + b * p.scale_buf_floats;
         const int ng = ti.K / kGroup;
 
-        // token rows of this chunk for the two n-tiles (column n = g of each)
+        // B rows (tokens) of this chunk for the two n-tiles: column n = g of each
+        // (16-bit elements: bf16 for the shared expert, fp16 for routed ones).
+        // Routed tasks also need, for the C columns 2c and 2c + 1, the group
+        // offsets (negc) and the rows' power-of-two scales.
         const bf16* brow[DC_NT];
+        const float* crow[DC_NT][2];
+        float cscale[DC_NT][2];
 #pragma unroll
         for (int nt = 0; nt < DC_NT; ++nt) {
             const int i = nt * 8 + g;
-            brow[nt] = nullptr;
+            brow[nt] = p.zero_row;          // tokens beyond the chunk read zeros
             if (i < ti.count) {
                 if (ti.kind == 0) brow[nt] = p.b_s + int64_t(ti.start + i) * p.ldb_s;
                 else if (MODE == 0) brow[nt] = p.b_r + int64_t(p.perm[ti.start + i] / p.k_top) * p.ldb_r;
                 else brow[nt] = p.b_r + int64_t(ti.start + i) * p.ldb_r;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int ic = nt * 8 + 2 * c + h;
+                crow[nt][h] = p.zero_corr;
+                cscale[nt][h] = 1.0f;
+                if (ti.kind == 1 && ic < ti.count) {
+                    const int64_t row = MODE == 0 ? int64_t(p.perm[ti.start + ic] / p.k_top) : int64_t(ti.start + ic);
+                    crow[nt][h] = p.corr_r + row * ng;
+                    cscale[nt][h] = p.rscale_r[row];
+                }
             }
         }
         const int nt_used = ti.count > 8 ? 2 : 1;
@@ -209,117 +376,48 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             for (int r = 0; r < 4; ++r) { acc0[nt][r] = 0.f; acc1[nt][r] = 0.f; }
 
         bool ok = true;
-        for (int s = q; s < ti.n_stages; s += DC_KPH) {
-            const uint32_t it = it_base + s;
-            const uint32_t slot = it % DC_NSTAGES;
-            if (!mbar_wait(&sm->full[slot], (it / DC_NSTAGES) & 1, p.status)) { ok = false; break; }
-            const unsigned char* st = ring + slot * DC_STAGE;
+        if (ti.kind == 1) {
+            ok = nt_used == 1
+                     ? consume_int4<MODE, 1>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
+                                             p.status)
+                     : consume_int4<MODE, 2>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
+                                             p.status);
+        } else {
+            // ---------------- bf16 weights (shared expert): 64 K per tile ----------------
+            // thread c takes the 8-blocks c and c + 4 of each 64-K tile
+            constexpr int UPS = MODE == 0 ? 1 : 2;           // 64-K units per stage
+            const int n_units = ti.K / 64;
+            uint4 xc[DC_NT][2], xn[DC_NT][2];
+            auto load = [&](int U, uint4 (&xv)[DC_NT][2]) {
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                // MODE 0: tile 0 = gate, tile 1 = up, same K.  MODE 1: two K tiles of one matrix.
-                if (MODE == 1 && ch == 1 && (2 * s + 1) * (ti.kind ? 256 : 64) >= ti.K) break;
-                if (MODE == 0 && ch == 1) break;   // handled together with tile 0 below
-                const unsigned char* t0 = st + ch * DC_CHUNK;
-                const unsigned char* t1 = st + DC_CHUNK;
-                if (ti.kind == 1) {
-                    // ---- int4: 2 groups of 128 K per tile ----
+                for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi) {
-                        const int G = (MODE == 0 ? s * 2 : (2 * s + ch) * 2) + gi;
-                        if (G >= ng) break;
-                        const int j = 4 * gi + c;
-                        const uint4 wa = lds128(swz(t0, row_a, j));
-                        const uint4 wb = lds128(swz(t0, row_b, j));
-                        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-                        if (MODE == 0) { va = lds128(swz(t1, row_a, j)); vb = lds128(swz(t1, row_b, j)); }
-                        uint4 xb[DC_NT][4];
+                    for (int h2 = 0; h2 < 2; ++h2)
+                        xv[nt][h2] = (nt < nt_used && brow[nt]) ? ldg_cached(brow[nt] + U * 64 + 8 * (c + 4 * h2))
+                                                                : make_uint4(0, 0, 0, 0);
+            };
+            if (q < ti.n_stages) load(q * UPS, xc);
+            for (int s = q; s < ti.n_stages; s += DC_KPH) {
+                const uint32_t it = it_base + s;
+                const uint32_t slot = it % DC_NSTAGES;
+                if (!mbar_wait(&sm->full[slot], (it / DC_NSTAGES) & 1, p.status)) { ok = false; break; }
+                const unsigned char* st = ring + slot * DC_STAGE;
 #pragma unroll
-                        for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                xb[nt][i] = (nt < nt_used && brow[nt])
-                                                ? ldg_cached(brow[nt] + G * kGroup + 32 * c + 8 * i)
-                                                : make_uint4(0, 0, 0, 0);
-                        float pg[DC_NT][4], pu[DC_NT][4];
-#pragma unroll
-                        for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                            for (int r = 0; r < 4; ++r) { pg[nt][r] = 0.f; pu[nt][r] = 0.f; }
-                        const uint32_t WA[4] = {wa.x ^ 0x88888888u, wa.y ^ 0x88888888u, wa.z ^ 0x88888888u, wa.w ^ 0x88888888u};
-                        const uint32_t WB[4] = {wb.x ^ 0x88888888u, wb.y ^ 0x88888888u, wb.z ^ 0x88888888u, wb.w ^ 0x88888888u};
-                        const uint32_t VA[4] = {va.x ^ 0x88888888u, va.y ^ 0x88888888u, va.z ^ 0x88888888u, va.w ^ 0x88888888u};
-                        const uint32_t VB[4] = {vb.x ^ 0x88888888u, vb.y ^ 0x88888888u, vb.z ^ 0x88888888u, vb.w ^ 0x88888888u};
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                uint32_t a0, a1, a2, a3;
-                                if (h == 0) {
-                                    a0 = int4x2_to_bf16x2<0>(WA[jj]); a2 = int4x2_to_bf16x2<4>(WA[jj]);
-                                    a1 = int4x2_to_bf16x2<0>(WB[jj]); a3 = int4x2_to_bf16x2<4>(WB[jj]);
-                                } else {
-                                    a0 = int4x2_to_bf16x2<8>(WA[jj]); a2 = int4x2_to_bf16x2<12>(WA[jj]);
-                                    a1 = int4x2_to_bf16x2<8>(WB[jj]); a3 = int4x2_to_bf16x2<12>(WB[jj]);
-                                }
-#pragma unroll
-                                for (int nt = 0; nt < DC_NT; ++nt) {
-                                    if (nt >= nt_used) break;
-                                    const uint32_t b0 = h == 0 ? xb[nt][jj].x : xb[nt][jj].z;
-                                    const uint32_t b1 = h == 0 ? xb[nt][jj].y : xb[nt][jj].w;
-                                    mma_bf16_16816(pg[nt], a0, a1, a2, a3, b0, b1);
-                                }
-                                if (MODE == 0) {
-                                    uint32_t u0, u1, u2, u3;
-                                    if (h == 0) {
-                                        u0 = int4x2_to_bf16x2<0>(VA[jj]); u2 = int4x2_to_bf16x2<4>(VA[jj]);
-                                        u1 = int4x2_to_bf16x2<0>(VB[jj]); u3 = int4x2_to_bf16x2<4>(VB[jj]);
-                                    } else {
-                                        u0 = int4x2_to_bf16x2<8>(VA[jj]); u2 = int4x2_to_bf16x2<12>(VA[jj]);
-                                        u1 = int4x2_to_bf16x2<8>(VB[jj]); u3 = int4x2_to_bf16x2<12>(VB[jj]);
-                                    }
-#pragma unroll
-                                    for (int nt = 0; nt < DC_NT; ++nt) {
-                                        if (nt >= nt_used) break;
-                                        const uint32_t b0 = h == 0 ? xb[nt][jj].x : xb[nt][jj].z;
-                                        const uint32_t b1 = h == 0 ? xb[nt][jj].y : xb[nt][jj].w;
-                                        mma_bf16_16816(pu[nt], u0, u1, u2, u3, b0, b1);
-                                    }
-                                }
-                            }
-                        }
-                        // group scales of rows row_a / row_b
-                        const float sga = sc[row_a * ng + G], sgb = sc[row_b * ng + G];
-                        float sua = 0.f, sub = 0.f;
-                        if (MODE == 0) { sua = sc[(DC_ROWS + row_a) * ng + G]; sub = sc[(DC_ROWS + row_b) * ng + G]; }
-#pragma unroll
-                        for (int nt = 0; nt < DC_NT; ++nt) {
-                            acc0[nt][0] = fmaf(pg[nt][0], sga, acc0[nt][0]);
-                            acc0[nt][1] = fmaf(pg[nt][1], sga, acc0[nt][1]);
-                            acc0[nt][2] = fmaf(pg[nt][2], sgb, acc0[nt][2]);
-                            acc0[nt][3] = fmaf(pg[nt][3], sgb, acc0[nt][3]);
-                            if (MODE == 0) {
-                                acc1[nt][0] = fmaf(pu[nt][0], sua, acc1[nt][0]);
-                                acc1[nt][1] = fmaf(pu[nt][1], sua, acc1[nt][1]);
-                                acc1[nt][2] = fmaf(pu[nt][2], sub, acc1[nt][2]);
-                                acc1[nt][3] = fmaf(pu[nt][3], sub, acc1[nt][3]);
-                            }
-                        }
-                    }
-                } else {
-                    // ---- bf16 (shared expert): 64 K per tile; thread c takes 8-blocks c and c + 4 ----
-                    const int kt = MODE == 0 ? s * 64 : (2 * s + ch) * 64;
+                for (int ul = 0; ul < UPS; ++ul) {
+                    const int U = s * UPS + ul;
+                    if (U >= n_units) break;
+                    int Un = -1;
+                    if (ul + 1 < UPS) Un = U + 1;
+                    else if (s + DC_KPH < ti.n_stages) Un = (s + DC_KPH) * UPS;
+                    if (Un >= 0 && Un < n_units) load(Un, xn);
+                    const unsigned char* ta = st + (MODE == 0 ? 0 : ul * DC_CHUNK);
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int j = c + 4 * h2;
-                        const uint4 wa = lds128(swz(t0, row_a, j));
-                        const uint4 wb = lds128(swz(t0, row_b, j));
+                        const uint4 wa = lds128(swz(ta, row_a, j));
+                        const uint4 wb = lds128(swz(ta, row_b, j));
                         uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-                        if (MODE == 0) { va = lds128(swz(t1, row_a, j)); vb = lds128(swz(t1, row_b, j)); }
-                        uint4 xb[DC_NT];
-#pragma unroll
-                        for (int nt = 0; nt < DC_NT; ++nt)
-                            xb[nt] = (nt < nt_used && brow[nt]) ? ldg_cached(brow[nt] + kt + 8 * j)
-                                                                : make_uint4(0, 0, 0, 0);
+                        if (MODE == 0) { va = lds128(swz(st + DC_CHUNK, row_a, j)); vb = lds128(swz(st + DC_CHUNK, row_b, j)); }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const uint32_t a0 = h == 0 ? prmt(wa.x, wa.z, 0x5410) : prmt(wa.y, wa.w, 0x5410);
@@ -329,8 +427,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 #pragma unroll
                             for (int nt = 0; nt < DC_NT; ++nt) {
                                 if (nt >= nt_used) break;
-                                const uint32_t b0 = h == 0 ? xb[nt].x : xb[nt].z;
-                                const uint32_t b1 = h == 0 ? xb[nt].y : xb[nt].w;
+                                const uint32_t b0 = h == 0 ? xc[nt][h2].x : xc[nt][h2].z;
+                                const uint32_t b1 = h == 0 ? xc[nt][h2].y : xc[nt][h2].w;
                                 mma_bf16_16816(acc0[nt], a0, a1, a2, a3, b0, b1);
                             }
                             if (MODE == 0) {
@@ -341,17 +439,21 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 #pragma unroll
                                 for (int nt = 0; nt < DC_NT; ++nt) {
                                     if (nt >= nt_used) break;
-                                    const uint32_t b0 = h == 0 ? xb[nt].x : xb[nt].z;
-                                    const uint32_t b1 = h == 0 ? xb[nt].y : xb[nt].w;
+                                    const uint32_t b0 = h == 0 ? xc[nt][h2].x : xc[nt][h2].z;
+                                    const uint32_t b1 = h == 0 ? xc[nt][h2].y : xc[nt][h2].w;
                                     mma_bf16_16816(acc1[nt], u0, u1, u2, u3, b0, b1);
                                 }
                             }
                         }
                     }
+#pragma unroll
+                    for (int nt = 0; nt < DC_NT; ++nt)
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) xc[nt][h2] = xn[nt][h2];
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->empty[slot]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->empty[slot]);
         }
         if (!ok) break;
 
@@ -376,6 +478,9 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     for (int r = 0; r < 4; ++r) { acc0[nt][r] += o[nt * 8 + r]; acc1[nt][r] += o[nt * 8 + 4 + r]; }
             }
             // ---- epilogue: C rows (row_a, row_b) x token columns (2c, 2c + 1) of each n-tile ----
+            // routed results are rescaled by their B row's power of two;
+            // routed h is stored in natural order (its fp16 copy is made next),
+            // the shared expert's h in the bf16 fragment order it is read in
 #pragma unroll
             for (int nt = 0; nt < DC_NT; ++nt) {
 #pragma unroll
@@ -383,15 +488,20 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     const int col = nt * 8 + 2 * c + (r & 1);
                     if (col >= ti.count) continue;
                     const int n = ti.row0 + (r < 2 ? row_a : row_b);
+                    const float cs = cscale[nt][r & 1];
                     if (MODE == 0) {
-                        const float hv = silu_f32(acc0[nt][r]) * acc1[nt][r];
-                        const int pos = (n & ~7) + frag_pos8(n & 7);
-                        if (ti.kind == 1) p.h_r[int64_t(ti.start + col) * p.n_rows_r + pos] = __float2bfloat16_rn(hv);
-                        else p.h_s[int64_t(ti.start + col) * p.n_rows_s + pos] = __float2bfloat16_rn(hv);
+                        if (ti.kind == 1) {
+                            const float hv = silu_f32(acc0[nt][r] * cs) * (acc1[nt][r] * cs);
+                            p.h_r[int64_t(ti.start + col) * p.n_rows_r + n] = __float2bfloat16_rn(hv);
+                        } else {
+                            const float hv = silu_f32(acc0[nt][r]) * acc1[nt][r];
+                            const int pos = (n & ~7) + frag_pos8(n & 7);
+                            p.h_s[int64_t(ti.start + col) * p.n_rows_s + pos] = __float2bfloat16_rn(hv);
+                        }
                     } else {
                         if (ti.kind == 1) {
                             const int pp = ti.start + col;
-                            p.y_r[int64_t(pp) * p.n_rows_r + n] = acc0[nt][r] * p.gates[p.perm[pp]];
+                            p.y_r[int64_t(pp) * p.n_rows_r + n] = acc0[nt][r] * cs * p.gates[p.perm[pp]];
                         } else {
                             p.y_s[int64_t(ti.start + col) * p.n_rows_s + n] = acc0[nt][r];
                         }
@@ -425,29 +535,6 @@ __global__ void combine_kernel(const float* __restrict__ y_s, const float* __res
         o.y = pack_bf16x2(a.z, a.w);
         *reinterpret_cast<uint2*>(out + t * D + d) = o;
     }
-}
-
-// One thread: the decode task list (token chunks of <= 16): the shared
-// expert's chunks first, then each routed expert's.
-__global__ void decode_plan_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
-                                   int T, int E, ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks,
-                                   int32_t* __restrict__ n_shared, int32_t* __restrict__ counters) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int n = 0;
-    for (int t0 = 0; t0 < T; t0 += 16) {
-        ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(16, T - t0); ce.pad = 0;
-        chunks[n++] = ce;
-    }
-    *n_shared = n;
-    for (int e = 0; e < E; ++e) {
-        for (int s = 0; s < counts[e]; s += 16) {
-            ChunkEntry ce; ce.expert = e; ce.start = offsets[e] + s; ce.count = min(16, counts[e] - s); ce.pad = 0;
-            chunks[n++] = ce;
-        }
-    }
-    *n_chunks = n;
-    counters[0] = 0;
-    counters[1] = 0;
 }
 
 int decode_max_chunks(int T, int k, int E) { return int(ceil_div(T, 16)) + int(ceil_div(int64_t(T) * k, 16)) + E; }
@@ -493,13 +580,6 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t in
     return r == CUDA_SUCCESS;
 }
 
-moe_status launch_decode_plan(const int32_t* counts, const int32_t* offsets, int T, int E, void* chunks,
-                              int32_t* n_chunks, int32_t* n_shared, int32_t* counters, cudaStream_t stream) {
-    decode_plan_kernel<<<1, 32, 0, stream>>>(counts, offsets, T, E, static_cast<ChunkEntry*>(chunks), n_chunks,
-                                             n_shared, counters);
-    return launch_status();
-}
-
 moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParams& prm, cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -524,6 +604,83 @@ moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv
     int64_t blocks = ceil_div(n4, 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
     combine_kernel<<<unsigned(blocks), 256, 0, stream>>>(y_s, y_r, inv_perm, T, D, k, out);
+    return launch_status();
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// fp16 operands for the int4 MMAs.
+//
+// One CTA per row of a bf16 matrix (x, or the routed experts' hidden h):
+//   scale = 2^-e with e chosen from the row's largest magnitude so that the
+//           scaled row stays below 2^15 (fp16 keeps every bf16 value exactly
+//           in that range); rscale[r] = 2^e undoes it on the MMA results;
+//   out16  every 8-block stored as x0 x4 x2 x6 x1/16 x5/16 x3/16 x7/16 (scaled)
+//          -- the K order and the 1/16 factors the int4 unpacking expects;
+//   negc   per group of 128: -(1032 * sum of the even-position stored values
+//          + 1152 * sum of the odd-position stored values), the offset the
+//          unpacked codes (1032 + q and 1152 + 16 q) add to a dot product.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in, int cols,
+                                                    __half* __restrict__ out16, float* __restrict__ negc,
+                                                    float* __restrict__ rscale) {
+    __shared__ float red[8];
+    const int64_t r = blockIdx.x;
+    const bf16* row = in + r * cols;
+    const int nblk = cols / 8;
+    float m = 0.0f;
+    for (int b = threadIdx.x; b < nblk; b += 256) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * b);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+    int e = 0;
+    if (m > 0.0f) {
+        e = int((__float_as_uint(m) >> 23) & 0xFF) - 127 - 14;
+        e = max(-100, min(e, 113));
+    }
+    const float down = __uint_as_float(uint32_t(127 - e) << 23);
+    if (threadIdx.x == 0) rscale[r] = __uint_as_float(uint32_t(127 + e) << 23);
+    // 256 threads take consecutive 8-blocks; 16 consecutive threads hold one group
+    for (int b0 = 0; b0 < nblk; b0 += 256) {
+        const int b = b0 + threadIdx.x;
+        float ev = 0.0f, od = 0.0f;
+        if (b < nblk) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * b);
+            const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+            const int order[8] = {0, 4, 2, 6, 1, 5, 3, 7};
+            __half h[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float s = x[order[i]] * down * (i < 4 ? 1.0f : 0.0625f);
+                h[i] = __float2half_rn(s);
+                if (i < 4) ev += __half2float(h[i]); else od += __half2float(h[i]);
+            }
+            *reinterpret_cast<uint4*>(out16 + r * cols + 8 * b) = *reinterpret_cast<const uint4*>(h);
+        }
+        float cs = 1032.0f * ev + 1152.0f * od;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+        if (b < nblk && (threadIdx.x & 15) == 0) negc[r * (cols / kGroup) + b / 16] = -cs;
+    }
+}
+
+moe_status launch_act16(const bf16* in, int64_t rows, int cols, __half* out16, float* negc, float* rscale,
+                        cudaStream_t stream) {
+    if (rows == 0) return MOE_OK;
+    act16_kernel<<<unsigned(rows), 256, 0, stream>>>(in, cols, out16, negc, rscale);
     return launch_status();
 }
 

@@ -14,10 +14,6 @@ moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, uint
 moe_status launch_quantize_fp8_rows(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
                                     int64_t num_valid, float scale_ub, uint8_t* q, float* scales,
                                     cudaStream_t stream);
-moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
-                        int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
-                        int32_t* inv_perm, bf16* x_frag, int32_t* zero_words, int n_zero, cudaStream_t stream,
-                        cudaEvent_t between = nullptr);
 }  // namespace moe
 
 using namespace moe;
@@ -40,8 +36,8 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
 
 // Workspace regions, each 256-byte aligned.
 struct WsLayout {
-    size_t status, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
-    size_t x_frag, h_r, h_s, y_r, y_s, x_in, out, total;
+    size_t status, zeros, zero_corr, zeros_end, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s, x_in, out, total;
 };
 
 WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
@@ -54,6 +50,10 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
     };
     const int64_t S = T * L.k;
     w.status = take(64);
+    const int maxdim = L.D > L.F ? (L.D > L.F_shared ? L.D : L.F_shared) : (L.F > L.F_shared ? L.F : L.F_shared);
+    w.zeros = take(size_t(maxdim) * 2);
+    w.zero_corr = take(size_t(maxdim / kGroup) * 4);
+    w.zeros_end = off;
     w.counters = take(64);
     w.ids = take(S * 4);
     w.gates = take(S * 4);
@@ -64,7 +64,13 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
     w.chunks = take(size_t(decode_max_chunks(int(T), L.k, L.E)) * sizeof(ChunkEntry));
     w.nchunks = take(16);
     w.x_frag = take(T * L.D * 2);
+    w.x16 = take(T * L.D * 2);
+    w.x_negc = take(T * (L.D / kGroup) * 4);
+    w.x_scale = take(T * 4);
     w.h_r = take(S * L.F * 2);
+    w.h16 = take(S * L.F * 2);
+    w.h_negc = take(S * (L.F / kGroup) * 4);
+    w.h_scale = take(S * 4);
     w.h_s = take(T * L.F_shared * 2);
     w.y_r = take(S * L.D * 4);
     w.y_s = take(T * L.D * 4);
@@ -101,9 +107,9 @@ struct Marks {
     }
 };
 
-const char* const kDecodeLaunches[] = {"route_topk", "bucket", "decode_plan", "decode_gate_up",
-                                       "decode_down", "combine"};
-constexpr int32_t kDecodeLaunchCount = 6;
+const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up",
+                                       "act16_h", "decode_down", "combine"};
+constexpr int32_t kDecodeLaunchCount = 7;
 
 template <typename T>
 T* at(void* base, size_t off) {
@@ -125,16 +131,21 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
     int32_t* nch = at<int32_t>(ws, W.nchunks);
 
+    RoutePrep prep;
+    prep.x_frag = x_frag;
+    prep.chunks = chunks;
+    prep.n_chunks = nch;
+    prep.zero_words = counters;
+    prep.n_zero = 2;
     mk.mark(st);
     moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                                 at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
-                                at<int32_t>(ws, W.offsets), perm, inv, x_frag, nullptr, 0, st,
+                                at<int32_t>(ws, W.offsets), perm, inv, &prep, st,
                                 (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
     ++mk.i;
     if (s != MOE_OK) return s;
     mk.mark(st);
-    s = launch_decode_plan(at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), T, L.E, chunks, nch, nch + 1,
-                           counters, st);
+    s = launch_act16(x, T, L.D, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale), st);
     if (s != MOE_OK) return s;
 
     DecodeMaps m1, m2;
@@ -162,18 +173,27 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.n_shared_chunks = nch + 1;
     p.perm = perm;
     p.gates = gates;
-    p.b_r = x_frag;
+    p.b_r = at<bf16>(ws, W.x16);
     p.ldb_r = L.D;
     p.b_s = x_frag;
     p.ldb_s = L.D;
     p.sc0 = L.s_gate;
     p.sc1 = L.s_up;
+    p.corr_r = at<float>(ws, W.x_negc);
+    p.rscale_r = at<float>(ws, W.x_scale);
     p.h_r = h_r;
     p.h_s = h_s;
+    p.zero_row = at<bf16>(ws, W.zeros);
+    p.zero_corr = at<float>(ws, W.zero_corr);
     p.task_counter = counters;
     p.status = status;
     mk.mark(st);
     s = launch_decode_ffn(0, m1, p, st);
+    if (s != MOE_OK) return s;
+
+    mk.mark(st);
+    s = launch_act16(h_r, int64_t(T) * L.k, L.F, at<__half>(ws, W.h16), at<float>(ws, W.h_negc),
+                     at<float>(ws, W.h_scale), st);
     if (s != MOE_OK) return s;
 
     p.n_rows_r = L.D;
@@ -181,12 +201,14 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.K_r = L.F;
     p.K_s = L.F_shared;
     p.scale_buf_floats = 32 * (L.F / kGroup);
-    p.b_r = h_r;
+    p.b_r = at<bf16>(ws, W.h16);
     p.ldb_r = L.F;
     p.b_s = h_s;
     p.ldb_s = L.F_shared;
     p.sc0 = L.s_down;
     p.sc1 = nullptr;
+    p.corr_r = at<float>(ws, W.h_negc);
+    p.rscale_r = at<float>(ws, W.h_scale);
     p.y_r = y_r;
     p.y_s = y_s;
     p.task_counter = counters + 1;
@@ -214,7 +236,9 @@ moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t 
         decode_smem_bytes(32 * (layer->F / kGroup)) > 227 * 1024)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (layer->path == MOE_PATH_PREFILL) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    // the device status word and the zero rows read in place of missing tokens
+    if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return ffn_decode_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
 }
 
@@ -269,8 +293,8 @@ moe_status moe_route(const void* x, int32_t T, int32_t D, const void* w_router, 
         if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
     if (router_bias && !aligned16(router_bias)) return MOE_ERR_INVALID_ARG;
     return launch_route(static_cast<const bf16*>(x), T, D, static_cast<const bf16*>(w_router), router_bias, E, k,
-                        topk_ids, topk_gates, expert_counts, expert_offsets, perm, nullptr, nullptr, nullptr, 0,
-                        as_stream(stream));
+                        topk_ids, topk_gates, expert_counts, expert_offsets, perm, nullptr, nullptr,
+                        as_stream(stream), nullptr);
 }
 
 size_t moe_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max) {

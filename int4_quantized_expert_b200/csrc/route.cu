@@ -7,33 +7,52 @@
 // the router is a linear layer; Scout keeps 1 of 16 experts, Maverick 8 of 128.
 //
 // Kernels:
-//   route_topk_kernel  logits = x W_r^T (+b) on tensor cores (m16n8k16, fp32
-//                      accumulate), then per token k passes of a warp argmax
-//                      (ties -> lower expert index), then the gate.
-//   bucket_kernel      one CTA: per-expert counts, exclusive offsets and the
-//                      stable permutation of slots, using warp match/ballot
-//                      ranks and a block scan over warps.
+//   router_kernel  16 tokens per CTA; up to 12 warps split the K dimension in
+//                  whole groups of 128, each computing 16 x E partial logits
+//                  with m16n8k16 tensor-core MMAs (fp32 accumulate) from
+//                  fragments loaded straight from global memory.  Partials are
+//                  summed in a fixed order (deterministic), the bias added, and
+//                  each token's top-k taken by k passes of a warp argmax (ties
+//                  -> lower expert index), then the gate.  For the weight-
+//                  streaming FFN it also writes x in the fragment order its
+//                  shared-expert MMAs read.
+//   bucket_kernel  one CTA: per-expert counts, exclusive offsets and the stable
+//                  permutation of slots from warp match ranks and a scan over
+//                  warps; optionally the weight-streaming FFN's task list.
 #include "common.cuh"
+#include "ffn_decode.cuh"
 
 namespace moe {
 
-constexpr int RT_TOK = 64;      // tokens per CTA (4 warps x 16)
-constexpr int RT_K = 64;        // K chunk staged in shared memory
+constexpr int RT_TOK = 16;      // tokens per CTA (one m16 tile)
+constexpr int RT_MAXW = 12;     // warps splitting K
 constexpr int RT_EPASS = 64;    // experts per accumulator pass (8 n-tiles)
-constexpr int RT_LD = RT_K + 8; // padded row length (bf16) -> conflict-free 32-bit reads
+constexpr size_t RT_SMEM_MAX = 160 * 1024;
 
-__global__ void __launch_bounds__(128) route_topk_kernel(
+// Warps used: the largest divisor of D / 128 that is <= 12 and whose partial
+// logits (warps x 16 tokens x E fp32) fit in RT_SMEM_MAX.
+inline int router_warps(int D, int E) {
+    const int groups = D / kGroup;
+    for (int w = RT_MAXW; w > 1; --w)
+        if (groups % w == 0 && size_t(w) * RT_TOK * E * sizeof(float) <= RT_SMEM_MAX) return w;
+    return 1;
+}
+
+__global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     const bf16* __restrict__ x, int T, int D, const bf16* __restrict__ wr,
     const float* __restrict__ bias, int E, int k, int32_t* __restrict__ ids,
     float* __restrict__ gates, bf16* __restrict__ x_frag) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    bf16* xs = reinterpret_cast<bf16*>(smem_raw);                 // [RT_TOK][RT_LD]
-    bf16* ws = xs + RT_TOK * RT_LD;                               // [RT_EPASS][RT_LD]
-    float* logits = reinterpret_cast<float*>(ws + RT_EPASS * RT_LD);  // [RT_TOK][E]
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    extern __shared__ __align__(16) float part[];     // [nw][RT_TOK][E]
+    const int nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int t0 = blockIdx.x * RT_TOK;
+    const int groups_per_warp = (D / kGroup) / nw;
+    const int k_begin = warp * groups_per_warp * kGroup;
+    const int k_end = k_begin + groups_per_warp * kGroup;
+    const bool row_a = t0 + g < T, row_b = t0 + g + 8 < T;
+    const bf16* xa_row = x + int64_t(t0 + g) * D;
+    const bf16* xb_row = x + int64_t(t0 + g + 8) * D;
 
     for (int e0 = 0; e0 < E; e0 += RT_EPASS) {
         float acc[8][4];
@@ -42,84 +61,81 @@ __global__ void __launch_bounds__(128) route_topk_kernel(
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
 
-        for (int k0 = 0; k0 < D; k0 += RT_K) {
-            __syncthreads();
-            // stage x[t0 .. t0+63][k0 .. k0+63] and W_r[e0 .. e0+63][k0 .. k0+63]
-            for (int i = tid; i < RT_TOK * (RT_K / 8); i += 128) {
-                const int r = i / (RT_K / 8), q = i % (RT_K / 8);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                const int t = t0 + r;
-                if (t < T) {
-                    v = *reinterpret_cast<const uint4*>(x + int64_t(t) * D + k0 + q * 8);
-                    // The first expert pass also writes x in the layout the
-                    // weight-streaming kernels read: every 8 consecutive values
-                    // stored as x0 x4 x1 x5 x2 x6 x3 x7.
-                    if (x_frag != nullptr && e0 == 0) {
-                        uint4 p;
-                        p.x = prmt(v.x, v.z, 0x5410);
-                        p.y = prmt(v.x, v.z, 0x7632);
-                        p.z = prmt(v.y, v.w, 0x5410);
-                        p.w = prmt(v.y, v.w, 0x7632);
-                        *reinterpret_cast<uint4*>(x_frag + int64_t(t) * D + k0 + q * 8) = p;
-                    }
+        // operands of the next 32-K chunk are loaded while the current one runs
+        const int n_tiles = min(8, (E - e0 + 7) / 8);
+        uint4 xa, xb, wv[8], nxa, nxb, nwv[8];
+        auto load = [&](int kk, uint4& a, uint4& b, uint4 (&w)[8]) {
+            a = row_a ? ldg_cached(xa_row + kk + 8 * c) : make_uint4(0, 0, 0, 0);
+            b = row_b ? ldg_cached(xb_row + kk + 8 * c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int e = e0 + n * 8 + g;
+                w[n] = (n < n_tiles && e < E) ? ldg_cached(wr + int64_t(e) * D + kk + 8 * c) : make_uint4(0, 0, 0, 0);
+            }
+        };
+        load(k_begin, xa, xb, wv);
+        for (int kk = k_begin; kk < k_end; kk += 32) {
+            if (kk + 32 < k_end) load(kk + 32, nxa, nxb, nwv);
+            // thread (g, c) holds K values kk + 8c .. kk + 8c + 7 of rows g and g + 8;
+            // the two MMAs below use them as K pairs (0,1)(2,3) and (4,5)(6,7)
+            // of A, and the expert rows of W_r in the same order as B.
+            if (x_frag != nullptr && e0 == 0) {
+                // x in the bf16 fragment order the shared expert's weight-
+                // streaming MMAs read (every 8 values stored x0 x4 x1 x5 x2 x6 x3 x7)
+                if (row_a) {
+                    uint4 p;
+                    p.x = prmt(xa.x, xa.z, 0x5410); p.y = prmt(xa.x, xa.z, 0x7632);
+                    p.z = prmt(xa.y, xa.w, 0x5410); p.w = prmt(xa.y, xa.w, 0x7632);
+                    *reinterpret_cast<uint4*>(x_frag + int64_t(t0 + g) * D + kk + 8 * c) = p;
                 }
-                *reinterpret_cast<uint4*>(xs + r * RT_LD + q * 8) = v;
-            }
-            for (int i = tid; i < RT_EPASS * (RT_K / 8); i += 128) {
-                const int r = i / (RT_K / 8), q = i % (RT_K / 8);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (e0 + r < E) v = *reinterpret_cast<const uint4*>(wr + int64_t(e0 + r) * D + k0 + q * 8);
-                *reinterpret_cast<uint4*>(ws + r * RT_LD + q * 8) = v;
-            }
-            __syncthreads();
-            const bf16* xa = xs + (warp * 16) * RT_LD;
-#pragma unroll
-            for (int kk = 0; kk < RT_K; kk += 16) {
-                const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xa + g * RT_LD + kk + 2 * c);
-                const uint32_t a1 = *reinterpret_cast<const uint32_t*>(xa + (g + 8) * RT_LD + kk + 2 * c);
-                const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xa + g * RT_LD + kk + 2 * c + 8);
-                const uint32_t a3 = *reinterpret_cast<const uint32_t*>(xa + (g + 8) * RT_LD + kk + 2 * c + 8);
-#pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    if (e0 + n * 8 >= E) break;
-                    const bf16* wb = ws + (n * 8 + g) * RT_LD + kk + 2 * c;
-                    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wb);
-                    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wb + 8);
-                    mma_bf16_16816(acc[n], a0, a1, a2, a3, b0, b1);
+                if (row_b) {
+                    uint4 p;
+                    p.x = prmt(xb.x, xb.z, 0x5410); p.y = prmt(xb.x, xb.z, 0x7632);
+                    p.z = prmt(xb.y, xb.w, 0x5410); p.w = prmt(xb.y, xb.w, 0x7632);
+                    *reinterpret_cast<uint4*>(x_frag + int64_t(t0 + g + 8) * D + kk + 8 * c) = p;
                 }
             }
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                if (n >= n_tiles) break;
+                mma_bf16_16816(acc[n], xa.x, xb.x, xa.y, xb.y, wv[n].x, wv[n].y);
+                mma_bf16_16816(acc[n], xa.z, xb.z, xa.w, xb.w, wv[n].z, wv[n].w);
+            }
+            xa = nxa;
+            xb = nxb;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) wv[n] = nwv[n];
         }
-        // scatter this pass's logits to shared memory
+        // C fragment: rows (tokens) g, g + 8; columns (experts) 2c, 2c + 1 of each n-tile
+        float* pw = part + warp * RT_TOK * E;
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
             const int e = e0 + n * 8 + 2 * c;
-            const int r0 = warp * 16 + g;
-            if (e < E) {
-                logits[r0 * E + e] = acc[n][0];
-                logits[(r0 + 8) * E + e] = acc[n][2];
-            }
-            if (e + 1 < E) {
-                logits[r0 * E + e + 1] = acc[n][1];
-                logits[(r0 + 8) * E + e + 1] = acc[n][3];
-            }
+            if (e < E) { pw[g * E + e] = acc[n][0]; pw[(g + 8) * E + e] = acc[n][2]; }
+            if (e + 1 < E) { pw[g * E + e + 1] = acc[n][1]; pw[(g + 8) * E + e + 1] = acc[n][3]; }
         }
     }
     __syncthreads();
 
-    // top-k per token: each warp takes 16 tokens; lane holds experts lane + 32 i
-    for (int r = warp * 16; r < warp * 16 + 16; ++r) {
+    // top-k per token; lane holds experts lane + 32 i
+    for (int r = warp; r < RT_TOK; r += nw) {
         const int t = t0 + r;
         if (t >= T) break;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = lane + 32 * i;
-            v[i] = (e < E) ? logits[r * E + e] + (bias ? bias[e] : 0.0f) : -INFINITY;
+            float s = -INFINITY;
+            if (e < E) {
+                s = 0.0f;
+                for (int w = 0; w < nw; ++w) s += part[(w * RT_TOK + r) * E + e];
+                if (bias) s += bias[e];
+            }
+            v[i] = s;
         }
         float chosen_val[8];
         int chosen_id[8];
         for (int j = 0; j < k; ++j) {
-            // lane-local best (largest value, lowest index among equals)
             float bv = -INFINITY;
             int bi = 0x7fffffff;
 #pragma unroll
@@ -135,16 +151,15 @@ __global__ void __launch_bounds__(128) route_topk_kernel(
             }
             chosen_val[j] = bv;
             chosen_id[j] = bi;
-            // remove the winner: a NaN never compares greater or equal, so it
-            // is never selected again
+            // remove the winner: a NaN never compares greater or equal
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 if (lane + 32 * i == bi) v[i] = __int_as_float(0x7fc00000u);
         }
         if (lane == 0) {
             if (k == 1) {
-                ids[int64_t(t)] = chosen_id[0];
-                gates[int64_t(t)] = 1.0f / (1.0f + expf(-chosen_val[0]));
+                ids[t] = chosen_id[0];
+                gates[t] = 1.0f / (1.0f + expf(-chosen_val[0]));
             } else {
                 float sum = 0.0f, ex[8];
                 for (int j = 0; j < k; ++j) { ex[j] = expf(chosen_val[j] - chosen_val[0]); sum += ex[j]; }
@@ -165,9 +180,10 @@ constexpr int BK_WARPS = BK_THREADS / 32;
 constexpr int BK_MAX_E = 256;
 
 __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
-    const int32_t* __restrict__ ids, int n_slots, int E, int32_t* __restrict__ counts,
+    const int32_t* __restrict__ ids, int n_slots, int T, int E, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-    int32_t* __restrict__ zero_words, int n_zero) {
+    ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int32_t* __restrict__ zero_words,
+    int n_zero) {
     __shared__ int s_count[BK_MAX_E];
     __shared__ int s_base[BK_MAX_E];
     __shared__ int s_warp[BK_WARPS][BK_MAX_E];   // per-warp counts, then exclusive prefix over warps
@@ -182,6 +198,23 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     if (tid == 0) {
         int run = 0;
         for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_count[e]; }
+        if (chunks != nullptr) {
+            // task list of the weight-streaming FFN: chunks of <= 16 tokens,
+            // the shared expert's first, then each routed expert's
+            int n = 0;
+            for (int t0 = 0; t0 < T; t0 += 16) {
+                ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(16, T - t0); ce.pad = 0;
+                chunks[n++] = ce;
+            }
+            n_chunks[1] = n;
+            for (int e = 0; e < E; ++e)
+                for (int s = 0; s < s_count[e]; s += 16) {
+                    ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s; ce.count = min(16, s_count[e] - s);
+                    ce.pad = 0;
+                    chunks[n++] = ce;
+                }
+            n_chunks[0] = n;
+        }
     }
     __syncthreads();
     for (int e = tid; e < E; e += BK_THREADS) {
@@ -222,25 +255,24 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     }
 }
 
-size_t route_smem_bytes(int E) {
-    return size_t(RT_TOK + RT_EPASS) * RT_LD * sizeof(bf16) + size_t(RT_TOK) * E * sizeof(float);
-}
+size_t router_smem_bytes(int D, int E) { return size_t(router_warps(D, E)) * RT_TOK * E * sizeof(float); }
 
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
-                        int32_t* inv_perm, bf16* x_frag, int32_t* zero_words, int n_zero,
-                        cudaStream_t stream, cudaEvent_t between) {
-    const size_t smem = route_smem_bytes(E);
-    cudaError_t err = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(route_smem_bytes(BK_MAX_E)));
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
-    route_topk_kernel<<<unsigned(ceil_div(T, RT_TOK)), 128, smem, stream>>>(x, T, D, wr, bias, E, k,
-                                                                            ids, gates, x_frag);
+                        int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between) {
+    const int nw = router_warps(D, E);
+    const size_t smem = router_smem_bytes(D, E);
+    if (cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(RT_SMEM_MAX)) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    router_kernel<<<unsigned(ceil_div(T, RT_TOK)), nw * 32, smem, stream>>>(
+        x, T, D, wr, bias, E, k, ids, gates, prep ? prep->x_frag : nullptr);
     moe_status st = launch_status();
     if (st != MOE_OK) return st;
     if (between) cudaEventRecord(between, stream);
-    bucket_kernel<<<1, BK_THREADS, 0, stream>>>(ids, T * k, E, counts, offsets, perm, inv_perm,
-                                                zero_words, n_zero);
+    bucket_kernel<<<1, BK_THREADS, 0, stream>>>(ids, T * k, T, E, counts, offsets, perm, inv_perm,
+                                                prep ? prep->chunks : nullptr, prep ? prep->n_chunks : nullptr,
+                                                prep ? prep->zero_words : nullptr, prep ? prep->n_zero : 0);
     return launch_status();
 }
 
