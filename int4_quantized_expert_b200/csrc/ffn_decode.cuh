@@ -51,6 +51,7 @@ struct RoutePrep {
     bf16* x_frag;         // x in bf16 fragment order [T, D] (shared expert)
     ChunkEntry* chunks;   // task list
     int32_t* n_chunks;    // [0] all chunks, [1] the shared expert's
+    int32_t chunk_tokens; // tokens per chunk (16 for the weight-streaming path, 256 for tensor-core tiles)
     int32_t* zero_words;  // zeroed (task counters)
     int32_t n_zero;
 };

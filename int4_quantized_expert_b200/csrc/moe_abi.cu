@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "ffn_decode.cuh"
+#include "tc_gemm.cuh"
 
 namespace moe {
 moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, uint8_t* codes, float* scales,
@@ -34,14 +35,26 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
     return MOE_OK;
 }
 
-// Workspace regions, each 256-byte aligned.
+// Workspace regions, each 256-byte aligned.  The regions up to `common_end`
+// are shared by both paths; the rest is laid out per path from there, and a
+// workspace must be large enough for either.
 struct WsLayout {
     size_t status, zeros, zero_corr, zeros_end, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
-    size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s, x_in, out, total;
+    size_t common_end;
+    // weight-streaming path
+    size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
+    // tensor-core path (row counts padded to whole 256-token tiles)
+    size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos;
+    // host staging of moe_ffn_forward_host
+    size_t x_in, out;
+    size_t total;
 };
 
-WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
+enum { PATH_SEL_DECODE = 1, PATH_SEL_PREFILL = 2 };
+
+WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     WsLayout w;
+    memset(&w, 0, sizeof(w));
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -49,6 +62,8 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
         return o;
     };
     const int64_t S = T * L.k;
+    const int64_t S_pad = ceil_div(S, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
+    const int64_t T_pad = ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
     w.status = take(64);
     const int maxdim = L.D > L.F ? (L.D > L.F_shared ? L.D : L.F_shared) : (L.F > L.F_shared ? L.F : L.F_shared);
     w.zeros = take(size_t(maxdim) * 2);
@@ -63,21 +78,42 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T) {
     w.inv_perm = take(S * 4);
     w.chunks = take(size_t(decode_max_chunks(int(T), L.k, L.E)) * sizeof(ChunkEntry));
     w.nchunks = take(16);
-    w.x_frag = take(T * L.D * 2);
-    w.x16 = take(T * L.D * 2);
-    w.x_negc = take(T * (L.D / kGroup) * 4);
-    w.x_scale = take(T * 4);
-    w.h_r = take(S * L.F * 2);
-    w.h16 = take(S * L.F * 2);
-    w.h_negc = take(S * (L.F / kGroup) * 4);
-    w.h_scale = take(S * 4);
-    w.h_s = take(T * L.F_shared * 2);
-    w.y_r = take(S * L.D * 4);
-    w.y_s = take(T * L.D * 4);
+    w.common_end = off;
+    if (path == PATH_SEL_DECODE) {
+        w.x_frag = take(T * L.D * 2);
+        w.x16 = take(T * L.D * 2);
+        w.x_negc = take(T * (L.D / kGroup) * 4);
+        w.x_scale = take(T * 4);
+        w.h_r = take(S * L.F * 2);
+        w.h16 = take(S * L.F * 2);
+        w.h_negc = take(S * (L.F / kGroup) * 4);
+        w.h_scale = take(S * 4);
+        w.h_s = take(T * L.F_shared * 2);
+        w.y_r = take(S * L.D * 4);
+        w.y_s = take(T * L.D * 4);
+    } else {
+        w.x_sorted = take(S_pad * L.D * 2);
+        w.h_sorted = take(S_pad * L.F * 2);
+        w.x_pad = take(T_pad * L.D * 2);
+        w.h_s_pad = take(T_pad * L.F_shared * 2);
+        w.y_pos = take(S * L.D * 4);
+    }
     w.x_in = take(T * L.D * 2);
     w.out = take(T * L.D * 2);
     w.total = off;
     return w;
+}
+
+size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
+    const size_t a = ws_layout(L, T, PATH_SEL_DECODE).total;
+    const size_t b = ws_layout(L, T, PATH_SEL_PREFILL).total;
+    return a > b ? a : b;
+}
+
+int choose_path(const moe_layer_desc& L, int64_t T) {
+    if (L.path == MOE_PATH_DECODE) return PATH_SEL_DECODE;
+    if (L.path == MOE_PATH_PREFILL) return PATH_SEL_PREFILL;
+    return T * L.k <= 4 * int64_t(L.E) ? PATH_SEL_DECODE : PATH_SEL_PREFILL;
 }
 
 moe_status check_layer(const moe_layer_desc* L) {
@@ -137,6 +173,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     prep.n_chunks = nch;
     prep.zero_words = counters;
     prep.n_zero = 2;
+    prep.chunk_tokens = 16;
     mk.mark(st);
     moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                                 at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
@@ -221,6 +258,99 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     return s;
 }
 
+const char* const kPrefillLaunches[] = {"router", "bucket", "gather", "tc_gate_up", "tc_down",
+                                        "tc_shared_gate_up", "tc_shared_down_combine"};
+constexpr int32_t kPrefillLaunchCount = 7;
+
+moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
+                            const WsLayout& W, cudaStream_t st, Marks& mk) {
+    int32_t* status = at<int32_t>(ws, W.status);
+    int32_t* perm = at<int32_t>(ws, W.perm);
+    int32_t* inv = at<int32_t>(ws, W.inv_perm);
+    float* gates = at<float>(ws, W.gates);
+    ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
+    int32_t* nch = at<int32_t>(ws, W.nchunks);
+    const int64_t S = int64_t(T) * L.k;
+    const uint64_t S_pad = uint64_t(ceil_div(S, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
+    const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
+    bf16* x_sorted = at<bf16>(ws, W.x_sorted);
+    bf16* h_sorted = at<bf16>(ws, W.h_sorted);
+    bf16* x_pad = at<bf16>(ws, W.x_pad);
+    bf16* h_s = at<bf16>(ws, W.h_s_pad);
+    float* y_pos = at<float>(ws, W.y_pos);
+
+    RoutePrep prep;
+    memset(&prep, 0, sizeof(prep));
+    prep.chunks = chunks;
+    prep.n_chunks = nch;
+    prep.chunk_tokens = TC_BLOCK_TOKENS;
+    mk.mark(st);
+    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+                                at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
+                                at<int32_t>(ws, W.offsets), perm, inv, &prep, st,
+                                (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
+    ++mk.i;
+    if (s != MOE_OK) return s;
+    mk.mark(st);
+    s = launch_gather_rows(x, perm, S, L.k, L.D, x_sorted, st);
+    if (s != MOE_OK) return s;
+    // the shared expert reads x through a 256-row tile map: copy it into whole tiles
+    if (cudaMemcpyAsync(x_pad, x, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+
+    const uint64_t E = uint64_t(L.E);
+    TcMaps m_gu, m_dn, m_sgu, m_sdn;
+    bool ok = make_tmap_2d(&m_gu.b, x_sorted, true, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D / 2, E * L.F, 32, 64, false) &&
+              make_tmap_2d(&m_gu.a1, L.w_up, false, L.D / 2, E * L.F, 32, 64, false) &&
+              make_tmap_2d(&m_dn.b, h_sorted, true, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_dn.a0, L.w_down, false, L.F / 2, E * L.D, 32, 64, false) &&
+              make_tmap_2d(&m_sgu.b, x_pad, true, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_sgu.a0, L.ws_gate, true, L.D, L.F_shared, 64, 16, true) &&
+              make_tmap_2d(&m_sgu.a1, L.ws_up, true, L.D, L.F_shared, 64, 16, true) &&
+              make_tmap_2d(&m_sdn.b, h_s, true, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_sdn.a0, L.ws_down, true, L.F_shared, L.D, 64, 16, true);
+    if (!ok) return MOE_ERR_CUDA;
+    m_dn.a1 = m_dn.a0;
+    m_sdn.a1 = m_sdn.a0;
+
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.chunks = chunks;
+    p.n_chunks = nch;
+    p.gates = gates;
+    p.perm = perm;
+    p.inv_perm = inv;
+    p.k_top = L.k;
+    p.status = status;
+
+    // routed gate/up -> h (bf16, fragment order, by slot position)
+    p.K = L.D; p.n_rows = L.F; p.n_fblocks = L.F / 64; p.routed = 1;
+    p.s0 = L.s_gate; p.s1 = L.s_up; p.h_out = h_sorted;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_GATEUP_INT4, m_gu, p, st);
+    if (s != MOE_OK) return s;
+    // routed down -> gate * y (fp32, by slot position)
+    p.K = L.F; p.n_rows = L.D; p.n_fblocks = L.D / 128;
+    p.s0 = L.s_down; p.s1 = nullptr; p.h_out = nullptr; p.y_out = y_pos;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_DOWN_INT4, m_dn, p, st);
+    if (s != MOE_OK) return s;
+    // shared gate/up -> h_s (bf16, natural order, by token)
+    p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
+    p.s0 = nullptr; p.y_out = nullptr; p.h_out = h_s;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_GATEUP_BF16, m_sgu, p, st);
+    if (s != MOE_OK) return s;
+    // shared down + the routed outputs of each token -> out
+    p.K = L.F_shared; p.n_rows = L.D; p.n_fblocks = L.D / 128;
+    p.h_out = nullptr; p.out = out; p.y_r = y_pos;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_COMBINE_BF16, m_sdn, p, st);
+    mk.mark(st);
+    return s;
+}
+
 moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t T, void* out, void* workspace,
                             size_t workspace_bytes, cudaStream_t st, Marks mk = Marks()) {
     moe_status s = check_layer(layer);
@@ -230,16 +360,18 @@ moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t 
     if (!x || !out || !workspace || !aligned16(x) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return MOE_ERR_INVALID_ARG;
-    const WsLayout W = ws_layout(*layer, T);
+    const int path = choose_path(*layer, T);
+    const WsLayout W = ws_layout(*layer, T, path);
     if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (decode_smem_bytes(2 * 32 * (layer->D / kGroup)) > 227 * 1024 ||
-        decode_smem_bytes(32 * (layer->F / kGroup)) > 227 * 1024)
+    if (path == PATH_SEL_DECODE && (decode_smem_bytes(2 * 32 * (layer->D / kGroup)) > 227 * 1024 ||
+                                    decode_smem_bytes(32 * (layer->F / kGroup)) > 227 * 1024))
         return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (layer->path == MOE_PATH_PREFILL) return MOE_ERR_UNSUPPORTED_SHAPE;
     // the device status word and the zero rows read in place of missing tokens
     if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
         return MOE_ERR_CUDA;
-    return ffn_decode_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
+    if (path == PATH_SEL_DECODE)
+        return ffn_decode_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
+    return ffn_prefill_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
 }
 
 }  // namespace
@@ -299,7 +431,7 @@ moe_status moe_route(const void* x, int32_t T, int32_t D, const void* w_router, 
 
 size_t moe_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max) {
     if (check_layer(layer) != MOE_OK || T_max < 1 || T_max > kMaxT) return 0;
-    return ws_layout(*layer, T_max).total;
+    return ws_bytes(*layer, T_max);
 }
 
 moe_status moe_ffn_forward(const moe_layer_desc* layer, const void* x, int32_t T, void* out, void* workspace,
@@ -314,7 +446,7 @@ moe_status moe_ffn_forward_host(const moe_layer_desc* layer, const void* x_host,
     s = check_route_shape(T, layer->D, layer->E, layer->k);
     if (s != MOE_OK) return s;
     if (!x_host || !out_host || !workspace) return MOE_ERR_INVALID_ARG;
-    const WsLayout W = ws_layout(*layer, T);
+    const WsLayout W = ws_layout(*layer, T, choose_path(*layer, T));
     if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = as_stream(stream);
     const size_t bytes = size_t(T) * layer->D * 2;
@@ -330,7 +462,9 @@ moe_status moe_ffn_forward_host(const moe_layer_desc* layer, const void* x_host,
 moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
                                  void* workspace, size_t workspace_bytes, void* stream, void* const* events,
                                  int32_t n_events) {
-    if (!events || n_events < kDecodeLaunchCount + 1) return MOE_ERR_INVALID_ARG;
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE ? kDecodeLaunchCount : kPrefillLaunchCount;
+    if (!events || n_events < need + 1) return MOE_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_events; ++i)
         if (!events[i]) return MOE_ERR_INVALID_ARG;
     Marks mk;
@@ -341,8 +475,10 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
 
 int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, const char** names, int32_t max_names) {
     if (check_layer(layer) != MOE_OK || T < 1) return 0;
-    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
-    return kDecodeLaunchCount;
+    const bool dec = choose_path(*layer, T) == PATH_SEL_DECODE;
+    const int32_t n = dec ? kDecodeLaunchCount : kPrefillLaunchCount;
+    for (int32_t i = 0; i < n && i < max_names && names; ++i) names[i] = dec ? kDecodeLaunches[i] : kPrefillLaunches[i];
+    return n;
 }
 
 moe_status moe_ffn_device_status(const void* workspace, void* stream) {
@@ -400,7 +536,7 @@ extern "C" moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const
     if (s != MOE_OK) return s;
     s = check_route_shape(T, layer->D, layer->E, layer->k);
     if (s != MOE_OK) return s;
-    if (ws_layout(*layer, T).total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_layout(*layer, T, choose_path(*layer, T)).total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = nullptr;
     s = noalloc_scratch_address(&scratch);
     if (s != MOE_OK) return s;

@@ -182,8 +182,8 @@ constexpr int BK_MAX_E = 256;
 __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     const int32_t* __restrict__ ids, int n_slots, int T, int E, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-    ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int32_t* __restrict__ zero_words,
-    int n_zero) {
+    ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int chunk_tokens,
+    int32_t* __restrict__ zero_words, int n_zero) {
     __shared__ int s_count[BK_MAX_E];
     __shared__ int s_base[BK_MAX_E];
     __shared__ int s_warp[BK_WARPS][BK_MAX_E];   // per-warp counts, then exclusive prefix over warps
@@ -199,17 +199,18 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
         int run = 0;
         for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_count[e]; }
         if (chunks != nullptr) {
-            // task list of the weight-streaming FFN: chunks of <= 16 tokens,
+            // task list of the FFN kernels: chunks of <= chunk_tokens tokens,
             // the shared expert's first, then each routed expert's
             int n = 0;
-            for (int t0 = 0; t0 < T; t0 += 16) {
-                ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(16, T - t0); ce.pad = 0;
+            for (int t0 = 0; t0 < T; t0 += chunk_tokens) {
+                ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(chunk_tokens, T - t0); ce.pad = 0;
                 chunks[n++] = ce;
             }
             n_chunks[1] = n;
             for (int e = 0; e < E; ++e)
-                for (int s = 0; s < s_count[e]; s += 16) {
-                    ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s; ce.count = min(16, s_count[e] - s);
+                for (int s = 0; s < s_count[e]; s += chunk_tokens) {
+                    ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s;
+                    ce.count = min(chunk_tokens, s_count[e] - s);
                     ce.pad = 0;
                     chunks[n++] = ce;
                 }
@@ -272,6 +273,7 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
     if (between) cudaEventRecord(between, stream);
     bucket_kernel<<<1, BK_THREADS, 0, stream>>>(ids, T * k, T, E, counts, offsets, perm, inv_perm,
                                                 prep ? prep->chunks : nullptr, prep ? prep->n_chunks : nullptr,
+                                                prep ? prep->chunk_tokens : 16,
                                                 prep ? prep->zero_words : nullptr, prep ? prep->n_zero : 0);
     return launch_status();
 }

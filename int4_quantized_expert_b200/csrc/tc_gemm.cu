@@ -1,0 +1,403 @@
+// tcgen05 grouped GEMMs of the MoE layer for many tokens per expert.
+//
+// The layer ("1 卡跑通 Llama 4" (discosf.com), "混合专家路由"; "Llama 开源模型
+// 系列" (docs.ifdog.com), "SwiGLU：门控激活的数学"): each expert runs
+// (silu(x Wg^T) * (x Wu^T)) Wd^T on its tokens; routed weights are int4 with
+// one fp32 scale per 128 K and zero point 0 ("Meta Llama Models Llama 4 单卡
+// 量化推理与选型指南" (lshu.cn), "量化环节做了什么"); the shared expert is bf16.
+//
+// One persistent CTA per SM, tiles of 128 output features x 256 tokens:
+//   A = weights (M = 128 rows), B = tokens (N = 256 rows), both K-major in
+//   shared memory with the 128-byte swizzle, K step 64; D = fp32 in tensor
+//   memory (TMEM), two 256-column accumulators so a tile's epilogue overlaps
+//   the next tile's MMAs.
+// Warp roles (12 warps):
+//   warp 0      TMA producer (one thread) and TMEM allocator
+//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 inputs
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32 (w % 4) ..), SwiGLU / gate scaling / combine, stores
+//   warps 8-11  int4 modes only: dequantize the stage's codes (w = q * s, s
+//               rounded to bf16) into the swizzled A tile, one thread per row
+// Gate/up tiles hold 64 features: A rows alternate 16 gate rows and the same
+// 16 up rows, so each epilogue warp finds g (lanes 0..15) and u (lanes 16..31)
+// of its 16 features together.  Routed activations are stored with every 8
+// consecutive K values in the order x0 x4 x1 x5 x2 x6 x3 x7, the order the
+// int4 unpacking produces; the dot products do not depend on the K order.
+#include <cuda.h>
+
+#include "tc_gemm.cuh"
+
+namespace moe {
+
+constexpr int TC_THREADS = 384;
+constexpr int TC_STAGES = 4;
+constexpr int TC_B_BYTES = TC_BLOCK_TOKENS * 64 * 2;   // 32 KB
+constexpr int TC_A_BYTES = 128 * 64 * 2;               // 16 KB
+constexpr int TC_C_BYTES = 128 * 32;                   // int4 codes of the A tile: 4 KB
+constexpr int TC_STAGE_BYTES = TC_B_BYTES + TC_A_BYTES + TC_C_BYTES;
+constexpr int TC_TMEM_COLS = 512;
+static_assert(TC_STAGE_BYTES % 1024 == 0, "stage alignment");
+
+struct TcSmem {
+    uint64_t full[TC_STAGES];      // TMA data of the stage landed (tx counted)
+    uint64_t a_ready[TC_STAGES];   // converter warps wrote the A tile
+    uint64_t empty[TC_STAGES];     // the stage's MMAs completed
+    uint64_t acc_full[2];          // accumulator holds a finished tile
+    uint64_t acc_empty[2];         // epilogue finished reading the accumulator
+    uint32_t tmem_base;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// arrive on `bar` once all previously issued tcgen05.mma of this thread complete
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(const void* smem) {
+    const uint64_t addr = smem_u32(smem);
+    return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ int frag_pos(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
+
+// ---------------------------------------------------------------------------
+template <int MODE>
+__global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
+    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a0,
+    const __grid_constant__ CUtensorMap tm_a1, TcParams p) {
+    constexpr bool INT4 = MODE == TC_GATEUP_INT4 || MODE == TC_DOWN_INT4;
+    constexpr bool GATEUP = MODE == TC_GATEUP_INT4 || MODE == TC_GATEUP_BF16;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    TcSmem* sm = reinterpret_cast<TcSmem*>(base + TC_STAGES * TC_STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < TC_STAGES; ++i) {
+            mbar_init(&sm->full[i], 1);
+            mbar_init(&sm->a_ready[i], 4);
+            mbar_init(&sm->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&sm->acc_full[i], 1); mbar_init(&sm->acc_empty[i], 4); }
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+
+    const int n_all = p.n_chunks[0], n_sh = p.n_chunks[1];
+    const int c_begin = p.routed ? n_sh : 0, c_end = p.routed ? n_all : n_sh;
+    const int n_tiles = (c_end - c_begin) * p.n_fblocks;
+    const int nk = p.K / 64;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            prefetch_tmap(&tm_b); prefetch_tmap(&tm_a0); prefetch_tmap(&tm_a1);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
+                const int fb = tile % p.n_fblocks;
+                const int e = ce.expert < 0 ? 0 : ce.expert;
+                for (int kk = 0; kk < nk; ++kk, ++it) {
+                    const uint32_t slot = it % TC_STAGES;
+                    if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status, 64)) { ok = false; break; }
+                    unsigned char* st = base + slot * TC_STAGE_BYTES;
+                    unsigned char* sa = st + TC_B_BYTES;
+                    unsigned char* sc = sa + TC_A_BYTES;
+                    mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES + (INT4 ? TC_C_BYTES : TC_A_BYTES));
+                    tma_load_2d(st, &tm_b, &sm->full[slot], kk * 64, ce.start);
+                    if (MODE == TC_GATEUP_INT4) {
+                        const int row = e * p.n_rows + fb * 64;
+                        tma_load_2d(sc, &tm_a0, &sm->full[slot], kk * 32, row);
+                        tma_load_2d(sc + 64 * 32, &tm_a1, &sm->full[slot], kk * 32, row);
+                    } else if (MODE == TC_DOWN_INT4) {
+                        const int row = e * p.n_rows + fb * 128;
+                        tma_load_2d(sc, &tm_a0, &sm->full[slot], kk * 32, row);
+                        tma_load_2d(sc + 64 * 32, &tm_a0, &sm->full[slot], kk * 32, row + 64);
+                    } else if (MODE == TC_GATEUP_BF16) {
+                        // 16-row boxes: gate rows, up rows, gate rows, ... (same features)
+#pragma unroll
+                        for (int b = 0; b < 8; ++b)
+                            tma_load_2d(sa + b * 2048, (b & 1) ? &tm_a1 : &tm_a0, &sm->full[slot], kk * 64,
+                                        fb * 64 + (b >> 1) * 16);
+                    } else {
+#pragma unroll
+                        for (int b = 0; b < 8; ++b)
+                            tma_load_2d(sa + b * 2048, &tm_a0, &sm->full[slot], kk * 64, fb * 128 + b * 16);
+                    }
+                }
+            }
+            // wind down: wait (bounded) for the stages still in flight to land
+            for (uint32_t i = 0; i < TC_STAGES && i < it; ++i) {
+                const uint32_t j = it - 1 - i;
+                mbar_wait(&sm->full[j % TC_STAGES], (j / TC_STAGES) & 1, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc_idesc(128, TC_BLOCK_TOKENS);
+            uint32_t it = 0, n = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++n) {
+                const uint32_t acc = n & 1;
+                if (!mbar_wait(&sm->acc_empty[acc], ((n >> 1) & 1) ^ 1, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * 256;
+                for (int kk = 0; kk < nk; ++kk, ++it) {
+                    const uint32_t slot = it % TC_STAGES;
+                    const uint32_t par = (it / TC_STAGES) & 1;
+                    if (!mbar_wait(&sm->full[slot], par, p.status)) { ok = false; break; }
+                    if (INT4 && !mbar_wait(&sm->a_ready[slot], par, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const unsigned char* st = base + slot * TC_STAGE_BYTES;
+                    const uint64_t bd = sw128_desc(st);
+                    const uint64_t ad = sw128_desc(st + TC_B_BYTES);
+#pragma unroll
+                    for (int k16 = 0; k16 < 4; ++k16)   // +32 bytes per 16 K inside the swizzle atom
+                        umma_f16(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (kk | k16) != 0);
+                    umma_commit(&sm->empty[slot]);
+                }
+                if (ok) umma_commit(&sm->acc_full[acc]);
+            }
+            // wind down: wait (bounded) for the last MMAs
+            if (it > 0) mbar_wait(&sm->empty[(it - 1) % TC_STAGES], ((it - 1) / TC_STAGES) & 1, nullptr);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------ epilogue ------------------------------
+        const int ew = warp & 3;                 // TMEM lanes 32 ew .. 32 ew + 31
+        uint32_t n = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++n) {
+            const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
+            const int fb = tile % p.n_fblocks;
+            const uint32_t acc = n & 1;
+            if (!mbar_wait(&sm->acc_full[acc], (n >> 1) & 1, p.status)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem + (uint32_t(32 * ew) << 16) + acc * 256;
+            for (int cc = 0; cc < TC_BLOCK_TOKENS / 32; ++cc) {
+                if (cc * 32 >= ce.count) break;        // warp-uniform
+                uint32_t v[32];
+                tmem_ld32(taddr + cc * 32, v);
+                const int col0 = cc * 32;
+                if (GATEUP) {
+                    // lanes 0..15: gate of features f + 0..15; lanes 16..31: up of the same
+                    const int f = fb * 64 + ew * 16 + (lane & 15);
+                    const int fpos = MODE == TC_GATEUP_INT4 ? (f & ~7) + frag_pos(f & 7) : f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float mine = __uint_as_float(v[j]);
+                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+                        // lanes 0..15 store even columns, lanes 16..31 odd ones
+                        if ((j & 1) == (lane >> 4)) {
+                            const float g = lane < 16 ? mine : other;
+                            const float u = lane < 16 ? other : mine;
+                            const int col = col0 + j;
+                            if (col < ce.count)
+                                p.h_out[int64_t(ce.start + col) * p.n_rows + fpos] = __float2bfloat16_rn(silu_f32(g) * u);
+                        }
+                    }
+                } else if (MODE == TC_DOWN_INT4) {
+                    const int d = fb * 128 + ew * 32 + lane;
+                    const int my_col = col0 + lane;
+                    const float my_gate = my_col < ce.count ? p.gates[p.perm[ce.start + my_col]] : 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float gt = __shfl_sync(0xffffffffu, my_gate, j);
+                        const int col = col0 + j;
+                        if (col < ce.count) p.y_out[int64_t(ce.start + col) * p.n_rows + d] = __uint_as_float(v[j]) * gt;
+                    }
+                } else {
+                    // out[t] = bf16(shared down + sum of the token's gate-scaled routed outputs)
+                    const int d = fb * 128 + ew * 32 + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = col0 + j;
+                        if (col >= ce.count) continue;
+                        const int64_t t = ce.start + col;
+                        float s = __uint_as_float(v[j]);
+                        for (int jj = 0; jj < p.k_top; ++jj)
+                            s += p.y_r[int64_t(p.inv_perm[t * p.k_top + jj]) * p.n_rows + d];
+                        p.out[t * p.n_rows + d] = __float2bfloat16_rn(s);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
+        }
+    } else if (INT4 && warp >= 8) {
+        // ------------------------------ int4 -> bf16 converters ------------------------------
+        const int i = threadIdx.x - 256;                     // A row 0..127
+        int code_row, srow_off;
+        const float* sbase;
+        if (MODE == TC_GATEUP_INT4) {
+            const int blk = i >> 4, local = i & 15;
+            code_row = (blk & 1) ? 64 + (blk >> 1) * 16 + local : (blk >> 1) * 16 + local;
+            srow_off = (blk >> 1) * 16 + local;
+            sbase = (blk & 1) ? p.s1 : p.s0;
+        } else {
+            code_row = i;
+            srow_off = i;
+            sbase = p.s0;
+        }
+        const int ng = p.K / kGroup;
+        const __nv_bfloat162 k136 = __floats2bfloat162_rn(136.0f, 136.0f);
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
+            const int fb = tile % p.n_fblocks;
+            const float* srow = sbase + int64_t(ce.expert * p.n_rows + fb * (GATEUP ? 64 : 128) + srow_off) * ng;
+            float s_next = ldg_f32(srow);
+            bool ok = true;
+            __nv_bfloat162 s2 = __floats2bfloat162_rn(0.f, 0.f);
+            for (int kk = 0; kk < nk; ++kk, ++it) {
+                if ((kk & 1) == 0) {                           // a new group of 128 K
+                    s2 = __floats2bfloat162_rn(s_next, s_next);
+                    const int gn = kk / 2 + 1;
+                    if (gn < ng) s_next = ldg_f32(srow + gn);
+                }
+                const uint32_t slot = it % TC_STAGES;
+                if (!mbar_wait(&sm->full[slot], (it / TC_STAGES) & 1, p.status)) { ok = false; break; }
+                unsigned char* st = base + slot * TC_STAGE_BYTES;
+                unsigned char* sa = st + TC_B_BYTES;
+                const unsigned char* sc = sa + TC_A_BYTES;
+                const uint4 c0 = *reinterpret_cast<const uint4*>(sc + code_row * 32);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(sc + code_row * 32 + 16);
+                const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    // 8 codes k0..k7 -> (k0,k4) (k1,k5) (k2,k6) (k3,k7), each (q * s) in bf16
+                    uint32_t o[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t t = ((w[j] >> (4 * h)) & 0x000F000Fu) ^ 0x43084308u;   // bf16 136 + q
+                        __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&t), k136);
+                        __nv_bfloat162 r = __hmul2(q, s2);
+                        o[h] = *reinterpret_cast<uint32_t*>(&r);
+                    }
+                    *reinterpret_cast<uint4*>(sa + i * 128 + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->a_ready[slot]);
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TC_TMEM_COLS);
+    }
+}
+
+// x_sorted[p] = x[perm[p] / k], every 8 values reordered x0 x4 x1 x5 x2 x6 x3 x7
+__global__ void gather_rows_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ perm, int64_t n,
+                                   int k, int D, bf16* __restrict__ out) {
+    const int chunks = D / 8;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n * chunks;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = i / chunks;
+        const int c = int(i % chunks);
+        const uint4 v = *reinterpret_cast<const uint4*>(x + int64_t(perm[r] / k) * D + 8 * c);
+        uint4 o;
+        o.x = prmt(v.x, v.z, 0x5410); o.y = prmt(v.x, v.z, 0x7632);
+        o.z = prmt(v.y, v.w, 0x5410); o.w = prmt(v.y, v.w, 0x7632);
+        *reinterpret_cast<uint4*>(out + r * D + 8 * c) = o;
+    }
+}
+
+size_t tc_smem_bytes() { return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + sizeof(TcSmem); }
+
+moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = tc_smem_bytes();
+#define TC_LAUNCH(M)                                                                                     \
+    do {                                                                                                 \
+        if (cudaFuncSetAttribute(tc_gemm_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+                                 int(smem)) != cudaSuccess)                                              \
+            return MOE_ERR_CUDA;                                                                         \
+        tc_gemm_kernel<M><<<sms, TC_THREADS, smem, stream>>>(maps.b, maps.a0, maps.a1, prm);           \
+    } while (0)
+    switch (mode) {
+        case TC_GATEUP_INT4: TC_LAUNCH(TC_GATEUP_INT4); break;
+        case TC_DOWN_INT4: TC_LAUNCH(TC_DOWN_INT4); break;
+        case TC_GATEUP_BF16: TC_LAUNCH(TC_GATEUP_BF16); break;
+        default: TC_LAUNCH(TC_COMBINE_BF16); break;
+    }
+#undef TC_LAUNCH
+    return launch_status();
+}
+
+moe_status launch_gather_rows(const bf16* x, const int32_t* perm, int64_t n, int k, int D, bf16* out,
+                              cudaStream_t stream) {
+    if (n == 0) return MOE_OK;
+    int64_t blocks = ceil_div(n * (D / 8), 256);
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    gather_rows_kernel<<<unsigned(blocks), 256, 0, stream>>>(x, perm, n, k, D, out);
+    return launch_status();
+}
+
+}  // namespace moe

@@ -1,0 +1,51 @@
+// tcgen05 (5th-generation tensor core) grouped GEMMs for many tokens per
+// expert: host/device interface.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ffn_decode.cuh"
+
+namespace moe {
+
+enum TcMode : int32_t {
+    TC_GATEUP_INT4 = 0,   // routed gate/up, int4 weights dequantized on chip, SwiGLU -> h (bf16)
+    TC_DOWN_INT4 = 1,     // routed down, int4 weights, gate-scaled fp32 y per slot
+    TC_GATEUP_BF16 = 2,   // shared gate/up, bf16 weights by TMA, SwiGLU -> h (bf16)
+    TC_COMBINE_BF16 = 3   // shared down, bf16 weights, + routed y of the token's slots -> bf16 out
+};
+
+struct TcParams {
+    int32_t K;                 // reduction length
+    int32_t n_rows;            // output features of one expert's matrix (F or D)
+    int32_t n_fblocks;         // feature blocks per token chunk (64 features for gate/up, 128 otherwise)
+    const ChunkEntry* chunks;  // token chunks of <= 256 (shared expert's first)
+    const int32_t* n_chunks;   // [0] all chunks, [1] the shared expert's
+    int32_t routed;            // 1: chunks [n_shared, n_all); 0: chunks [0, n_shared)
+    const float* s0;           // int4 scales [E * rows, K / 128] (gate or down)
+    const float* s1;           // int4 scales (up)
+    bf16* h_out;               // gate/up output rows [*, n_rows] (row = slot position or token)
+    float* y_out;              // routed down output [slots, n_rows] (by position)
+    const float* gates;        // per slot
+    const int32_t* perm;       // position -> slot
+    bf16* out;                 // combine output [T, n_rows]
+    const float* y_r;          // routed y by position
+    const int32_t* inv_perm;   // slot -> position
+    int32_t k_top;
+    int32_t* status;
+};
+
+struct TcMaps {
+    CUtensorMap b;       // tokens: bf16 [rows, K], box 64 x 256, 128-byte swizzle
+    CUtensorMap a0, a1;  // int4 codes uint8 [E * rows, K / 2], box 32 x 64; or bf16 weights, box 64 x 16
+};
+
+constexpr int TC_BLOCK_TOKENS = 256;
+
+size_t tc_smem_bytes();
+moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream);
+moe_status launch_gather_rows(const bf16* x, const int32_t* perm, int64_t n, int k, int D, bf16* out,
+                              cudaStream_t stream);
+
+}  // namespace moe

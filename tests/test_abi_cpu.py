@@ -98,12 +98,12 @@ def test_forward_rejects_small_workspace_and_bad_pointers(lib):
     d = _desc()
     f = 1 << 20
     need = lib.moe_ffn_workspace_size(ctypes.byref(d), 16)
-    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f, need - 256, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f, 4096, None) == S.WORKSPACE_TOO_SMALL
     assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f + 16, need, None) == S.INVALID_ARG  # ws not 256-aligned
     assert lib.moe_ffn_forward(ctypes.byref(d), None, 16, f, f, need, None) == S.INVALID_ARG
     assert lib.moe_ffn_forward(ctypes.byref(d), f, 0, f, f, need, None) == S.UNSUPPORTED_SHAPE
     assert lib.moe_ffn_forward(None, f, 16, f, f, need, None) == S.INVALID_ARG
-    assert lib.moe_ffn_forward_host(ctypes.byref(d), f, 16, f, f, need - 256, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_ffn_forward_host(ctypes.byref(d), f, 16, f, f, 4096, None) == S.WORKSPACE_TOO_SMALL
     assert lib.moe_ffn_device_status(None, None) == S.INVALID_ARG
     ev = (ctypes.c_void_p * 2)(f, f)
     assert lib.moe_ffn_forward_timed(ctypes.byref(d), f, 16, f, f, need, None, ev, 2) == S.INVALID_ARG

@@ -24,23 +24,28 @@ def _run(b, path=moe.PATH_AUTO, tokens=None):
     return got[sel], ref["out"]
 
 
-@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_DECODE])
+@pytest.mark.parametrize("path", [moe.PATH_AUTO, moe.PATH_DECODE, moe.PATH_PREFILL])
 def test_tiny(path):
     b = build(synth.SHAPES["tiny"])
     got, ref = _run(b, path)
     assert rel_err(got, ref) <= TOL
 
 
-@pytest.mark.parametrize("T,D,F,Fs,E,k", [
+RAGGED = [
     (1, 256, 512, 512, 4, 1),        # one token
-    (37, 384, 640, 384, 5, 2),       # ragged: 3 groups along D, 2 token chunks + 5
+    (37, 384, 640, 384, 5, 2),       # ragged: 3 groups along D, token chunks + tail
     (16, 128, 256, 128, 1, 1),       # a single expert
     (50, 256, 384, 256, 6, 3),
     (16, 512, 1024, 768, 16, 1),
-])
-def test_ragged_decode(T, D, F, Fs, E, k):
+    (300, 256, 256, 128, 3, 2),      # more than one 256-token tile per expert
+]
+
+
+@pytest.mark.parametrize("path", [moe.PATH_DECODE, moe.PATH_PREFILL])
+@pytest.mark.parametrize("T,D,F,Fs,E,k", RAGGED)
+def test_ragged(T, D, F, Fs, E, k, path):
     b = build(synth.LayerShape("r", T, D, F, E, k, Fs))
-    got, ref = _run(b, moe.PATH_DECODE)
+    got, ref = _run(b, path)
     assert rel_err(got, ref) <= TOL
 
 
@@ -52,8 +57,9 @@ def test_all_tokens_on_one_expert_and_empty_experts():
     b.gpu.tensors[0].copy_(wr.cuda())
     b.oracle.w_router = wr
     b.x = torch.ones(40, 256, dtype=torch.bfloat16) * torch.linspace(0.5, 1.5, 40).to(torch.bfloat16)[:, None]
-    got, ref = _run(b, moe.PATH_DECODE)
-    assert rel_err(got, ref) <= TOL
+    for path in (moe.PATH_DECODE, moe.PATH_PREFILL):
+        got, ref = _run(b, path)
+        assert rel_err(got, ref) <= TOL
 
 
 def test_repeat_calls_identical():
@@ -79,4 +85,28 @@ def test_scout_decode_full_size():
     every token checked against the oracle."""
     b = build(synth.SHAPES["scout_decode"])
     got, ref = _run(b)
+    assert rel_err(got, ref) <= TOL
+
+
+def _sampled(name, n_tokens, seed=0):
+    shape = synth.SHAPES[name]
+    b = build(shape)
+    rng = np.random.default_rng(seed)
+    tokens = np.sort(rng.choice(shape.T, n_tokens, replace=False))
+    got, ref = _run(b, moe.PATH_AUTO, tokens=tokens)
+    return got, ref
+
+
+@pytest.mark.slow
+def test_scout_prefill_full_size_sampled():
+    """The prefill workload at full size (T=8192) through the tensor-core
+    path, 24 sampled tokens checked against the oracle."""
+    got, ref = _sampled("scout_prefill", 24)
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.slow
+def test_skewed_full_size_sampled():
+    """The Zipf-routed workload at full size (T=32768), 24 sampled tokens."""
+    got, ref = _sampled("skewed", 24, seed=1)
     assert rel_err(got, ref) <= TOL
