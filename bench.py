@@ -41,13 +41,17 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+FALLBACK_BF16_TFLOPS = 1400.0   # sustained under the power cap
+
+
 def peaks():
+    """(HBM GB/s, sustained dense bf16 TFLOP/s, source)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def workload_text(s: synth.LayerShape) -> str:
@@ -138,10 +142,12 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
     return layer, x, (wr, bias)
 
 
-def kernel_bytes(shape: synth.LayerShape, n_touched: int) -> dict:
-    """Algorithmic HBM bytes per launch of each decode-path kernel: every
-    weight byte of a touched expert and of the shared expert read once, every
-    activation read and written once."""
+def kernel_work(shape: synth.LayerShape, n_touched: int) -> dict:
+    """Algorithmic work per launch of each kernel, as (kind, amount):
+    ("bytes", HBM bytes with every weight byte of a touched expert and of the
+    shared expert read once and every activation read and written once) for
+    the weight-streaming kernels, ("flops", 2 * multiply-adds) for the
+    tensor-core ones."""
     T, D, F, Fs, E, k = shape.T, shape.D, shape.F, shape.F_shared, shape.E, shape.k
     S = T * k
     codes_gu = 2 * F * D // 2
@@ -149,13 +155,26 @@ def kernel_bytes(shape: synth.LayerShape, n_touched: int) -> dict:
     codes_d = D * F // 2
     scales_d = D * (F // 128) * 4
     return {
-        "route_topk": T * D * 2 + E * D * 2 + T * D * 2 + S * 8,
-        "bucket": S * 4 * 3 + (E + 1) * 8,
-        "decode_plan": (E + 1) * 8,
-        "decode_gate_up": n_touched * (codes_gu + scales_gu) + 2 * Fs * D * 2 + T * D * 2 + (S * F + T * Fs) * 2,
-        "decode_down": n_touched * (codes_d + scales_d) + D * Fs * 2 + (S * F + T * Fs) * 2 + (S + T) * D * 4,
-        "combine": (S + T) * D * 4 + T * D * 2,
+        "router": ("flops", 2 * T * D * E),
+        "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
+        "act16_x": ("bytes", T * D * 2 * 2),
+        "decode_gate_up": ("bytes", n_touched * (codes_gu + scales_gu) + 2 * Fs * D * 2 + T * D * 2
+                           + (S * F + T * Fs) * 2),
+        "act16_h": ("bytes", S * F * 2 * 2),
+        "decode_down": ("bytes", n_touched * (codes_d + scales_d) + D * Fs * 2 + (S * F + T * Fs) * 2
+                        + (S + T) * D * 4),
+        "combine": ("bytes", (S + T) * D * 4 + T * D * 2),
+        "gather": ("bytes", S * D * 2 * 2),
+        "tc_gate_up": ("flops", 2 * S * D * 2 * F),
+        "tc_down": ("flops", 2 * S * F * D),
+        "tc_shared_gate_up": ("flops", 2 * T * D * 2 * Fs),
+        "tc_shared_down_combine": ("flops", 2 * T * Fs * D),
     }
+
+
+def layer_flops(shape: synth.LayerShape) -> int:
+    T, D, F, Fs, E, k = shape.T, shape.D, shape.F, shape.F_shared, shape.E, shape.k
+    return 2 * T * D * E + 2 * T * k * 3 * D * F + 2 * T * 3 * D * Fs
 
 
 def run_ours(args, rank: int, world: int, dev: torch.device):
@@ -238,12 +257,21 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
-    kb = kernel_bytes(shape, n_touched)
+    work = kernel_work(shape, n_touched)
     dom = int(np.argmax(per_kernel))
     dom_name = names[dom]
-    peak, peak_src = peaks()
-    achieved = kb[dom_name] / (per_kernel[dom] * 1e-3) / 1e9
-    layer_bytes = sum(kb.values())
+    hbm_peak, tc_peak, peak_src = peaks()
+    kind, amount = work[dom_name]
+    if kind == "bytes":
+        roof = {"bound": "hbm", "kernel": dom_name, "achieved": amount / (per_kernel[dom] * 1e-3) / 1e9,
+                "peak": hbm_peak, "peak_source": peak_src + " copy bandwidth", "unit": "GB/s",
+                "traffic": None, "algorithmic_bytes": amount}
+    else:
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": amount / (per_kernel[dom] * 1e-3) / 1e12,
+                "peak": tc_peak, "peak_source": peak_src + " sustained dense bf16", "unit": "TFLOP/s",
+                "traffic": None, "algorithmic_flops": amount}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    layer_bytes = sum(a for kd, a in (work[n] for n in names) if kd == "bytes")
 
     result = {
         "metric": METRIC,
@@ -263,23 +291,13 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
             "weights": "routed int4 g128 (fp32 scales, zero point 0); router and shared bf16",
             "parallelism": "replicas" if world > 1 else "single GPU",
             "experts_touched": n_touched,
-            "l2": "flushed between steps (256 MB write); weights 1.3 GB exceed L2",
+            "l2": "flushed between steps (256 MB write)",
         },
-        "roofline": {
-            "bound": "hbm",
-            "kernel": dom_name,
-            "achieved": achieved,
-            "peak": peak,
-            "peak_source": peak_src,
-            "unit": "GB/s",
-            "frac": achieved / peak,
-            "traffic": None,
-            "algorithmic_bytes": kb[dom_name],
-        },
+        "roofline": roof,
         "layer": {
-            "algorithmic_bytes": layer_bytes,
-            "achieved_gbs": layer_bytes / (ms * 1e-3) / 1e9,
-            "frac_of_peak": layer_bytes / (ms * 1e-3) / 1e9 / peak,
+            "streamed_bytes": layer_bytes,
+            "flops": layer_flops(shape),
+            "tflops": layer_flops(shape) / (ms * 1e-3) / 1e12,
             "per_kernel_ms": {n: float(v) for n, v in zip(names, per_kernel)},
         },
         "e2e": {
@@ -386,7 +404,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="scout_decode", choices=["tiny", "scout_decode"])
+    ap.add_argument("--workload", default="scout_decode",
+                    choices=["tiny", "scout_decode", "scout_prefill", "skewed"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -45,6 +45,7 @@ struct WsLayout {
     size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
     // tensor-core path (row counts padded to whole 256-token tiles)
     size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos;
+    size_t xq, xq_scale, hq, hq_scale;   // e4m3 activations of FP8_ROW layers
     // host staging of moe_ffn_forward_host
     size_t x_in, out;
     size_t total;
@@ -92,7 +93,14 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
         w.y_r = take(S * L.D * 4);
         w.y_s = take(T * L.D * 4);
     } else {
-        w.x_sorted = take(S_pad * L.D * 2);
+        if (L.format == MOE_WEIGHTS_FP8_ROW) {
+            w.xq = take(S_pad * L.D);
+            w.xq_scale = take(S * 4);
+            w.hq = take(S_pad * L.F);
+            w.hq_scale = take(S * 4);
+        } else {
+            w.x_sorted = take(S_pad * L.D * 2);
+        }
         w.h_sorted = take(S_pad * L.F * 2);
         w.x_pad = take(T_pad * L.D * 2);
         w.h_s_pad = take(T_pad * L.F_shared * 2);
@@ -111,6 +119,7 @@ size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
 }
 
 int choose_path(const moe_layer_desc& L, int64_t T) {
+    if (L.format == MOE_WEIGHTS_FP8_ROW) return PATH_SEL_PREFILL;   // e4m3 layers run on tensor-core tiles
     if (L.path == MOE_PATH_DECODE) return PATH_SEL_DECODE;
     if (L.path == MOE_PATH_PREFILL) return PATH_SEL_PREFILL;
     return T * L.k <= 4 * int64_t(L.E) ? PATH_SEL_DECODE : PATH_SEL_PREFILL;
@@ -120,8 +129,9 @@ moe_status check_layer(const moe_layer_desc* L) {
     if (!L) return MOE_ERR_INVALID_ARG;
     if (L->E < 1 || L->E > 256 || L->k < 1 || L->k > L->E || L->k > 8) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!valid_dim(L->D) || !valid_dim(L->F) || !valid_dim(L->F_shared)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (L->format != MOE_WEIGHTS_INT4_G128) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (L->group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->format != MOE_WEIGHTS_INT4_G128 && L->format != MOE_WEIGHTS_FP8_ROW) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->format == MOE_WEIGHTS_INT4_G128 && L->group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->format == MOE_WEIGHTS_FP8_ROW && !(L->act_scale_ub > 0.0f)) return MOE_ERR_INVALID_ARG;
     if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
     const void* ptrs[] = {L->w_router, L->w_gate, L->s_gate, L->w_up, L->s_up, L->w_down, L->s_down,
                           L->ws_gate, L->ws_up, L->ws_down};
@@ -261,6 +271,9 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
 const char* const kPrefillLaunches[] = {"router", "bucket", "gather", "tc_gate_up", "tc_down",
                                         "tc_shared_gate_up", "tc_shared_down_combine"};
 constexpr int32_t kPrefillLaunchCount = 7;
+const char* const kFp8Launches[] = {"router", "bucket", "quantize_x", "tc_gate_up", "quantize_h", "tc_down",
+                                    "tc_shared_gate_up", "tc_shared_down_combine"};
+constexpr int32_t kFp8LaunchCount = 8;
 
 moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
                             const WsLayout& W, cudaStream_t st, Marks& mk) {
@@ -292,7 +305,12 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     ++mk.i;
     if (s != MOE_OK) return s;
     mk.mark(st);
-    s = launch_gather_rows(x, perm, S, L.k, L.D, x_sorted, st);
+    const bool fp8 = L.format == MOE_WEIGHTS_FP8_ROW;
+    if (fp8)   // e4m3 rows of x, written to each token's slot positions
+        s = launch_quantize_fp8_scatter(x, T, L.D, L.act_scale_ub, inv, L.k, at<uint8_t>(ws, W.xq),
+                                        at<float>(ws, W.xq_scale), st);
+    else
+        s = launch_gather_rows(x, perm, S, L.k, L.D, x_sorted, st);
     if (s != MOE_OK) return s;
     // the shared expert reads x through a 256-row tile map: copy it into whole tiles
     if (cudaMemcpyAsync(x_pad, x, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -300,12 +318,20 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
 
     const uint64_t E = uint64_t(L.E);
     TcMaps m_gu, m_dn, m_sgu, m_sdn;
-    bool ok = make_tmap_2d(&m_gu.b, x_sorted, true, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D / 2, E * L.F, 32, 64, false) &&
-              make_tmap_2d(&m_gu.a1, L.w_up, false, L.D / 2, E * L.F, 32, 64, false) &&
-              make_tmap_2d(&m_dn.b, h_sorted, true, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_dn.a0, L.w_down, false, L.F / 2, E * L.D, 32, 64, false) &&
-              make_tmap_2d(&m_sgu.b, x_pad, true, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+    bool ok;
+    if (fp8)
+        ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), false, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D, E * L.F, 128, 16, true) &&
+             make_tmap_2d(&m_gu.a1, L.w_up, false, L.D, E * L.F, 128, 16, true) &&
+             make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), false, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_dn.a0, L.w_down, false, L.F, E * L.D, 128, 16, true);
+    else
+        ok = make_tmap_2d(&m_gu.b, x_sorted, true, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D / 2, E * L.F, 32, 64, false) &&
+             make_tmap_2d(&m_gu.a1, L.w_up, false, L.D / 2, E * L.F, 32, 64, false) &&
+             make_tmap_2d(&m_dn.b, h_sorted, true, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_dn.a0, L.w_down, false, L.F / 2, E * L.D, 32, 64, false);
+    ok = ok && make_tmap_2d(&m_sgu.b, x_pad, true, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
               make_tmap_2d(&m_sgu.a0, L.ws_gate, true, L.D, L.F_shared, 64, 16, true) &&
               make_tmap_2d(&m_sgu.a1, L.ws_up, true, L.D, L.F_shared, 64, 16, true) &&
               make_tmap_2d(&m_sdn.b, h_s, true, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
@@ -324,18 +350,27 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.k_top = L.k;
     p.status = status;
 
-    // routed gate/up -> h (bf16, fragment order, by slot position)
+    // routed gate/up -> h (bf16 by slot position; int4: fragment order, e4m3: natural order)
     p.K = L.D; p.n_rows = L.F; p.n_fblocks = L.F / 64; p.routed = 1;
     p.s0 = L.s_gate; p.s1 = L.s_up; p.h_out = h_sorted;
+    p.tok_scale = fp8 ? at<float>(ws, W.xq_scale) : nullptr;
     mk.mark(st);
-    s = launch_tc_gemm(TC_GATEUP_INT4, m_gu, p, st);
+    s = launch_tc_gemm(fp8 ? TC_GATEUP_FP8 : TC_GATEUP_INT4, m_gu, p, st);
     if (s != MOE_OK) return s;
+    if (fp8) {   // e4m3 rows of h (every expert matmul quantizes its input rows)
+        mk.mark(st);
+        s = launch_quantize_fp8_rows(h_sorted, MOE_DTYPE_BF16, S, L.F, S, L.act_scale_ub, at<uint8_t>(ws, W.hq),
+                                     at<float>(ws, W.hq_scale), st);
+        if (s != MOE_OK) return s;
+    }
     // routed down -> gate * y (fp32, by slot position)
     p.K = L.F; p.n_rows = L.D; p.n_fblocks = L.D / 128;
     p.s0 = L.s_down; p.s1 = nullptr; p.h_out = nullptr; p.y_out = y_pos;
+    p.tok_scale = fp8 ? at<float>(ws, W.hq_scale) : nullptr;
     mk.mark(st);
-    s = launch_tc_gemm(TC_DOWN_INT4, m_dn, p, st);
+    s = launch_tc_gemm(fp8 ? TC_DOWN_FP8 : TC_DOWN_INT4, m_dn, p, st);
     if (s != MOE_OK) return s;
+    p.tok_scale = nullptr;
     // shared gate/up -> h_s (bf16, natural order, by token)
     p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
     p.s0 = nullptr; p.y_out = nullptr; p.h_out = h_s;
@@ -463,7 +498,9 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
                                  void* workspace, size_t workspace_bytes, void* stream, void* const* events,
                                  int32_t n_events) {
     if (!layer) return MOE_ERR_INVALID_ARG;
-    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE ? kDecodeLaunchCount : kPrefillLaunchCount;
+    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE
+                             ? kDecodeLaunchCount
+                             : (layer->format == MOE_WEIGHTS_FP8_ROW ? kFp8LaunchCount : kPrefillLaunchCount);
     if (!events || n_events < need + 1) return MOE_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_events; ++i)
         if (!events[i]) return MOE_ERR_INVALID_ARG;
@@ -476,8 +513,10 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
 int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, const char** names, int32_t max_names) {
     if (check_layer(layer) != MOE_OK || T < 1) return 0;
     const bool dec = choose_path(*layer, T) == PATH_SEL_DECODE;
-    const int32_t n = dec ? kDecodeLaunchCount : kPrefillLaunchCount;
-    for (int32_t i = 0; i < n && i < max_names && names; ++i) names[i] = dec ? kDecodeLaunches[i] : kPrefillLaunches[i];
+    const bool fp8 = layer->format == MOE_WEIGHTS_FP8_ROW;
+    const char* const* list = dec ? kDecodeLaunches : (fp8 ? kFp8Launches : kPrefillLaunches);
+    const int32_t n = dec ? kDecodeLaunchCount : (fp8 ? kFp8LaunchCount : kPrefillLaunchCount);
+    for (int32_t i = 0; i < n && i < max_names && names; ++i) names[i] = list[i];
     return n;
 }
 

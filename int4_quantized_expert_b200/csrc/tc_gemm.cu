@@ -25,6 +25,8 @@
 // int4 unpacking produces; the dot products do not depend on the K order.
 #include <cuda.h>
 
+#include <cuda_fp8.h>
+
 #include "tc_gemm.cuh"
 
 namespace moe {
@@ -69,14 +71,22 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 inputs) or kind::f8f6f4 (e4m3 inputs)
+template <bool FP8>
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                     uint32_t accumulate) {
+    if (FP8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+            :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 // arrive on `bar` once all previously issued tcgen05.mma of this thread complete
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -103,9 +113,11 @@ __device__ __forceinline__ uint64_t sw128_desc(const void* smem) {
     return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+// Instruction descriptor: fp32 D, A and B K-major; bf16 inputs (kind::f16,
+// format code 1) or e4m3 inputs (kind::f8f6f4, format code 0).
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool fp8) {
+    return (1u << 4) | ((fp8 ? 0u : 1u) << 7) | ((fp8 ? 0u : 1u) << 10) | (uint32_t(N >> 3) << 17) |
+           (uint32_t(M >> 4) << 24);
 }
 
 __device__ __forceinline__ int frag_pos(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
@@ -116,7 +128,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a0,
     const __grid_constant__ CUtensorMap tm_a1, TcParams p) {
     constexpr bool INT4 = MODE == TC_GATEUP_INT4 || MODE == TC_DOWN_INT4;
-    constexpr bool GATEUP = MODE == TC_GATEUP_INT4 || MODE == TC_GATEUP_BF16;
+    constexpr bool FP8 = MODE == TC_GATEUP_FP8 || MODE == TC_DOWN_FP8;
+    constexpr bool GATEUP = MODE == TC_GATEUP_INT4 || MODE == TC_GATEUP_BF16 || MODE == TC_GATEUP_FP8;
+    constexpr int KSTEP = FP8 ? 128 : 64;     // K values per 128-byte row of a stage
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -144,7 +158,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     const int n_all = p.n_chunks[0], n_sh = p.n_chunks[1];
     const int c_begin = p.routed ? n_sh : 0, c_end = p.routed ? n_all : n_sh;
     const int n_tiles = (c_end - c_begin) * p.n_fblocks;
-    const int nk = p.K / 64;
+    const int nk = p.K / KSTEP;
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
@@ -163,7 +177,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     unsigned char* sa = st + TC_B_BYTES;
                     unsigned char* sc = sa + TC_A_BYTES;
                     mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES + (INT4 ? TC_C_BYTES : TC_A_BYTES));
-                    tma_load_2d(st, &tm_b, &sm->full[slot], kk * 64, ce.start);
+                    tma_load_2d(st, &tm_b, &sm->full[slot], kk * KSTEP, ce.start);
                     if (MODE == TC_GATEUP_INT4) {
                         const int row = e * p.n_rows + fb * 64;
                         tma_load_2d(sc, &tm_a0, &sm->full[slot], kk * 32, row);
@@ -178,10 +192,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                         for (int b = 0; b < 8; ++b)
                             tma_load_2d(sa + b * 2048, (b & 1) ? &tm_a1 : &tm_a0, &sm->full[slot], kk * 64,
                                         fb * 64 + (b >> 1) * 16);
-                    } else {
+                    } else if (MODE == TC_COMBINE_BF16) {
 #pragma unroll
                         for (int b = 0; b < 8; ++b)
                             tma_load_2d(sa + b * 2048, &tm_a0, &sm->full[slot], kk * 64, fb * 128 + b * 16);
+                    } else if (MODE == TC_GATEUP_FP8) {
+#pragma unroll
+                        for (int b = 0; b < 8; ++b)
+                            tma_load_2d(sa + b * 2048, (b & 1) ? &tm_a1 : &tm_a0, &sm->full[slot], kk * 128,
+                                        e * p.n_rows + fb * 64 + (b >> 1) * 16);
+                    } else {
+#pragma unroll
+                        for (int b = 0; b < 8; ++b)
+                            tma_load_2d(sa + b * 2048, &tm_a0, &sm->full[slot], kk * 128,
+                                        e * p.n_rows + fb * 128 + b * 16);
                     }
                 }
             }
@@ -194,7 +218,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            constexpr uint32_t idesc = tc_idesc(128, TC_BLOCK_TOKENS);
+            constexpr uint32_t idesc = tc_idesc(128, TC_BLOCK_TOKENS, FP8);
             uint32_t it = 0, n = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++n) {
@@ -212,8 +236,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     const uint64_t bd = sw128_desc(st);
                     const uint64_t ad = sw128_desc(st + TC_B_BYTES);
 #pragma unroll
-                    for (int k16 = 0; k16 < 4; ++k16)   // +32 bytes per 16 K inside the swizzle atom
-                        umma_f16(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (kk | k16) != 0);
+                    for (int k16 = 0; k16 < 4; ++k16)   // +32 bytes (16 bf16 / 32 e4m3 K) per MMA inside the swizzle atom
+                        umma<FP8>(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (kk | k16) != 0);
                     umma_commit(&sm->empty[slot]);
                 }
                 if (ok) umma_commit(&sm->acc_full[acc]);
@@ -241,9 +265,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     // lanes 0..15: gate of features f + 0..15; lanes 16..31: up of the same
                     const int f = fb * 64 + ew * 16 + (lane & 15);
                     const int fpos = MODE == TC_GATEUP_INT4 ? (f & ~7) + frag_pos(f & 7) : f;
+                    // e4m3: scale of this lane's weight row, and of each column's token row
+                    float wrow = 1.0f, tcol = 1.0f;
+                    if (FP8) {
+                        wrow = (lane < 16 ? p.s0 : p.s1)[int64_t(ce.expert) * p.n_rows + f];
+                        tcol = col0 + lane < ce.count ? p.tok_scale[ce.start + col0 + lane] : 0.0f;
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float mine = __uint_as_float(v[j]);
+                        float mine = __uint_as_float(v[j]);
+                        if (FP8) mine *= wrow * __shfl_sync(0xffffffffu, tcol, j);
                         const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
                         // lanes 0..15 store even columns, lanes 16..31 odd ones
                         if ((j & 1) == (lane >> 4)) {
@@ -254,28 +285,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                                 p.h_out[int64_t(ce.start + col) * p.n_rows + fpos] = __float2bfloat16_rn(silu_f32(g) * u);
                         }
                     }
-                } else if (MODE == TC_DOWN_INT4) {
+                } else if (MODE == TC_DOWN_INT4 || MODE == TC_DOWN_FP8) {
                     const int d = fb * 128 + ew * 32 + lane;
                     const int my_col = col0 + lane;
-                    const float my_gate = my_col < ce.count ? p.gates[p.perm[ce.start + my_col]] : 0.0f;
+                    float my_gate = my_col < ce.count ? p.gates[p.perm[ce.start + my_col]] : 0.0f;
+                    float wrow = 1.0f;
+                    if (FP8) {   // e4m3: token-row scale folded into the gate, weight-row scale per lane
+                        if (my_col < ce.count) my_gate *= p.tok_scale[ce.start + my_col];
+                        wrow = p.s0[int64_t(ce.expert) * p.n_rows + d];
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float gt = __shfl_sync(0xffffffffu, my_gate, j);
+                        const float gt = __shfl_sync(0xffffffffu, my_gate, j) * wrow;
                         const int col = col0 + j;
                         if (col < ce.count) p.y_out[int64_t(ce.start + col) * p.n_rows + d] = __uint_as_float(v[j]) * gt;
                     }
                 } else {
-                    // out[t] = bf16(shared down + sum of the token's gate-scaled routed outputs)
+                    // out[t] = bf16(shared down + sum of the token's gate-scaled routed outputs);
+                    // lane j first fetches the slot positions of column j's token
                     const int d = fb * 128 + ew * 32 + lane;
+                    int pos[8];
+                    const bool lane_col = col0 + lane < ce.count;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        pos[jj] = (jj < p.k_top && lane_col)
+                                      ? p.inv_perm[int64_t(ce.start + col0 + lane) * p.k_top + jj] : 0;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int col = col0 + j;
-                        if (col >= ce.count) continue;
-                        const int64_t t = ce.start + col;
                         float s = __uint_as_float(v[j]);
-                        for (int jj = 0; jj < p.k_top; ++jj)
-                            s += p.y_r[int64_t(p.inv_perm[t * p.k_top + jj]) * p.n_rows + d];
-                        p.out[t * p.n_rows + d] = __float2bfloat16_rn(s);
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int pp = __shfl_sync(0xffffffffu, pos[jj], j);
+                            if (jj < p.k_top) s += p.y_r[int64_t(pp) * p.n_rows + d];
+                        }
+                        const int col = col0 + j;
+                        if (col < ce.count) p.out[int64_t(ce.start + col) * p.n_rows + d] = __float2bfloat16_rn(s);
                     }
                 }
             }
@@ -367,6 +411,63 @@ __global__ void gather_rows_kernel(const bf16* __restrict__ x, const int32_t* __
     }
 }
 
+// Per-row e4m3 quantization of bf16 x (the same rule as moe_quantize_fp8_rows),
+// each token's codes and scale written to the positions of its k slots.
+__global__ void __launch_bounds__(256) quantize_fp8_scatter_kernel(const bf16* __restrict__ x, int cols,
+                                                                   float scale_ub, const int32_t* __restrict__ inv,
+                                                                   int k, uint8_t* __restrict__ q,
+                                                                   float* __restrict__ scales) {
+    __shared__ float red[8];
+    const int64_t t = blockIdx.x;
+    const bf16* row = x + t * cols;
+    float m = 0.0f;
+    for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+    const float s = __fdiv_rn(fmaxf(fminf(m, scale_ub), 1e-12f), 448.0f);
+    for (int c = threadIdx.x * 8; c < cols; c += 256 * 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + c);
+        const float f[8] = {__fdiv_rn(bf16_lo(v.x), s), __fdiv_rn(bf16_hi(v.x), s), __fdiv_rn(bf16_lo(v.y), s),
+                            __fdiv_rn(bf16_hi(v.y), s), __fdiv_rn(bf16_lo(v.z), s), __fdiv_rn(bf16_hi(v.z), s),
+                            __fdiv_rn(bf16_lo(v.w), s), __fdiv_rn(bf16_hi(v.w), s)};
+        uint32_t o[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * h + 2 * i], f[4 * h + 2 * i + 1]),
+                                                                  __NV_SATFINITE, __NV_E4M3);
+                word |= uint32_t(b) << (16 * i);
+            }
+            o[h] = word;
+        }
+        for (int j = 0; j < k; ++j) {
+            const int64_t pos = inv[t * k + j];
+            *reinterpret_cast<uint2*>(q + pos * cols + c) = make_uint2(o[0], o[1]);
+        }
+    }
+    if (threadIdx.x < k) scales[inv[t * k + threadIdx.x]] = s;
+}
+
+moe_status launch_quantize_fp8_scatter(const bf16* x, int64_t rows, int cols, float scale_ub,
+                                       const int32_t* inv_perm, int k, uint8_t* q, float* scales,
+                                       cudaStream_t stream) {
+    if (rows == 0) return MOE_OK;
+    quantize_fp8_scatter_kernel<<<unsigned(rows), 256, 0, stream>>>(x, cols, scale_ub, inv_perm, k, q, scales);
+    return launch_status();
+}
+
 size_t tc_smem_bytes() { return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + sizeof(TcSmem); }
 
 moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream) {
@@ -385,6 +486,8 @@ moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cud
         case TC_GATEUP_INT4: TC_LAUNCH(TC_GATEUP_INT4); break;
         case TC_DOWN_INT4: TC_LAUNCH(TC_DOWN_INT4); break;
         case TC_GATEUP_BF16: TC_LAUNCH(TC_GATEUP_BF16); break;
+        case TC_GATEUP_FP8: TC_LAUNCH(TC_GATEUP_FP8); break;
+        case TC_DOWN_FP8: TC_LAUNCH(TC_DOWN_FP8); break;
         default: TC_LAUNCH(TC_COMBINE_BF16); break;
     }
 #undef TC_LAUNCH

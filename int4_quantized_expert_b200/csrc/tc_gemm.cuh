@@ -13,7 +13,9 @@ enum TcMode : int32_t {
     TC_GATEUP_INT4 = 0,   // routed gate/up, int4 weights dequantized on chip, SwiGLU -> h (bf16)
     TC_DOWN_INT4 = 1,     // routed down, int4 weights, gate-scaled fp32 y per slot
     TC_GATEUP_BF16 = 2,   // shared gate/up, bf16 weights by TMA, SwiGLU -> h (bf16)
-    TC_COMBINE_BF16 = 3   // shared down, bf16 weights, + routed y of the token's slots -> bf16 out
+    TC_COMBINE_BF16 = 3,  // shared down, bf16 weights, + routed y of the token's slots -> bf16 out
+    TC_GATEUP_FP8 = 4,    // routed gate/up, e4m3 weights and tokens by TMA, row scales -> h (bf16)
+    TC_DOWN_FP8 = 5       // routed down, e4m3 weights and h rows, row scales, gate-scaled fp32 y
 };
 
 struct TcParams {
@@ -23,8 +25,9 @@ struct TcParams {
     const ChunkEntry* chunks;  // token chunks of <= 256 (shared expert's first)
     const int32_t* n_chunks;   // [0] all chunks, [1] the shared expert's
     int32_t routed;            // 1: chunks [n_shared, n_all); 0: chunks [0, n_shared)
-    const float* s0;           // int4 scales [E * rows, K / 128] (gate or down)
-    const float* s1;           // int4 scales (up)
+    const float* s0;           // weight scales (gate or down): int4 [E * rows, K / 128]; e4m3 [E * rows]
+    const float* s1;           // weight scales (up)
+    const float* tok_scale;    // e4m3 modes: row scale of each token row of B (by slot position)
     bf16* h_out;               // gate/up output rows [*, n_rows] (row = slot position or token)
     float* y_out;              // routed down output [slots, n_rows] (by position)
     const float* gates;        // per slot
@@ -38,13 +41,17 @@ struct TcParams {
 
 struct TcMaps {
     CUtensorMap b;       // tokens: bf16 [rows, K], box 64 x 256, 128-byte swizzle
-    CUtensorMap a0, a1;  // int4 codes uint8 [E * rows, K / 2], box 32 x 64; or bf16 weights, box 64 x 16
+    CUtensorMap a0, a1;  // int4 codes uint8 [E * rows, K / 2], box 32 x 64; bf16 weights, box 64 x 16;
+                         // or e4m3 weights uint8 [E * rows, K], box 128 x 16
 };
 
 constexpr int TC_BLOCK_TOKENS = 256;
 
 size_t tc_smem_bytes();
 moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream);
+moe_status launch_quantize_fp8_scatter(const bf16* x, int64_t rows, int cols, float scale_ub,
+                                       const int32_t* inv_perm, int k, uint8_t* q, float* scales,
+                                       cudaStream_t stream);
 moe_status launch_gather_rows(const bf16* x, const int32_t* perm, int64_t n, int k, int D, bf16* out,
                               cudaStream_t stream);
 

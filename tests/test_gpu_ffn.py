@@ -110,3 +110,27 @@ def test_skewed_full_size_sampled():
     """The Zipf-routed workload at full size (T=32768), 24 sampled tokens."""
     got, ref = _sampled("skewed", 24, seed=1)
     assert rel_err(got, ref) <= TOL
+
+
+FP8_SHAPES = [
+    synth.LayerShape("fp8_tiny", 64, 256, 512, 8, 2, 256, "fp8"),
+    synth.LayerShape("fp8_ragged", 37, 384, 640, 5, 3, 384, "fp8"),
+    synth.LayerShape("fp8_one", 1, 256, 256, 4, 4, 128, "fp8"),
+]
+
+
+@pytest.mark.parametrize("shape", FP8_SHAPES, ids=lambda s: s.name)
+def test_fp8_layers(shape):
+    """e4m3 row-quantized experts (weights and every expert input), bf16
+    shared expert, softmax over the top-k gates."""
+    b = build(shape)
+    got, ref = _run(b)
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.slow
+def test_maverick_fp8_full_size_sampled():
+    """The Maverick-shaped FP8 layer at full size (T=4096, 128 experts, top-8),
+    8 sampled tokens (up to 64 experts) checked against the oracle."""
+    got, ref = _sampled("maverick_fp8", 8, seed=2)
+    assert rel_err(got, ref) <= TOL
