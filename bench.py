@@ -54,6 +54,39 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+KERNEL_SOURCES = {   # the files a kernel's code comes from (a change invalidates its ncu numbers)
+    "decode_gate_up": ["ffn_decode.cu", "ffn_decode.cuh", "common.cuh"],
+    "decode_down": ["ffn_decode.cu", "ffn_decode.cuh", "common.cuh"],
+    "tc_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
+    "tc_down": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
+    "tc_shared_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
+    "tc_shared_down": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "int4_quantized_expert_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu summary, or None if absent or taken on another source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return e["dram_bytes"]
+
+
 def workload_text(s: synth.LayerShape) -> str:
     w = "int4 g128" if s.fmt == "int4" else "fp8 e4m3 rows"
     gate = "sigmoid" if s.k == 1 else "softmax over top-%d" % s.k
@@ -129,15 +162,23 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
     bias = synth.router_bias(shape)
     bias = None if bias is None else torch.from_numpy(bias).to(dev)
     sg, su, sd = (t.to(dev) for t in synth.shared_weights(seed, D, Fs))
-    alloc = lambda n, kk: (torch.empty(E, n, kk // 2, dtype=torch.uint8, device=dev),
-                           torch.empty(E, n, kk // 128, dtype=torch.float32, device=dev))
+    if shape.fmt == "int4":
+        alloc = lambda n, kk: (torch.empty(E, n, kk // 2, dtype=torch.uint8, device=dev),
+                               torch.empty(E, n, kk // 128, dtype=torch.float32, device=dev))
+        quant = lambda w, out: moe.quantize_int4(w, out=out)
+        fmt = moe.FMT_INT4
+    else:
+        alloc = lambda n, kk: (torch.empty(E, n, kk, dtype=torch.uint8, device=dev),
+                               torch.empty(E, n, dtype=torch.float32, device=dev))
+        quant = lambda w, out: moe.quantize_fp8_rows(w, out=out)
+        fmt = moe.FMT_FP8
     gate, up, down = alloc(F, D), alloc(F, D), alloc(D, F)
-    for e, g, u, d in synth.iter_expert_weights(seed, range(E), D, F):
+    for e, g, u, d in synth.iter_expert_weights(seed, range(E), D, F, workers=min(16, os.cpu_count() or 1)):
         for w, (c, s) in ((g, gate), (u, up), (d, down)):
-            moe.quantize_int4(torch.from_numpy(w).to(dev), out=(c[e], s[e]))
+            quant(torch.from_numpy(w).to(dev), (c[e], s[e]))
     torch.cuda.synchronize()
     layer = moe.MoELayer(E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr, router_bias=bias, gate=gate,
-                         up=up, down=down, shared=(sg, su, sd), T_max=shape.T)
+                         up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T)
     x = synth.tokens(seed, shape.T, D).to(dev)
     return layer, x, (wr, bias)
 
@@ -154,6 +195,18 @@ def kernel_work(shape: synth.LayerShape, n_touched: int) -> dict:
     scales_gu = 2 * F * (D // 128) * 4
     codes_d = D * F // 2
     scales_d = D * (F // 128) * 4
+    if shape.fmt == "fp8":   # e4m3 routed experts: one tensor-core pass each, bf16-equivalent flop count
+        return {
+            "router": ("flops", 2 * T * D * E),
+            "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
+            "quantize_x": ("bytes", T * D * 2 + S * D),
+            "tc_gate_up": ("flops", 2 * S * D * 2 * F),
+            "quantize_h": ("bytes", S * F * 2 * 2 + S * F),
+            "tc_down": ("flops", 2 * S * F * D),
+            "tc_shared_gate_up": ("flops", 2 * T * D * 2 * Fs),
+            "tc_shared_down": ("flops", 2 * T * Fs * D),
+            "combine": ("bytes", (S + T) * D * 4 + T * D * 2),
+        }
     return {
         "router": ("flops", 2 * T * D * E),
         "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
@@ -168,7 +221,7 @@ def kernel_work(shape: synth.LayerShape, n_touched: int) -> dict:
         "tc_gate_up": ("flops", 2 * S * D * 2 * F),
         "tc_down": ("flops", 2 * S * F * D),
         "tc_shared_gate_up": ("flops", 2 * T * D * 2 * Fs),
-        "tc_shared_down_combine": ("flops", 2 * T * Fs * D),
+        "tc_shared_down": ("flops", 2 * T * Fs * D),
     }
 
 
@@ -267,10 +320,14 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
                 "peak": hbm_peak, "peak_source": peak_src + " copy bandwidth", "unit": "GB/s",
                 "traffic": None, "algorithmic_bytes": amount}
     else:
+        fp8_kernel = shape.fmt == "fp8" and dom_name in ("tc_gate_up", "tc_down")
+        peak = tc_peak * (2.0 if fp8_kernel else 1.0)   # e4m3: nominal 2x the bf16 rate
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": amount / (per_kernel[dom] * 1e-3) / 1e12,
-                "peak": tc_peak, "peak_source": peak_src + " sustained dense bf16", "unit": "TFLOP/s",
-                "traffic": None, "algorithmic_flops": amount}
+                "peak": peak, "unit": "TFLOP/s", "traffic": None, "algorithmic_flops": amount,
+                "peak_source": peak_src + (" sustained dense bf16 x 2 (e4m3)" if fp8_kernel
+                                           else " sustained dense bf16")}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(dom_name, shape.name)
     layer_bytes = sum(a for kd, a in (work[n] for n in names) if kd == "bytes")
 
     result = {
@@ -405,7 +462,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scout_decode",
-                    choices=["tiny", "scout_decode", "scout_prefill", "skewed"])
+                    choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -44,7 +44,7 @@ struct WsLayout {
     // weight-streaming path
     size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
     // tensor-core path (row counts padded to whole 256-token tiles)
-    size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos;
+    size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos, y_shared;
     size_t xq, xq_scale, hq, hq_scale;   // e4m3 activations of FP8_ROW layers
     // host staging of moe_ffn_forward_host
     size_t x_in, out;
@@ -105,6 +105,7 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
         w.x_pad = take(T_pad * L.D * 2);
         w.h_s_pad = take(T_pad * L.F_shared * 2);
         w.y_pos = take(S * L.D * 4);
+        w.y_shared = take(T * L.D * 4);
     }
     w.x_in = take(T * L.D * 2);
     w.out = take(T * L.D * 2);
@@ -268,12 +269,24 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     return s;
 }
 
-const char* const kPrefillLaunches[] = {"router", "bucket", "gather", "tc_gate_up", "tc_down",
-                                        "tc_shared_gate_up", "tc_shared_down_combine"};
-constexpr int32_t kPrefillLaunchCount = 7;
-const char* const kFp8Launches[] = {"router", "bucket", "quantize_x", "tc_gate_up", "quantize_h", "tc_down",
-                                    "tc_shared_gate_up", "tc_shared_down_combine"};
-constexpr int32_t kFp8LaunchCount = 8;
+// Kernel launches of the tensor-core path, in order (the combine only when a
+// token has more than one routed slot).
+int prefill_launches(const moe_layer_desc& L, const char** names, int max_names) {
+    const bool fp8 = L.format == MOE_WEIGHTS_FP8_ROW;
+    const char* list[9];
+    int n = 0;
+    list[n++] = "router";
+    list[n++] = "bucket";
+    list[n++] = fp8 ? "quantize_x" : "gather";
+    list[n++] = "tc_shared_gate_up";
+    list[n++] = "tc_shared_down";
+    list[n++] = "tc_gate_up";
+    if (fp8) list[n++] = "quantize_h";
+    list[n++] = "tc_down";
+    if (L.k > 1) list[n++] = "combine";
+    for (int i = 0; i < n && i < max_names && names; ++i) names[i] = list[i];
+    return n;
+}
 
 moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
                             const WsLayout& W, cudaStream_t st, Marks& mk) {
@@ -349,10 +362,23 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.inv_perm = inv;
     p.k_top = L.k;
     p.status = status;
+    float* y_shared = at<float>(ws, W.y_shared);
 
+    // shared gate/up -> h_s (bf16, natural order, by token)
+    p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
+    p.h_out = h_s;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_GATEUP_BF16, m_sgu, p, st);
+    if (s != MOE_OK) return s;
+    // shared down -> y_s (fp32, by token)
+    p.K = L.F_shared; p.n_rows = L.D; p.n_fblocks = L.D / 128;
+    p.h_out = nullptr; p.y_out = y_shared;
+    mk.mark(st);
+    s = launch_tc_gemm(TC_DOWN_BF16, m_sdn, p, st);
+    if (s != MOE_OK) return s;
     // routed gate/up -> h (bf16 by slot position; int4: fragment order, e4m3: natural order)
     p.K = L.D; p.n_rows = L.F; p.n_fblocks = L.F / 64; p.routed = 1;
-    p.s0 = L.s_gate; p.s1 = L.s_up; p.h_out = h_sorted;
+    p.s0 = L.s_gate; p.s1 = L.s_up; p.h_out = h_sorted; p.y_out = nullptr;
     p.tok_scale = fp8 ? at<float>(ws, W.xq_scale) : nullptr;
     mk.mark(st);
     s = launch_tc_gemm(fp8 ? TC_GATEUP_FP8 : TC_GATEUP_INT4, m_gu, p, st);
@@ -363,25 +389,20 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
                                      at<float>(ws, W.hq_scale), st);
         if (s != MOE_OK) return s;
     }
-    // routed down -> gate * y (fp32, by slot position)
+    // routed down: with one slot per token it finishes the layer (shared + gate * y);
+    // otherwise gate * y by slot, summed per token by the combine
     p.K = L.F; p.n_rows = L.D; p.n_fblocks = L.D / 128;
-    p.s0 = L.s_down; p.s1 = nullptr; p.h_out = nullptr; p.y_out = y_pos;
+    p.s0 = L.s_down; p.s1 = nullptr; p.h_out = nullptr;
     p.tok_scale = fp8 ? at<float>(ws, W.hq_scale) : nullptr;
+    if (L.k == 1) { p.out = out; p.y_r = y_shared; p.y_out = nullptr; }
+    else { p.out = nullptr; p.y_r = nullptr; p.y_out = y_pos; }
     mk.mark(st);
     s = launch_tc_gemm(fp8 ? TC_DOWN_FP8 : TC_DOWN_INT4, m_dn, p, st);
     if (s != MOE_OK) return s;
-    p.tok_scale = nullptr;
-    // shared gate/up -> h_s (bf16, natural order, by token)
-    p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
-    p.s0 = nullptr; p.y_out = nullptr; p.h_out = h_s;
-    mk.mark(st);
-    s = launch_tc_gemm(TC_GATEUP_BF16, m_sgu, p, st);
-    if (s != MOE_OK) return s;
-    // shared down + the routed outputs of each token -> out
-    p.K = L.F_shared; p.n_rows = L.D; p.n_fblocks = L.D / 128;
-    p.h_out = nullptr; p.out = out; p.y_r = y_pos;
-    mk.mark(st);
-    s = launch_tc_gemm(TC_COMBINE_BF16, m_sdn, p, st);
+    if (L.k > 1) {
+        mk.mark(st);
+        s = launch_combine_slots(y_shared, y_pos, T, L.D, L.k, out, st);
+    }
     mk.mark(st);
     return s;
 }
@@ -498,9 +519,8 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
                                  void* workspace, size_t workspace_bytes, void* stream, void* const* events,
                                  int32_t n_events) {
     if (!layer) return MOE_ERR_INVALID_ARG;
-    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE
-                             ? kDecodeLaunchCount
-                             : (layer->format == MOE_WEIGHTS_FP8_ROW ? kFp8LaunchCount : kPrefillLaunchCount);
+    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE ? kDecodeLaunchCount
+                                                                   : prefill_launches(*layer, nullptr, 0);
     if (!events || n_events < need + 1) return MOE_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_events; ++i)
         if (!events[i]) return MOE_ERR_INVALID_ARG;
@@ -512,12 +532,9 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
 
 int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, const char** names, int32_t max_names) {
     if (check_layer(layer) != MOE_OK || T < 1) return 0;
-    const bool dec = choose_path(*layer, T) == PATH_SEL_DECODE;
-    const bool fp8 = layer->format == MOE_WEIGHTS_FP8_ROW;
-    const char* const* list = dec ? kDecodeLaunches : (fp8 ? kFp8Launches : kPrefillLaunches);
-    const int32_t n = dec ? kDecodeLaunchCount : (fp8 ? kFp8LaunchCount : kPrefillLaunchCount);
-    for (int32_t i = 0; i < n && i < max_names && names; ++i) names[i] = list[i];
-    return n;
+    if (choose_path(*layer, T) != PATH_SEL_DECODE) return prefill_launches(*layer, names, max_names);
+    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
+    return kDecodeLaunchCount;
 }
 
 moe_status moe_ffn_device_status(const void* workspace, void* stream) {

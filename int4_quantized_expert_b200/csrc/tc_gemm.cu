@@ -122,6 +122,23 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool fp8) {
 
 __device__ __forceinline__ int frag_pos(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
 
+// Tile order: feature blocks in groups of 16; within a group, chunk by chunk.
+// A wave of ~148 concurrent tiles then touches ~9 token chunks and 16 weight
+// blocks, which stay in L2, instead of every weight block of one chunk.
+constexpr int TC_FB_GROUP = 16;
+__device__ __forceinline__ void tile_coords(int tile, int n_chunks, int n_fblocks, int& chunk, int& fb) {
+    const int gf = min(TC_FB_GROUP, n_fblocks);
+    const int n_groups = (n_fblocks + gf - 1) / gf;
+    const int g = min(tile / (n_chunks * gf), n_groups - 1);
+    const int r = tile - g * n_chunks * gf;
+    const int gsize = min(gf, n_fblocks - g * gf);
+    chunk = r / gsize;
+    fb = g * gf + r % gsize;
+}
+
+// N of the MMA for a chunk of `count` tokens: whole multiples of 16 columns.
+__device__ __forceinline__ int tile_n(int count) { return min(TC_BLOCK_TOKENS, (count + 15) & ~15); }
+
 // ---------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
@@ -167,8 +184,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
-                const int fb = tile % p.n_fblocks;
+                int ci, fb;
+                tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
+                const ChunkEntry ce = p.chunks[c_begin + ci];
                 const int e = ce.expert < 0 ? 0 : ce.expert;
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const uint32_t slot = it % TC_STAGES;
@@ -192,7 +210,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                         for (int b = 0; b < 8; ++b)
                             tma_load_2d(sa + b * 2048, (b & 1) ? &tm_a1 : &tm_a0, &sm->full[slot], kk * 64,
                                         fb * 64 + (b >> 1) * 16);
-                    } else if (MODE == TC_COMBINE_BF16) {
+                    } else if (MODE == TC_DOWN_BF16) {
 #pragma unroll
                         for (int b = 0; b < 8; ++b)
                             tma_load_2d(sa + b * 2048, &tm_a0, &sm->full[slot], kk * 64, fb * 128 + b * 16);
@@ -218,10 +236,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            constexpr uint32_t idesc = tc_idesc(128, TC_BLOCK_TOKENS, FP8);
             uint32_t it = 0, n = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++n) {
+                int ci, fb;
+                tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
+                // a partial chunk multiplies only its tokens' columns (rounded up to 16)
+                const uint32_t idesc = tc_idesc(128, tile_n(p.chunks[c_begin + ci].count), FP8);
                 const uint32_t acc = n & 1;
                 if (!mbar_wait(&sm->acc_empty[acc], ((n >> 1) & 1) ^ 1, p.status)) { ok = false; break; }
                 tc_fence_after();
@@ -250,8 +271,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         const int ew = warp & 3;                 // TMEM lanes 32 ew .. 32 ew + 31
         uint32_t n = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++n) {
-            const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
-            const int fb = tile % p.n_fblocks;
+            int ci, fb;
+            tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
+            const ChunkEntry ce = p.chunks[c_begin + ci];
             const uint32_t acc = n & 1;
             if (!mbar_wait(&sm->acc_full[acc], (n >> 1) & 1, p.status)) break;
             tc_fence_after();
@@ -288,38 +310,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 } else if (MODE == TC_DOWN_INT4 || MODE == TC_DOWN_FP8) {
                     const int d = fb * 128 + ew * 32 + lane;
                     const int my_col = col0 + lane;
-                    float my_gate = my_col < ce.count ? p.gates[p.perm[ce.start + my_col]] : 0.0f;
+                    const int my_slot = my_col < ce.count ? p.perm[ce.start + my_col] : 0;
+                    float my_gate = my_col < ce.count ? p.gates[my_slot] : 0.0f;
                     float wrow = 1.0f;
                     if (FP8) {   // e4m3: token-row scale folded into the gate, weight-row scale per lane
                         if (my_col < ce.count) my_gate *= p.tok_scale[ce.start + my_col];
                         wrow = p.s0[int64_t(ce.expert) * p.n_rows + d];
                     }
+                    if (p.out != nullptr) {
+                        // one slot per token: finish the token here,
+                        // out[t] = bf16(shared expert + gate * y), t = slot
+                        float ys[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float gt = __shfl_sync(0xffffffffu, my_gate, j) * wrow;
-                        const int col = col0 + j;
-                        if (col < ce.count) p.y_out[int64_t(ce.start + col) * p.n_rows + d] = __uint_as_float(v[j]) * gt;
+                        for (int j = 0; j < 32; ++j) {   // all loads first, one latency per 32 columns
+                            const int slot = __shfl_sync(0xffffffffu, my_slot, j);
+                            ys[j] = col0 + j < ce.count ? p.y_r[int64_t(slot) * p.n_rows + d] : 0.0f;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float gt = __shfl_sync(0xffffffffu, my_gate, j) * wrow;
+                            const int slot = __shfl_sync(0xffffffffu, my_slot, j);
+                            if (col0 + j < ce.count)
+                                p.out[int64_t(slot) * p.n_rows + d] = __float2bfloat16_rn(fmaf(__uint_as_float(v[j]), gt, ys[j]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            // y is stored by slot (t k + j), so the combine reads it without indirection
+                            const float gt = __shfl_sync(0xffffffffu, my_gate, j) * wrow;
+                            const int slot = __shfl_sync(0xffffffffu, my_slot, j);
+                            if (col0 + j < ce.count) p.y_out[int64_t(slot) * p.n_rows + d] = __uint_as_float(v[j]) * gt;
+                        }
                     }
                 } else {
-                    // out[t] = bf16(shared down + sum of the token's gate-scaled routed outputs);
-                    // lane j first fetches the slot positions of column j's token
+                    // shared expert's down projection: fp32 y_s[t] (read by the routed down
+                    // projection or the combine)
                     const int d = fb * 128 + ew * 32 + lane;
-                    int pos[8];
-                    const bool lane_col = col0 + lane < ce.count;
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
-                        pos[jj] = (jj < p.k_top && lane_col)
-                                      ? p.inv_perm[int64_t(ce.start + col0 + lane) * p.k_top + jj] : 0;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        float s = __uint_as_float(v[j]);
-#pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) {
-                            const int pp = __shfl_sync(0xffffffffu, pos[jj], j);
-                            if (jj < p.k_top) s += p.y_r[int64_t(pp) * p.n_rows + d];
-                        }
                         const int col = col0 + j;
-                        if (col < ce.count) p.out[int64_t(ce.start + col) * p.n_rows + d] = __float2bfloat16_rn(s);
+                        if (col < ce.count) p.y_out[int64_t(ce.start + col) * p.n_rows + d] = __uint_as_float(v[j]);
                     }
                 }
             }
@@ -346,8 +376,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         const __nv_bfloat162 k136 = __floats2bfloat162_rn(136.0f, 136.0f);
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            const ChunkEntry ce = p.chunks[c_begin + tile / p.n_fblocks];
-            const int fb = tile % p.n_fblocks;
+            int ci, fb;
+            tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
+            const ChunkEntry ce = p.chunks[c_begin + ci];
             const float* srow = sbase + int64_t(ce.expert * p.n_rows + fb * (GATEUP ? 64 : 128) + srow_off) * ng;
             float s_next = ldg_f32(srow);
             bool ok = true;
@@ -468,6 +499,33 @@ moe_status launch_quantize_fp8_scatter(const bf16* x, int64_t rows, int cols, fl
     return launch_status();
 }
 
+// out[t] = bf16(y_s[t] + sum_j y[t k + j])  (routed outputs stored by slot)
+__global__ void combine_slots_kernel(const float* __restrict__ y_s, const float* __restrict__ y, int64_t T, int D,
+                                     int k, bf16* __restrict__ out) {
+    const int64_t n4 = T * D / 4;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = i / (D / 4);
+        const int d = int(i % (D / 4)) * 4;
+        float4 a = *reinterpret_cast<const float4*>(y_s + t * D + d);
+        for (int j = 0; j < k; ++j) {
+            const float4 b = *reinterpret_cast<const float4*>(y + (t * k + j) * D + d);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(a.x, a.y);
+        o.y = pack_bf16x2(a.z, a.w);
+        *reinterpret_cast<uint2*>(out + t * D + d) = o;
+    }
+}
+
+moe_status launch_combine_slots(const float* y_s, const float* y, int64_t T, int D, int k, bf16* out,
+                                cudaStream_t stream) {
+    int64_t blocks = ceil_div(T * D / 4, 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    combine_slots_kernel<<<unsigned(blocks), 256, 0, stream>>>(y_s, y, T, D, k, out);
+    return launch_status();
+}
+
 size_t tc_smem_bytes() { return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + sizeof(TcSmem); }
 
 moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream) {
@@ -488,7 +546,7 @@ moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cud
         case TC_GATEUP_BF16: TC_LAUNCH(TC_GATEUP_BF16); break;
         case TC_GATEUP_FP8: TC_LAUNCH(TC_GATEUP_FP8); break;
         case TC_DOWN_FP8: TC_LAUNCH(TC_DOWN_FP8); break;
-        default: TC_LAUNCH(TC_COMBINE_BF16); break;
+        default: TC_LAUNCH(TC_DOWN_BF16); break;
     }
 #undef TC_LAUNCH
     return launch_status();

@@ -13,7 +13,7 @@ enum TcMode : int32_t {
     TC_GATEUP_INT4 = 0,   // routed gate/up, int4 weights dequantized on chip, SwiGLU -> h (bf16)
     TC_DOWN_INT4 = 1,     // routed down, int4 weights, gate-scaled fp32 y per slot
     TC_GATEUP_BF16 = 2,   // shared gate/up, bf16 weights by TMA, SwiGLU -> h (bf16)
-    TC_COMBINE_BF16 = 3,  // shared down, bf16 weights, + routed y of the token's slots -> bf16 out
+    TC_DOWN_BF16 = 3,     // shared down, bf16 weights -> fp32 y_s [T, D]
     TC_GATEUP_FP8 = 4,    // routed gate/up, e4m3 weights and tokens by TMA, row scales -> h (bf16)
     TC_DOWN_FP8 = 5       // routed down, e4m3 weights and h rows, row scales, gate-scaled fp32 y
 };
@@ -29,11 +29,11 @@ struct TcParams {
     const float* s1;           // weight scales (up)
     const float* tok_scale;    // e4m3 modes: row scale of each token row of B (by slot position)
     bf16* h_out;               // gate/up output rows [*, n_rows] (row = slot position or token)
-    float* y_out;              // routed down output [slots, n_rows] (by position)
+    float* y_out;              // down output: routed [slots, n_rows] by slot t * k + j; shared [T, n_rows]
     const float* gates;        // per slot
     const int32_t* perm;       // position -> slot
-    bf16* out;                 // combine output [T, n_rows]
-    const float* y_r;          // routed y by position
+    bf16* out;                 // routed down with one slot per token: the layer output [T, n_rows]
+    const float* y_r;          // ... and the shared expert's y_s it adds
     const int32_t* inv_perm;   // slot -> position
     int32_t k_top;
     int32_t* status;
@@ -52,6 +52,8 @@ moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cud
 moe_status launch_quantize_fp8_scatter(const bf16* x, int64_t rows, int cols, float scale_ub,
                                        const int32_t* inv_perm, int k, uint8_t* q, float* scales,
                                        cudaStream_t stream);
+moe_status launch_combine_slots(const float* y_s, const float* y, int64_t T, int D, int k, bf16* out,
+                                cudaStream_t stream);
 moe_status launch_gather_rows(const bf16* x, const int32_t* perm, int64_t n, int k, int D, bf16* out,
                               cudaStream_t stream);
 
