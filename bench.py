@@ -1,13 +1,17 @@
 """Benchmark of the int4 mixture-of-experts FFN layer (libmoe_int4) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload scout_decode]
+                    [--workload scout_decode|scout_prefill|skewed|maverick_fp8|tiny|quantize]
 
 One step = one full layer forward (routing, bucketing, routed SwiGLU experts,
 shared expert, weighted combine) over one batch of synthetic tokens already
 resident in HBM.  For N > 1 (launched by torch.distributed.run) every rank
 runs an independent replica of the workload (the layer does not shard), and
 the reported throughput is all ranks' tokens over the slowest rank's time.
+
+``--workload quantize`` instead times int4_row_quantize of a 16-expert
+Scout-shaped weight set (gate and up [8192, 5120], down [5120, 8192] per
+expert, fp32), one step = all three projections, reported in GB/s moved.
 
 ``--impl reference`` times the CPU oracle (the plain numpy restatement of the
 layer) on rank 0 on a bounded sample of the same workload; other ranks exit.
@@ -85,6 +89,37 @@ def ncu_traffic(kernel: str, workload: str):
     if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e["dram_bytes"]
+
+
+QUANT_E, QUANT_D, QUANT_F = 16, 5120, 8192
+QUANT_METRIC = "int4_row_quantize GB/s moved (fp32 weights read, int4 codes and fp32 scales written); % of HBM roofline"
+
+
+def quant_matrices():
+    """(name, rows, cols) of the quantize workload: each projection of all
+    16 experts as one [E * N, K] matrix."""
+    E, D, F = QUANT_E, QUANT_D, QUANT_F
+    return [("gate", E * F, D), ("up", E * F, D), ("down", E * D, F)]
+
+
+def quant_bytes(rows: int, cols: int) -> int:
+    """Algorithmic bytes of int4_row_quantize: fp32 in, codes + scales out."""
+    return rows * cols * 4 + rows * cols // 2 + rows * (cols // 128) * 4
+
+
+def max_over_ranks(values, dev, world: int):
+    """Element-wise max of per-rank floats (all ranks call it, in the same order)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weights_text(s: synth.LayerShape) -> str:
+    if s.fmt == "int4":
+        return "routed int4 g128 (fp32 scales, zero point 0); router and shared bf16"
+    return "routed e4m3 rows (fp32 row scales), e4m3 per-row activations; router and shared bf16"
 
 
 def workload_text(s: synth.LayerShape) -> str:
@@ -280,11 +315,7 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
             per_kernel[j] += evs[j].elapsed_time(evs[j + 1])
         step_ms[i] = evs[0].elapsed_time(evs[-1])
     per_kernel /= args.steps
-    ms = float(step_ms.mean())
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([float(step_ms.mean())], dev, world)[0]
 
     # end to end through the host-buffer entry point (copies inside the timed region)
     xh = x.cpu().pin_memory()
@@ -304,11 +335,7 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-    e2e_ms /= n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks([e2e_ms / n_e2e], dev, world)[0]
 
     work = kernel_work(shape, n_touched)
     dom = int(np.argmax(per_kernel))
@@ -341,11 +368,11 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if shape.fmt == "int4" else "e4m3 (routed experts), bf16 (shared expert)",
         "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
         "config": {
             "workload": workload_text(shape),
-            "weights": "routed int4 g128 (fp32 scales, zero point 0); router and shared bf16",
+            "weights": weights_text(shape),
             "parallelism": "replicas" if world > 1 else "single GPU",
             "experts_touched": n_touched,
             "l2": "flushed between steps (256 MB write)",
@@ -368,6 +395,124 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         "clocks": clocks,
     }
     return result, shape
+
+
+# ---------------------------------------------------------------------------
+# the quantize workload (int4_row_quantize of a 16-expert weight set)
+# ---------------------------------------------------------------------------
+def run_quantize(args, rank: int, world: int, dev: torch.device):
+    import int4_quantized_expert_b200 as moe
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed * 1000 + rank)
+    mats = []
+    for name, rows, cols in quant_matrices():
+        w = torch.randn(rows, cols, generator=gen, device=dev, dtype=torch.float32).mul_(synth.WEIGHT_STD)
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(rows, cols // 128, dtype=torch.float32, device=dev)
+        mats.append((name, w, codes, scales))
+    step_bytes = sum(quant_bytes(w.shape[0], w.shape[1]) for _, w, _, _ in mats)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for _, w, c, sc in mats:
+            moe.quantize_int4(w, out=(c, sc))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for e0, e1 in evs:          # inputs (8 GB) far exceed L2: no flush needed
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.summary(t0, t1) if sampler else None
+    if sampler:
+        sampler.stop()
+    ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in evs]))], dev, world)[0]
+
+    # end to end: each projection's fp32 weights from pinned host memory, its
+    # codes and scales back to pinned host memory, inside the timed region
+    host = [(w.cpu().pin_memory(), torch.empty_like(c, device="cpu").pin_memory(),
+             torch.empty_like(sc, device="cpu").pin_memory()) for _, w, c, sc in mats]
+    n_e2e = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(n_e2e + 1):
+        e0.record(stream)
+        for (_, w, c, sc), (wh, ch, sh) in zip(mats, host):
+            w.copy_(wh, non_blocking=True)
+            moe.quantize_int4(w, out=(c, sc))
+            ch.copy_(c, non_blocking=True)
+            sh.copy_(sc, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i > 0:                # the first pass is a warm-up
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks([e2e_ms / n_e2e], dev, world)[0]
+
+    hbm_peak, _, peak_src = peaks()
+    achieved = step_bytes / (ms * 1e-3) / 1e9
+    h2d = sum(w.numel() * 4 for _, w, _, _ in mats)
+    d2h = sum(c.numel() + sc.numel() * 4 for _, _, c, sc in mats)
+    result = {
+        "metric": QUANT_METRIC,
+        "value": world * step_bytes / (ms * 1e-3) / 1e9,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32 -> int4 (fp32 scales)",
+        "data": "synthetic (N(0, 0.02) fp32 weights from torch's seeded device generator)",
+        "config": {
+            "workload": "quantize: int4_row_quantize (group 128) of 16 experts x {gate [8192, 5120], "
+                        "up [8192, 5120], down [5120, 8192]} fp32 = 2.01 G weights, 3 calls per step",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "inputs (8.05 GB) larger than L2; no flush",
+        },
+        "roofline": {"bound": "hbm", "kernel": "quantize_int4", "achieved": achieved, "peak": hbm_peak,
+                     "peak_source": peak_src + " copy bandwidth", "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": None, "algorithmic_bytes": step_bytes // len(mats)},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": len(mats) * args.steps,
+        "clocks": clocks,
+    }
+    return result
+
+
+def time_oracle_quantize(seed: int, budget_s: float, n_steps: int, n_warm: int):
+    """The oracle's int4_row_quantize (then packing) on row blocks of the gate
+    projection's shape, sized so a step takes about budget_s; returns (GB/s
+    of algorithmic bytes, sample text, seconds per step)."""
+    from oracle import quant as oq
+    w = synth.expert_weights(seed, 0, QUANT_D, QUANT_F)[0]       # [8192, 5120] fp32
+    t = time.perf_counter()
+    oq.pack_int4(oq.int4_row_quantize(w[:64])[0])
+    c64 = max(time.perf_counter() - t, 1e-4)
+    rows = int(min(w.shape[0], max(64, budget_s / c64 * 64 // 64 * 64)))
+    blk = np.ascontiguousarray(w[:rows])
+    for _ in range(n_warm):
+        oq.pack_int4(oq.int4_row_quantize(blk)[0])
+    t = time.perf_counter()
+    for _ in range(n_steps):
+        oq.pack_int4(oq.int4_row_quantize(blk)[0])
+    el = (time.perf_counter() - t) / max(n_steps, 1)
+    sample = ("the first %d of 8192 rows of expert 0's gate projection [8192, 5120] per step (%.2f%% of "
+              "the 2.01 G-weight set); GB/s of algorithmic bytes" % (rows, 100.0 * rows * QUANT_D / 2.01e9))
+    return quant_bytes(rows, QUANT_D) / el / 1e9, sample, el
 
 
 # ---------------------------------------------------------------------------
@@ -397,7 +542,8 @@ def oracle_sample_layer(shape: synth.LayerShape, seed: int, f_sub: int, token: i
     experts = {}
     for e in ids:
         g, u, d = synth.expert_weights(seed, int(e), shape.D, shape.F)
-        experts[int(e)] = tuple(oq.int4_row_quantize(np.ascontiguousarray(w))
+        quant = oq.int4_row_quantize if shape.fmt == "int4" else oq.fp8_row_quantize
+        experts[int(e)] = tuple(quant(np.ascontiguousarray(w))
                                 for w in (g[:f_sub], u[:f_sub], d[:, :f_sub]))
     return offn.Layer(shape.fmt, shape.k, wr, bias, experts.__getitem__,
                       (sg[:fs_sub], su[:fs_sub], sd[:, :fs_sub].contiguous())), fs_sub
@@ -430,8 +576,20 @@ def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: in
 
 
 def run_reference(args):
-    shape = synth.SHAPES[args.workload]
     budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
+    if args.workload == "quantize":
+        v, sample, per_step = time_oracle_quantize(args.seed, budget, args.steps, args.warmup)
+        return {
+            "impl": "reference", "metric": QUANT_METRIC, "value": v, "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 -> int4",
+            "data": "synthetic (seeded N(0, 0.02) fp32 weights)",
+            "config": {"workload": "quantize (CPU oracle on a row sample)",
+                       "parallelism": "CPU oracle on the host cores"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+    shape = synth.SHAPES[args.workload]
     v, sample, per_step = time_oracle(shape, args.seed, budget, args.steps, args.warmup)
     cores = oracle_cores()
     return {
@@ -448,7 +606,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
-        "config": {"workload": workload_text(shape), "weights": "routed int4 g128; router and shared bf16",
+        "config": {"workload": workload_text(shape), "weights": weights_text(shape),
                    "parallelism": "CPU oracle on the host cores"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -462,7 +620,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scout_decode",
-                    choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8"])
+                    choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8", "quantize"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -487,11 +645,18 @@ def main(argv=None):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    result, shape = run_ours(args, rank, world, dev)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, _ = time_oracle(shape, args.seed, budget_s=10.0, n_steps=2, n_warm=0)
-        result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle_cores(),
-                                  "kind": "oracle", "sample": sample}
+    if args.workload == "quantize":
+        result = run_quantize(args, rank, world, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, sample, _ = time_oracle_quantize(args.seed, budget_s=5.0, n_steps=2, n_warm=0)
+            result["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": 1,   # element-wise numpy: one thread
+                                      "kind": "oracle", "sample": sample}
+    else:
+        result, shape = run_ours(args, rank, world, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, sample, _ = time_oracle(shape, args.seed, budget_s=10.0, n_steps=2, n_warm=0)
+            result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle_cores(),
+                                      "kind": "oracle", "sample": sample}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -143,6 +143,7 @@ MOE_API moe_status moe_route(const void* x, int32_t T, int32_t D,
  *              quantizes its input rows to e4m3 with bound act_scale_ub.
  *   ws_gate, ws_up bf16 [F_shared, D]; ws_down bf16 [D, F_shared].
  *   path: a moe_path; AUTO picks DECODE when T * k <= 4 * E, else PREFILL.
+ *         FP8_ROW layers always run on the tensor-core tiles (PREFILL).
  */
 typedef struct moe_layer_desc {
     int32_t E, k, D, F, F_shared;
@@ -163,7 +164,10 @@ typedef struct moe_layer_desc {
 /*
  * Bytes of device workspace moe_ffn_forward needs for up to T_max tokens
  * (0 if the layer description is invalid).  Includes room for the host
- * staging of moe_ffn_forward_host.
+ * staging of moe_ffn_forward_host.  The size depends on `layer->path`: a
+ * fixed DECODE or PREFILL path (FP8_ROW layers always take PREFILL) needs
+ * only that path's buffers, AUTO the larger of the two, since the path it
+ * takes depends on T.
  */
 MOE_API size_t moe_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max);
 

@@ -210,14 +210,20 @@ class MoELayer:
         return n
 
     def reserve(self, T_max: int) -> None:
+        """Make the workspace large enough for up to ``T_max`` tokens with the
+        current path setting (its size depends on the path)."""
         if T_max <= self.T_max:
             return
         n = self.workspace_bytes(T_max)
-        self.workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
+        if self.workspace is None or self.workspace.numel() < n:
+            self.workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
         self.T_max = T_max
 
     def set_path(self, path: int) -> None:
-        self.desc.path = path
+        if path != self.desc.path:
+            self.desc.path = path
+            T_max, self.T_max = self.T_max, 0
+            self.reserve(T_max)
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         T = x.shape[0]

@@ -113,9 +113,13 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     return w;
 }
 
+// Workspace for every call with this descriptor and at most T tokens: the
+// fixed path's layout, or the larger of the two when the path depends on T.
 size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
     const size_t a = ws_layout(L, T, PATH_SEL_DECODE).total;
     const size_t b = ws_layout(L, T, PATH_SEL_PREFILL).total;
+    if (L.format == MOE_WEIGHTS_FP8_ROW || L.path == MOE_PATH_PREFILL) return b;
+    if (L.path == MOE_PATH_DECODE) return a;
     return a > b ? a : b;
 }
 
