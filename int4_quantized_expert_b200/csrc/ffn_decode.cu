@@ -14,11 +14,12 @@
 //     expert first, and streams the task's weights with 2-D TMA loads
 //     (32 rows x 128 bytes, 128-byte swizzle) through a ring of 8 KB stages;
 //     the task's int4 scales arrive with one 1-D bulk copy.
-//   * 8 consumer warps: 2 row blocks of 16 rows x 4 K phases (stage s goes to
-//     phase s % 4).  Each converts int4 codes to exact bf16 integers in
+//   * 12 consumer warps: 2 row blocks of 16 rows x 6 K phases (stage s goes
+//     to phase s % 6), three per SM sub-partition to hide each one's MMA and
+//     load latencies.  Each converts int4 codes to exact bf16 integers in
 //     registers (no scale multiply per element), runs m16n8k16 tensor-core
 //     MMAs against the tokens (fp32 accumulate), and applies the group's scale
-//     to the 128-K partial sum.  The 4 K phases are summed through shared
+//     to the 128-K partial sum.  The 6 K phases are summed through shared
 //     memory, then the epilogue applies SwiGLU (gate/up pass) or the gate
 //     (down pass).
 //   * Tokens are the MMA's N operand (8 per n-tile).  Their rows are read with
@@ -32,20 +33,20 @@
 namespace moe {
 
 constexpr int DC_ROWS = 32;                 // output rows per task
-constexpr int DC_KPH = 4;                   // K phases
-constexpr int DC_CONSUMERS = 8;             // 2 row blocks x 4 K phases
-// Three warpgroups: warpgroup 0 holds the producer (warp 0, one thread) and
-// gives most of its registers to warpgroups 1 and 2, the 8 consumer warps:
-// 128 x 40 + 256 x 232 = 384 x 168, the registers the block launches with.
-constexpr int DC_THREADS = 384;
+constexpr int DC_KPH = 6;                   // K phases
+constexpr int DC_CONSUMERS = 12;            // 2 row blocks x 6 K phases: 3 warps per SM sub-partition
+// Four warpgroups: warpgroup 0 holds the producer (warp 0, one thread) and
+// gives most of its registers to warpgroups 1 to 3, the 12 consumer warps:
+// 128 x 40 + 384 x 152 <= 512 x 128, the registers the block launches with.
+constexpr int DC_THREADS = 512;
 constexpr int DC_PRODUCER_REGS = 40;
-constexpr int DC_CONSUMER_REGS = 232;
-static_assert(128 * DC_PRODUCER_REGS + 256 * DC_CONSUMER_REGS <= DC_THREADS * 168, "register split");
+constexpr int DC_CONSUMER_REGS = 152;
+static_assert(128 * DC_PRODUCER_REGS + 32 * DC_CONSUMERS * DC_CONSUMER_REGS <= DC_THREADS * 128, "register split");
 constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 32 rows x 128 B
 constexpr int DC_STAGE = 2 * DC_CHUNK;      // 8 KB
 constexpr int DC_NSTAGES = 16;              // ring: 128 KB in flight
 constexpr int DC_NT = 2;                    // n-tiles of 8 tokens per task
-constexpr int DC_RED_FLOATS = 6 * 32 * DC_NT * 8;   // partial sums of K phases 1..3
+constexpr int DC_RED_FLOATS = (DC_KPH - 1) * 2 * 32 * DC_NT * 8;   // partial sums of K phases 1..5
 
 struct TaskInfo {
     int32_t kind;       // 0 = shared (bf16), 1 = routed (int4), -1 = done
@@ -63,8 +64,8 @@ struct DecodeSmem {
     uint64_t empty[DC_NSTAGES];
     uint64_t sfull[2];
     uint64_t sempty[2];
-    uint64_t red_full;    // K phases 1..3 -> phase 0: partial sums written
-    uint64_t red_empty;   // phase 0 -> phases 1..3: partial sums consumed
+    uint64_t red_full;    // K phases 1..5 -> phase 0: partial sums written
+    uint64_t red_empty;   // phase 0 -> phases 1..5: partial sums consumed
     TaskInfo task[2];
 };
 
@@ -80,10 +81,7 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 }
 
 
-// position of element i (0..7) of an 8-block in the x0 x4 x1 x5 x2 x6 x3 x7 layout
-__device__ __forceinline__ int frag_pos8(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
-
-// The int4 part of a decode task: the warp's stages q, q + 4, ... of groups
+// The int4 part of a decode task: the warp's stages q, q + 6, ... of groups
 // of 128 K, NT token tiles.  Returns false if a wait timed out.
 //
 // Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
@@ -139,58 +137,82 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
         if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
         const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
         const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
-        // two accumulation chains per matrix (even / odd words); the even one
-        // starts from the group offset, the odd one from zero
-        float pg[2][NT][4], pu[2][NT][4];
+        // CH independent accumulation chains per matrix (word jj feeds chain
+        // jj % CH; chain 0 starts from the group offset, the others from
+        // zero).  Every word's even-nibble MMAs are issued before any
+        // odd-nibble one, so consecutive MMAs of a warp do not depend on
+        // each other.
+        constexpr int CH = NT == 1 ? 4 : 2;
+        float pg[CH][NT][4], pu[CH][NT][4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
             const uint32_t ea0 = f16_lo_nibbles(WA[jj]), ea1 = f16_lo_nibbles(WB[jj]);
             const uint32_t ea2 = f16_lo_nibbles(wa8), ea3 = f16_lo_nibbles(wb8);
-            const uint32_t oa0 = f16_hi_nibbles(WA[jj]), oa1 = f16_hi_nibbles(WB[jj]);
-            const uint32_t oa2 = f16_hi_nibbles(wa8), oa3 = f16_hi_nibbles(wb8);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float* d = pg[jj & 1][nt];
+                float* d = pg[jj % CH][nt];
                 if (jj == 0) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y,
                                            cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
-                else if (jj == 1) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
+                else if (jj < CH) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
                 else mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y);
-                mma_f16_16816(d, oa0, oa1, oa2, oa3, xc[nt][jj].z, xc[nt][jj].w);
             }
             if (MODE == 0) {
                 const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
                 const uint32_t eu0 = f16_lo_nibbles(VA[jj]), eu1 = f16_lo_nibbles(VB[jj]);
                 const uint32_t eu2 = f16_lo_nibbles(va8), eu3 = f16_lo_nibbles(vb8);
-                const uint32_t ou0 = f16_hi_nibbles(VA[jj]), ou1 = f16_hi_nibbles(VB[jj]);
-                const uint32_t ou2 = f16_hi_nibbles(va8), ou3 = f16_hi_nibbles(vb8);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    float* d = pu[jj & 1][nt];
+                    float* d = pu[jj % CH][nt];
                     if (jj == 0) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y,
                                                cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
-                    else if (jj == 1) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
+                    else if (jj < CH) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
                     else mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y);
-                    mma_f16_16816(d, ou0, ou1, ou2, ou3, xc[nt][jj].z, xc[nt][jj].w);
                 }
             }
         }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
+            const uint32_t oa0 = f16_hi_nibbles(WA[jj]), oa1 = f16_hi_nibbles(WB[jj]);
+            const uint32_t oa2 = f16_hi_nibbles(wa8), oa3 = f16_hi_nibbles(wb8);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_f16_16816(pg[jj % CH][nt], oa0, oa1, oa2, oa3, xc[nt][jj].z, xc[nt][jj].w);
+            if (MODE == 0) {
+                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                const uint32_t ou0 = f16_hi_nibbles(VA[jj]), ou1 = f16_hi_nibbles(VB[jj]);
+                const uint32_t ou2 = f16_hi_nibbles(va8), ou3 = f16_hi_nibbles(vb8);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_f16_16816(pu[jj % CH][nt], ou0, ou1, ou2, ou3, xc[nt][jj].z, xc[nt][jj].w);
+            }
+        }
+#pragma unroll
+        for (int k = 1; k < CH; ++k)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    pg[0][nt][r] += pg[k][nt][r];
+                    if (MODE == 0) pu[0][nt][r] += pu[k][nt][r];
+                }
         const float sga = sga_p[G], sgb = sgb_p[G];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            acc0[nt][0] = fmaf(pg[0][nt][0] + pg[1][nt][0], sga, acc0[nt][0]);
-            acc0[nt][1] = fmaf(pg[0][nt][1] + pg[1][nt][1], sga, acc0[nt][1]);
-            acc0[nt][2] = fmaf(pg[0][nt][2] + pg[1][nt][2], sgb, acc0[nt][2]);
-            acc0[nt][3] = fmaf(pg[0][nt][3] + pg[1][nt][3], sgb, acc0[nt][3]);
+            acc0[nt][0] = fmaf(pg[0][nt][0], sga, acc0[nt][0]);
+            acc0[nt][1] = fmaf(pg[0][nt][1], sga, acc0[nt][1]);
+            acc0[nt][2] = fmaf(pg[0][nt][2], sgb, acc0[nt][2]);
+            acc0[nt][3] = fmaf(pg[0][nt][3], sgb, acc0[nt][3]);
         }
         if (MODE == 0) {
             const float sua = sua_p[G], sub = sub_p[G];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                acc1[nt][0] = fmaf(pu[0][nt][0] + pu[1][nt][0], sua, acc1[nt][0]);
-                acc1[nt][1] = fmaf(pu[0][nt][1] + pu[1][nt][1], sua, acc1[nt][1]);
-                acc1[nt][2] = fmaf(pu[0][nt][2] + pu[1][nt][2], sub, acc1[nt][2]);
-                acc1[nt][3] = fmaf(pu[0][nt][3] + pu[1][nt][3], sub, acc1[nt][3]);
+                acc1[nt][0] = fmaf(pu[0][nt][0], sua, acc1[nt][0]);
+                acc1[nt][1] = fmaf(pu[0][nt][1], sua, acc1[nt][1]);
+                acc1[nt][2] = fmaf(pu[0][nt][2], sub, acc1[nt][2]);
+                acc1[nt][3] = fmaf(pu[0][nt][3], sub, acc1[nt][3]);
             }
         }
     };
@@ -246,11 +268,14 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         mbar_init(&sm->red_empty, 2);
         fence_barrier_init();
     }
+    griddep_launch_dependents();
     __syncthreads();
 
+    // The shared expert's chunks (16 tokens each) follow from T alone, so its
+    // tasks start before the routing step has finished; the routed chunk
+    // list is read after the grid dependency wait.
     const int nbs = p.n_rows_s / DC_ROWS, nbr = p.n_rows_r / DC_ROWS;
-    const int n_chunks = *p.n_chunks, n_sh = *p.n_shared_chunks;
-    const int n_tasks = n_sh * nbs + (n_chunks - n_sh) * nbr;
+    const int n_sh = int(ceil_div(p.T, 16));
 
     if (warp < 4) {
         // ------------------------------ producer ------------------------------
@@ -258,9 +283,15 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         if (warp == 0 && lane == 0) {
             prefetch_tmap(&tm_r0); prefetch_tmap(&tm_r1); prefetch_tmap(&tm_s0); prefetch_tmap(&tm_s1);
             uint32_t it = 0;
-            bool ok = true;
+            bool ok = true, waited = false;
+            int n_tasks = n_sh * nbs;   // grows by the routed tasks after the wait
             for (uint32_t tn = 0; ok; ++tn) {
                 const int t = atomicAdd(p.task_counter, 1);
+                if (t >= n_sh * nbs && !waited) {
+                    griddep_wait();   // the routing step's chunk list is complete
+                    n_tasks += (*p.n_chunks - n_sh) * nbr;
+                    waited = true;
+                }
                 const int b = tn & 1;
                 if (!mbar_wait(&sm->sempty[b], ((tn >> 1) & 1) ^ 1, p.status, 128)) break;
                 TaskInfo ti;
@@ -272,9 +303,19 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     break;
                 }
                 int ci, blk;
-                if (t < n_sh * nbs) { ci = t / nbs; blk = t % nbs; }
-                else { const int u = t - n_sh * nbs; ci = n_sh + u / nbr; blk = u % nbr; }
-                const ChunkEntry ce = p.chunks[ci];
+                ChunkEntry ce;
+                if (t < n_sh * nbs) {
+                    ci = t / nbs;
+                    blk = t % nbs;
+                    ce.expert = -1;
+                    ce.start = ci * 16;
+                    ce.count = min(16, p.T - ci * 16);
+                } else {
+                    const int u = t - n_sh * nbs;
+                    ci = n_sh + u / nbr;
+                    blk = u % nbr;
+                    ce = p.chunks[ci];
+                }
                 ti.kind = ce.expert < 0 ? 0 : 1;
                 ti.expert = ce.expert;
                 ti.row0 = blk * DC_ROWS;
@@ -315,6 +356,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     }
                 }
             }
+            // this grid completes only after the kernels before it
+            if (!waited) griddep_wait();
             // wind down: wait (bounded) for every stage still in flight to land
             for (uint32_t i = 0; i < DC_NSTAGES && i < it; ++i) {
                 const uint32_t j = it - 1 - i;
@@ -331,11 +374,18 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const int g = lane >> 2, c = lane & 3;
     const int row_a = 16 * rb + sigma8(g), row_b = row_a + 8;
     uint32_t it_base = 0;
+    bool waited = false;
     for (uint32_t tn = 0;; ++tn) {
         const int b = tn & 1;
         if (!mbar_wait(&sm->sfull[b], (tn >> 1) & 1, p.status)) break;
         const TaskInfo ti = sm->task[b];
         if (ti.kind < 0) break;
+        // everything but the shared expert's tokens (the layer input) comes
+        // from the kernels before this one
+        if (!waited && (MODE == 1 || ti.kind == 1)) {
+            griddep_wait();
+            waited = true;
+        }
         const float* sc = sbuf + b * p.scale_buf_floats;
         const int ng = ti.K / kGroup;
 
@@ -377,11 +427,9 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 
         bool ok = true;
         if (ti.kind == 1) {
-            ok = nt_used == 1
-                     ? consume_int4<MODE, 1>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
-                                             p.status)
-                     : consume_int4<MODE, 2>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
-                                             p.status);
+            // routed chunks hold at most 8 tokens: one n-tile
+            ok = consume_int4<MODE, 1>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
+                                       p.status);
         } else {
             // ---------------- bf16 weights (shared expert): 64 K per tile ----------------
             // thread c takes the 8-blocks c and c + 4 of each 64-K tile
@@ -420,10 +468,10 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                         if (MODE == 0) { va = lds128(swz(st + DC_CHUNK, row_a, j)); vb = lds128(swz(st + DC_CHUNK, row_b, j)); }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t a0 = h == 0 ? prmt(wa.x, wa.z, 0x5410) : prmt(wa.y, wa.w, 0x5410);
-                            const uint32_t a2 = h == 0 ? prmt(wa.x, wa.z, 0x7632) : prmt(wa.y, wa.w, 0x7632);
-                            const uint32_t a1 = h == 0 ? prmt(wb.x, wb.z, 0x5410) : prmt(wb.y, wb.w, 0x5410);
-                            const uint32_t a3 = h == 0 ? prmt(wb.x, wb.z, 0x7632) : prmt(wb.y, wb.w, 0x7632);
+                            // MMA h takes K values 8 j + 4 h .. + 3 of the rows (natural order):
+                            // its k-slots 2c, 2c+1 get the first pair, 2c+8, 2c+9 the second
+                            const uint32_t a0 = h == 0 ? wa.x : wa.z, a2 = h == 0 ? wa.y : wa.w;
+                            const uint32_t a1 = h == 0 ? wb.x : wb.z, a3 = h == 0 ? wb.y : wb.w;
 #pragma unroll
                             for (int nt = 0; nt < DC_NT; ++nt) {
                                 if (nt >= nt_used) break;
@@ -432,10 +480,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                                 mma_bf16_16816(acc0[nt], a0, a1, a2, a3, b0, b1);
                             }
                             if (MODE == 0) {
-                                const uint32_t u0 = h == 0 ? prmt(va.x, va.z, 0x5410) : prmt(va.y, va.w, 0x5410);
-                                const uint32_t u2 = h == 0 ? prmt(va.x, va.z, 0x7632) : prmt(va.y, va.w, 0x7632);
-                                const uint32_t u1 = h == 0 ? prmt(vb.x, vb.z, 0x5410) : prmt(vb.y, vb.w, 0x5410);
-                                const uint32_t u3 = h == 0 ? prmt(vb.x, vb.z, 0x7632) : prmt(vb.y, vb.w, 0x7632);
+                                const uint32_t u0 = h == 0 ? va.x : va.z, u2 = h == 0 ? va.y : va.w;
+                                const uint32_t u1 = h == 0 ? vb.x : vb.z, u3 = h == 0 ? vb.y : vb.w;
 #pragma unroll
                                 for (int nt = 0; nt < DC_NT; ++nt) {
                                     if (nt >= nt_used) break;
@@ -457,7 +503,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         }
         if (!ok) break;
 
-        // ---- sum the 4 K phases (phases 1..3 hand their partial sums to phase 0) ----
+        // ---- sum the K phases (phases 1..5 hand their partial sums to phase 0) ----
         if (q > 0) {
             if (!mbar_wait(&sm->red_empty, (tn & 1) ^ 1, p.status)) break;
             float* my = red + ((q - 1) * 2 + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
@@ -479,8 +525,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             }
             // ---- epilogue: C rows (row_a, row_b) x token columns (2c, 2c + 1) of each n-tile ----
             // routed results are rescaled by their B row's power of two;
-            // routed h is stored in natural order (its fp16 copy is made next),
-            // the shared expert's h in the bf16 fragment order it is read in
+            // h is stored in natural order (the routed rows' fp16 copy is made next)
 #pragma unroll
             for (int nt = 0; nt < DC_NT; ++nt) {
 #pragma unroll
@@ -495,8 +540,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                             p.h_r[int64_t(ti.start + col) * p.n_rows_r + n] = __float2bfloat16_rn(hv);
                         } else {
                             const float hv = silu_f32(acc0[nt][r]) * acc1[nt][r];
-                            const int pos = (n & ~7) + frag_pos8(n & 7);
-                            p.h_s[int64_t(ti.start + col) * p.n_rows_s + pos] = __float2bfloat16_rn(hv);
+                            p.h_s[int64_t(ti.start + col) * p.n_rows_s + n] = __float2bfloat16_rn(hv);
                         }
                     } else {
                         if (ti.kind == 1) {
@@ -520,6 +564,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 __global__ void combine_kernel(const float* __restrict__ y_s, const float* __restrict__ y_r,
                                const int32_t* __restrict__ inv_perm, int T, int D, int k,
                                bf16* __restrict__ out) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int64_t n4 = int64_t(T) * D / 4;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
         const int64_t t = i / (D / 4);
@@ -537,7 +583,8 @@ __global__ void combine_kernel(const float* __restrict__ y_s, const float* __res
     }
 }
 
-int decode_max_chunks(int T, int k, int E) { return int(ceil_div(T, 16)) + int(ceil_div(int64_t(T) * k, 16)) + E; }
+// shared-expert chunks of 16 tokens, routed ones of 8 (at most one partial chunk per expert)
+int decode_max_chunks(int T, int k, int E) { return int(ceil_div(T, 16)) + int(ceil_div(int64_t(T) * k, 8)) + E; }
 
 size_t decode_smem_bytes(int scale_buf_floats) {
     return 1024 + size_t(DC_NSTAGES) * DC_STAGE + 2 * size_t(scale_buf_floats) * 4 + DC_RED_FLOATS * 4 +
@@ -586,16 +633,10 @@ moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParam
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = decode_smem_bytes(prm.scale_buf_floats);
     cudaError_t e;
-    if (mode == 0) {
-        e = cudaFuncSetAttribute(decode_ffn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        decode_ffn_kernel<0><<<sms, DC_THREADS, smem, stream>>>(maps.r0, maps.r1, maps.s0, maps.s1, prm);
-    } else {
-        e = cudaFuncSetAttribute(decode_ffn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        decode_ffn_kernel<1><<<sms, DC_THREADS, smem, stream>>>(maps.r0, maps.r1, maps.s0, maps.s1, prm);
-    }
-    return launch_status();
+    auto kern = mode == 0 ? decode_ffn_kernel<0> : decode_ffn_kernel<1>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return launch_pdl(kern, dim3(sms), dim3(DC_THREADS), smem, stream, maps.r0, maps.r1, maps.s0, maps.s1, prm);
 }
 
 moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
@@ -603,8 +644,7 @@ moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv
     const int64_t n4 = int64_t(T) * D / 4;
     int64_t blocks = ceil_div(n4, 256);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    combine_kernel<<<unsigned(blocks), 256, 0, stream>>>(y_s, y_r, inv_perm, T, D, k, out);
-    return launch_status();
+    return launch_pdl(combine_kernel, dim3(unsigned(blocks)), dim3(256), 0, stream, y_s, y_r, inv_perm, T, D, k, out);
 }
 
 }  // namespace moe
@@ -628,6 +668,8 @@ __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in,
                                                     __half* __restrict__ out16, float* __restrict__ negc,
                                                     float* __restrict__ rscale) {
     __shared__ float red[8];
+    griddep_launch_dependents();
+    griddep_wait();   // the rows come from the kernel before (h), or are the layer input (x)
     const int64_t r = blockIdx.x;
     const bf16* row = in + r * cols;
     const int nblk = cols / 8;
@@ -678,8 +720,10 @@ __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in,
 }
 
 moe_status launch_act16(const bf16* in, int64_t rows, int cols, __half* out16, float* negc, float* rscale,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool after_kernel) {
     if (rows == 0) return MOE_OK;
+    if (after_kernel)
+        return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, out16, negc, rscale);
     act16_kernel<<<unsigned(rows), 256, 0, stream>>>(in, cols, out16, negc, rscale);
     return launch_status();
 }

@@ -18,6 +18,7 @@ struct ChunkEntry {
 };
 
 struct DecodeParams {
+    int32_t T;              // tokens (the shared expert's chunks are the 16-token runs of 0..T-1)
     int32_t n_rows_r;       // output rows of each routed matrix (F for gate/up, D for down)
     int32_t n_rows_s;       // output rows of each shared matrix (F_shared for gate/up, D for down)
     int32_t K_r, K_s;       // reduction lengths (routed, shared)
@@ -51,9 +52,11 @@ struct RoutePrep {
     bf16* x_frag;         // x in bf16 fragment order [T, D] (shared expert)
     ChunkEntry* chunks;   // task list
     int32_t* n_chunks;    // [0] all chunks, [1] the shared expert's
-    int32_t chunk_tokens; // tokens per chunk (16 for the weight-streaming path, 256 for tensor-core tiles)
-    int32_t* zero_words;  // zeroed (task counters)
+    int32_t chunk_tokens;         // tokens per shared-expert chunk (16 weight streaming, 256 tensor cores)
+    int32_t routed_chunk_tokens;  // tokens per routed-expert chunk (8 weight streaming, 256 tensor cores)
+    int32_t* zero_words;  // zeroed by the bucketing kernel (or null)
     int32_t n_zero;
+    bool router_after_kernel;   // the router may start while the kernel before it runs
 };
 
 struct DecodeMaps {
@@ -69,7 +72,7 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between);
 moe_status launch_act16(const bf16* in, int64_t rows, int cols, __half* out16, float* negc, float* rscale,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool after_kernel);
 moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
                           bf16* out, cudaStream_t stream);
 

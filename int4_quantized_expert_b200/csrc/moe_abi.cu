@@ -42,7 +42,7 @@ struct WsLayout {
     size_t status, zeros, zero_corr, zeros_end, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
     size_t common_end;
     // weight-streaming path
-    size_t x_frag, x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
+    size_t x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
     // tensor-core path (row counts padded to whole 256-token tiles)
     size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos, y_shared;
     size_t xq, xq_scale, hq, hq_scale;   // e4m3 activations of FP8_ROW layers
@@ -66,11 +66,11 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     const int64_t S_pad = ceil_div(S, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
     const int64_t T_pad = ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
     w.status = take(64);
+    w.counters = take(64);   // task counters of the weight-streaming kernels
     const int maxdim = L.D > L.F ? (L.D > L.F_shared ? L.D : L.F_shared) : (L.F > L.F_shared ? L.F : L.F_shared);
     w.zeros = take(size_t(maxdim) * 2);
     w.zero_corr = take(size_t(maxdim / kGroup) * 4);
-    w.zeros_end = off;
-    w.counters = take(64);
+    w.zeros_end = off;   // [status, zeros_end) is cleared at the start of every call
     w.ids = take(S * 4);
     w.gates = take(S * 4);
     w.counts = take(size_t(L.E) * 4);
@@ -81,7 +81,6 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.nchunks = take(16);
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
-        w.x_frag = take(T * L.D * 2);
         w.x16 = take(T * L.D * 2);
         w.x_negc = take(T * (L.D / kGroup) * 4);
         w.x_scale = take(T * 4);
@@ -158,7 +157,7 @@ struct Marks {
     }
 };
 
-const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up",
+const char* const kDecodeLaunches[] = {"act16_x", "router", "bucket", "decode_gate_up",
                                        "act16_h", "decode_down", "combine"};
 constexpr int32_t kDecodeLaunchCount = 7;
 
@@ -174,7 +173,6 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     int32_t* perm = at<int32_t>(ws, W.perm);
     int32_t* inv = at<int32_t>(ws, W.inv_perm);
     float* gates = at<float>(ws, W.gates);
-    bf16* x_frag = at<bf16>(ws, W.x_frag);
     bf16* h_r = at<bf16>(ws, W.h_r);
     bf16* h_s = at<bf16>(ws, W.h_s);
     float* y_r = at<float>(ws, W.y_r);
@@ -182,22 +180,29 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
     int32_t* nch = at<int32_t>(ws, W.nchunks);
 
+    // Launch order: act16_x, router, bucket, gate/up, act16_h, down, combine;
+    // every launch after the first may start while the one before it runs
+    // (programmatic dependent launch) and waits before reading its outputs.
+    mk.mark(st);
+    moe_status s = launch_act16(x, T, L.D, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale),
+                                st, /*after_kernel=*/false);
+    if (s != MOE_OK) return s;
+
     RoutePrep prep;
-    prep.x_frag = x_frag;
+    memset(&prep, 0, sizeof(prep));
+    prep.x_frag = nullptr;
     prep.chunks = chunks;
     prep.n_chunks = nch;
-    prep.zero_words = counters;
-    prep.n_zero = 2;
+    prep.zero_words = nullptr;      // the task counters are cleared with the status word
+    prep.n_zero = 0;
     prep.chunk_tokens = 16;
+    prep.routed_chunk_tokens = 8;   // one 8-column n-tile per routed chunk
+    prep.router_after_kernel = true;
     mk.mark(st);
-    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
-                                at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
-                                at<int32_t>(ws, W.offsets), perm, inv, &prep, st,
-                                (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
+    s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+                     at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
+                     &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
     ++mk.i;
-    if (s != MOE_OK) return s;
-    mk.mark(st);
-    s = launch_act16(x, T, L.D, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale), st);
     if (s != MOE_OK) return s;
 
     DecodeMaps m1, m2;
@@ -214,6 +219,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
 
     DecodeParams p;
     memset(&p, 0, sizeof(p));
+    p.T = T;
     p.n_rows_r = L.F;
     p.n_rows_s = L.F_shared;
     p.K_r = L.D;
@@ -227,7 +233,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.gates = gates;
     p.b_r = at<bf16>(ws, W.x16);
     p.ldb_r = L.D;
-    p.b_s = x_frag;
+    p.b_s = x;   // the shared expert reads the layer input itself
     p.ldb_s = L.D;
     p.sc0 = L.s_gate;
     p.sc1 = L.s_up;
@@ -245,7 +251,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
 
     mk.mark(st);
     s = launch_act16(h_r, int64_t(T) * L.k, L.F, at<__half>(ws, W.h16), at<float>(ws, W.h_negc),
-                     at<float>(ws, W.h_scale), st);
+                     at<float>(ws, W.h_scale), st, /*after_kernel=*/true);
     if (s != MOE_OK) return s;
 
     p.n_rows_r = L.D;
@@ -311,9 +317,11 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
 
     RoutePrep prep;
     memset(&prep, 0, sizeof(prep));
+    memset(&prep, 0, sizeof(prep));
     prep.chunks = chunks;
     prep.n_chunks = nch;
     prep.chunk_tokens = TC_BLOCK_TOKENS;
+    prep.routed_chunk_tokens = TC_BLOCK_TOKENS;
     mk.mark(st);
     moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                                 at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),

@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     const float* __restrict__ bias, int E, int k, int32_t* __restrict__ ids,
     float* __restrict__ gates, bf16* __restrict__ x_frag) {
     extern __shared__ __align__(16) float part[];     // [nw][RT_TOK][E]
+    griddep_launch_dependents();
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -170,6 +171,9 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
             }
         }
     }
+    // reads nothing of the kernel before it (if launched dependent on one),
+    // but completes only after it
+    griddep_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -182,12 +186,14 @@ constexpr int BK_MAX_E = 256;
 __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     const int32_t* __restrict__ ids, int n_slots, int T, int E, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-    ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int chunk_tokens,
+    ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int chunk_tokens, int routed_chunk_tokens,
     int32_t* __restrict__ zero_words, int n_zero) {
     __shared__ int s_count[BK_MAX_E];
     __shared__ int s_base[BK_MAX_E];
     __shared__ int s_warp[BK_WARPS][BK_MAX_E];   // per-warp counts, then exclusive prefix over warps
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_launch_dependents();
+    griddep_wait();   // the router's ids
 
     if (zero_words != nullptr)
         for (int i = tid; i < n_zero; i += BK_THREADS) zero_words[i] = 0;
@@ -199,8 +205,9 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
         int run = 0;
         for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_count[e]; }
         if (chunks != nullptr) {
-            // task list of the FFN kernels: chunks of <= chunk_tokens tokens,
-            // the shared expert's first, then each routed expert's
+            // task list of the FFN kernels: the shared expert's chunks of
+            // <= chunk_tokens tokens, then each routed expert's of
+            // <= routed_chunk_tokens
             int n = 0;
             for (int t0 = 0; t0 < T; t0 += chunk_tokens) {
                 ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(chunk_tokens, T - t0); ce.pad = 0;
@@ -208,9 +215,9 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
             }
             n_chunks[1] = n;
             for (int e = 0; e < E; ++e)
-                for (int s = 0; s < s_count[e]; s += chunk_tokens) {
+                for (int s = 0; s < s_count[e]; s += routed_chunk_tokens) {
                     ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s;
-                    ce.count = min(chunk_tokens, s_count[e] - s);
+                    ce.count = min(routed_chunk_tokens, s_count[e] - s);
                     ce.pad = 0;
                     chunks[n++] = ce;
                 }
@@ -266,16 +273,23 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
     if (cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(RT_SMEM_MAX)) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    router_kernel<<<unsigned(ceil_div(T, RT_TOK)), nw * 32, smem, stream>>>(
-        x, T, D, wr, bias, E, k, ids, gates, prep ? prep->x_frag : nullptr);
-    moe_status st = launch_status();
+    moe_status st;
+    bf16* x_frag = prep ? prep->x_frag : nullptr;
+    if (prep && prep->router_after_kernel)   // may overlap the kernel before it (it reads only x and W_r)
+        st = launch_pdl(router_kernel, dim3(unsigned(ceil_div(T, RT_TOK))), dim3(nw * 32), smem, stream, x, T, D,
+                        wr, bias, E, k, ids, gates, x_frag);
+    else {
+        router_kernel<<<unsigned(ceil_div(T, RT_TOK)), nw * 32, smem, stream>>>(x, T, D, wr, bias, E, k, ids,
+                                                                               gates, x_frag);
+        st = launch_status();
+    }
     if (st != MOE_OK) return st;
     if (between) cudaEventRecord(between, stream);
-    bucket_kernel<<<1, BK_THREADS, 0, stream>>>(ids, T * k, T, E, counts, offsets, perm, inv_perm,
-                                                prep ? prep->chunks : nullptr, prep ? prep->n_chunks : nullptr,
-                                                prep ? prep->chunk_tokens : 16,
-                                                prep ? prep->zero_words : nullptr, prep ? prep->n_zero : 0);
-    return launch_status();
+    return launch_pdl(bucket_kernel, dim3(1), dim3(BK_THREADS), 0, stream, (const int32_t*)ids, T * k, T, E, counts,
+                      offsets, perm, inv_perm, prep ? prep->chunks : (ChunkEntry*)nullptr,
+                      prep ? prep->n_chunks : (int32_t*)nullptr, prep ? prep->chunk_tokens : 16,
+                      prep ? prep->routed_chunk_tokens : 16, prep ? prep->zero_words : (int32_t*)nullptr,
+                      prep ? prep->n_zero : 0);
 }
 
 }  // namespace moe
