@@ -12,14 +12,14 @@
 //   * one persistent CTA per SM; a producer warp takes tasks (32 output rows of
 //     one matrix pair x one chunk of <= 16 tokens) from a global counter, shared
 //     expert first, and streams the task's weights with 2-D TMA loads
-//     (32 rows x 128 bytes, 128-byte swizzle) through a ring of 8 KB stages;
+//     (64 rows x 128 bytes, 128-byte swizzle) through a ring of 16 KB stages;
 //     the task's int4 scales arrive with one 1-D bulk copy.
-//   * 12 consumer warps: 2 row blocks of 16 rows x 6 K phases (stage s goes
-//     to phase s % 6), three per SM sub-partition to hide each one's MMA and
+//   * 12 consumer warps: 4 row blocks of 16 rows x 3 K phases (stage s goes
+//     to phase s % 3), three per SM sub-partition to hide each one's MMA and
 //     load latencies.  Each converts int4 codes to exact bf16 integers in
 //     registers (no scale multiply per element), runs m16n8k16 tensor-core
 //     MMAs against the tokens (fp32 accumulate), and applies the group's scale
-//     to the 128-K partial sum.  The 6 K phases are summed through shared
+//     to the 128-K partial sum.  The 3 K phases are summed through shared
 //     memory, then the epilogue applies SwiGLU (gate/up pass) or the gate
 //     (down pass).
 //   * Tokens are the MMA's N operand (8 per n-tile).  Their rows are read with
@@ -32,9 +32,10 @@
 
 namespace moe {
 
-constexpr int DC_ROWS = 32;                 // output rows per task
-constexpr int DC_KPH = 6;                   // K phases
-constexpr int DC_CONSUMERS = 12;            // 2 row blocks x 6 K phases: 3 warps per SM sub-partition
+constexpr int DC_RB = 4;                    // row blocks of 16 rows per task
+constexpr int DC_ROWS = 16 * DC_RB;         // output rows per task
+constexpr int DC_KPH = 3;                   // K phases
+constexpr int DC_CONSUMERS = DC_RB * DC_KPH;   // 12: 3 warps per SM sub-partition
 // Four warpgroups: warpgroup 0 holds the producer (warp 0, one thread) and
 // gives most of its registers to warpgroups 1 to 3, the 12 consumer warps:
 // 128 x 40 + 384 x 152 <= 512 x 128, the registers the block launches with.
@@ -42,11 +43,11 @@ constexpr int DC_THREADS = 512;
 constexpr int DC_PRODUCER_REGS = 40;
 constexpr int DC_CONSUMER_REGS = 152;
 static_assert(128 * DC_PRODUCER_REGS + 32 * DC_CONSUMERS * DC_CONSUMER_REGS <= DC_THREADS * 128, "register split");
-constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 32 rows x 128 B
-constexpr int DC_STAGE = 2 * DC_CHUNK;      // 8 KB
-constexpr int DC_NSTAGES = 16;              // ring: 128 KB in flight
+constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 64 rows x 128 B
+constexpr int DC_STAGE = 2 * DC_CHUNK;      // 16 KB
+constexpr int DC_NSTAGES = 8;               // ring: 128 KB in flight
 constexpr int DC_NT = 2;                    // n-tiles of 8 tokens per task
-constexpr int DC_RED_FLOATS = (DC_KPH - 1) * 2 * 32 * DC_NT * 8;   // partial sums of K phases 1..5
+constexpr int DC_RED_FLOATS = (DC_KPH - 1) * DC_RB * 32 * DC_NT * 8;   // partial sums of K phases 1..2
 
 struct TaskInfo {
     int32_t kind;       // 0 = shared (bf16), 1 = routed (int4), -1 = done
@@ -64,8 +65,8 @@ struct DecodeSmem {
     uint64_t empty[DC_NSTAGES];
     uint64_t sfull[2];
     uint64_t sempty[2];
-    uint64_t red_full;    // K phases 1..5 -> phase 0: partial sums written
-    uint64_t red_empty;   // phase 0 -> phases 1..5: partial sums consumed
+    uint64_t red_full;    // K phases 1..2 -> phase 0: partial sums written
+    uint64_t red_empty;   // phase 0 -> phases 1..2: partial sums consumed
     TaskInfo task[2];
 };
 
@@ -81,7 +82,7 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 }
 
 
-// The int4 part of a decode task: the warp's stages q, q + 6, ... of groups
+// The int4 part of a decode task: the warp's stages q, q + 3, ... of groups
 // of 128 K, NT token tiles.  Returns false if a wait timed out.
 //
 // Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
@@ -262,10 +263,10 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < DC_NSTAGES; ++i) { mbar_init(&sm->full[i], 1); mbar_init(&sm->empty[i], 2); }
+        for (int i = 0; i < DC_NSTAGES; ++i) { mbar_init(&sm->full[i], 1); mbar_init(&sm->empty[i], DC_RB); }
         for (int i = 0; i < 2; ++i) { mbar_init(&sm->sfull[i], 1); mbar_init(&sm->sempty[i], DC_CONSUMERS); }
-        mbar_init(&sm->red_full, (DC_KPH - 1) * 2);
-        mbar_init(&sm->red_empty, 2);
+        mbar_init(&sm->red_full, (DC_KPH - 1) * DC_RB);
+        mbar_init(&sm->red_empty, DC_RB);
         fence_barrier_init();
     }
     griddep_launch_dependents();
@@ -370,7 +371,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     // ------------------------------ consumers ------------------------------
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(DC_CONSUMER_REGS));
     const int ci = warp - 4;
-    const int rb = ci & 1, q = ci >> 1;
+    const int rb = ci % DC_RB, q = ci / DC_RB;   // a stage's DC_RB warps sit on different sub-partitions
     const int g = lane >> 2, c = lane & 3;
     const int row_a = 16 * rb + sigma8(g), row_b = row_a + 8;
     uint32_t it_base = 0;
@@ -402,8 +403,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             brow[nt] = p.zero_row;          // tokens beyond the chunk read zeros
             if (i < ti.count) {
                 if (ti.kind == 0) brow[nt] = p.b_s + int64_t(ti.start + i) * p.ldb_s;
-                else if (MODE == 0) brow[nt] = p.b_r + int64_t(p.perm[ti.start + i] / p.k_top) * p.ldb_r;
-                else brow[nt] = p.b_r + int64_t(ti.start + i) * p.ldb_r;
+                else brow[nt] = p.b_r + int64_t(ti.start + i) * p.ldb_r;   // routed rows by position
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 crow[nt][h] = p.zero_corr;
                 cscale[nt][h] = 1.0f;
                 if (ti.kind == 1 && ic < ti.count) {
-                    const int64_t row = MODE == 0 ? int64_t(p.perm[ti.start + ic] / p.k_top) : int64_t(ti.start + ic);
+                    const int64_t row = ti.start + ic;
                     crow[nt][h] = p.corr_r + row * ng;
                     cscale[nt][h] = p.rscale_r[row];
                 }
@@ -503,10 +503,10 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         }
         if (!ok) break;
 
-        // ---- sum the K phases (phases 1..5 hand their partial sums to phase 0) ----
+        // ---- sum the K phases (phases 1..2 hand their partial sums to phase 0) ----
         if (q > 0) {
             if (!mbar_wait(&sm->red_empty, (tn & 1) ^ 1, p.status)) break;
-            float* my = red + ((q - 1) * 2 + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
+            float* my = red + ((q - 1) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
 #pragma unroll
             for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             if (!mbar_wait(&sm->red_full, tn & 1, p.status)) break;
 #pragma unroll
             for (int qq = 1; qq < DC_KPH; ++qq) {
-                const float* o = red + ((qq - 1) * 2 + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
+                const float* o = red + ((qq - 1) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
 #pragma unroll
                 for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
@@ -585,6 +585,11 @@ __global__ void combine_kernel(const float* __restrict__ y_s, const float* __res
 
 // shared-expert chunks of 16 tokens, routed ones of 8 (at most one partial chunk per expert)
 int decode_max_chunks(int T, int k, int E) { return int(ceil_div(T, 16)) + int(ceil_div(int64_t(T) * k, 8)) + E; }
+
+int decode_task_rows() { return DC_ROWS; }
+
+// floats of one task's int4 scale buffer: gate and up rows (mode 0) or down rows
+int decode_scale_floats(int mode, int K) { return (mode == 0 ? 2 : 1) * DC_ROWS * (K / kGroup); }
 
 size_t decode_smem_bytes(int scale_buf_floats) {
     return 1024 + size_t(DC_NSTAGES) * DC_STAGE + 2 * size_t(scale_buf_floats) * 4 + DC_RED_FLOATS * 4 +
@@ -654,7 +659,9 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // fp16 operands for the int4 MMAs.
 //
-// One CTA per row of a bf16 matrix (x, or the routed experts' hidden h):
+// One CTA per output row of a bf16 matrix (the tokens x gathered into
+// expert-sorted position order, or the routed experts' hidden h, already by
+// position):
 //   scale = 2^-e with e chosen from the row's largest magnitude so that the
 //           scaled row stays below 2^15 (fp16 keeps every bf16 value exactly
 //           in that range); rscale[r] = 2^e undoes it on the MMA results;
@@ -665,13 +672,15 @@ namespace moe {
 //          unpacked codes (1032 + q and 1152 + 16 q) add to a dot product.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in, int cols,
+                                                    const int32_t* __restrict__ src_perm, int k,
                                                     __half* __restrict__ out16, float* __restrict__ negc,
                                                     float* __restrict__ rscale) {
     __shared__ float red[8];
     griddep_launch_dependents();
-    griddep_wait();   // the rows come from the kernel before (h), or are the layer input (x)
+    griddep_wait();   // the rows (h) or the permutation come from the kernels before
     const int64_t r = blockIdx.x;
-    const bf16* row = in + r * cols;
+    // out row r: input row src_perm[r] / k (tokens into expert-sorted positions), else row r
+    const bf16* row = in + (src_perm ? int64_t(src_perm[r] / k) : r) * cols;
     const int nblk = cols / 8;
     float m = 0.0f;
     for (int b = threadIdx.x; b < nblk; b += 256) {
@@ -719,13 +728,11 @@ __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in,
     }
 }
 
-moe_status launch_act16(const bf16* in, int64_t rows, int cols, __half* out16, float* negc, float* rscale,
-                        cudaStream_t stream, bool after_kernel) {
+moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
+                        float* negc, float* rscale, cudaStream_t stream) {
     if (rows == 0) return MOE_OK;
-    if (after_kernel)
-        return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, out16, negc, rscale);
-    act16_kernel<<<unsigned(rows), 256, 0, stream>>>(in, cols, out16, negc, rscale);
-    return launch_status();
+    return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, src_perm, k, out16, negc,
+                      rscale);
 }
 
 }  // namespace moe

@@ -29,14 +29,14 @@ struct DecodeParams {
     const int32_t* n_shared_chunks;
     const int32_t* perm;    // sorted position -> slot (t * k + j)
     const float* gates;     // per slot
-    const bf16* b_r;        // B rows, routed (fp16 bits; see act16): gate/up: tokens; down: h rows by position
+    const bf16* b_r;        // B rows, routed, by sorted position (fp16 bits; see act16): tokens or h rows
     int32_t ldb_r;
     const bf16* b_s;        // B rows, shared: gate/up: tokens; down: shared h rows
     int32_t ldb_s;
     const float* sc0;       // routed scales: gate/up: gate; down: down   ([E * rows, K / 128])
     const float* sc1;       // routed scales: gate/up: up
-    const float* corr_r;    // routed B rows: group offsets negc [rows, K_r / 128] (see act16)
-    const float* rscale_r;  // routed B rows: power-of-two scale of each row
+    const float* corr_r;    // routed B rows (by position): group offsets negc [rows, K_r / 128] (see act16)
+    const float* rscale_r;  // routed B rows (by position): power-of-two scale of each row
     bf16* h_r;              // gate/up outputs: routed [T*k, F] (natural order), shared [T, F_shared] (fragment order)
     bf16* h_s;
     float* y_r;             // down outputs: routed gate * y [T*k, D] (by position), shared [T, D]
@@ -67,12 +67,14 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t in
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);
 int decode_max_chunks(int T, int k, int E);
 size_t decode_smem_bytes(int scale_buf_floats);
+int decode_task_rows();
+int decode_scale_floats(int mode, int K);
 moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParams& prm, cudaStream_t stream);
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between);
-moe_status launch_act16(const bf16* in, int64_t rows, int cols, __half* out16, float* negc, float* rscale,
-                        cudaStream_t stream, bool after_kernel);
+moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
+                        float* negc, float* rscale, cudaStream_t stream);
 moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
                           bf16* out, cudaStream_t stream);
 

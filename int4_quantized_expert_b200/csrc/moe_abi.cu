@@ -23,6 +23,7 @@ namespace {
 
 constexpr int kMaxT = 1 << 20;
 constexpr int kMaxDim = 16384;
+constexpr size_t kMaxDecodeSmem = 227 * 1024;
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
@@ -81,9 +82,9 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.nchunks = take(16);
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
-        w.x16 = take(T * L.D * 2);
-        w.x_negc = take(T * (L.D / kGroup) * 4);
-        w.x_scale = take(T * 4);
+        w.x16 = take(S * L.D * 2);                 // tokens by expert-sorted position
+        w.x_negc = take(S * (L.D / kGroup) * 4);
+        w.x_scale = take(S * 4);
         w.h_r = take(S * L.F * 2);
         w.h16 = take(S * L.F * 2);
         w.h_negc = take(S * (L.F / kGroup) * 4);
@@ -122,11 +123,17 @@ size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
     return a > b ? a : b;
 }
 
+// The weight-streaming kernels keep a task's int4 scales in shared memory.
+bool decode_fits(const moe_layer_desc& L) {
+    return decode_smem_bytes(decode_scale_floats(0, L.D)) <= kMaxDecodeSmem &&
+           decode_smem_bytes(decode_scale_floats(1, L.F)) <= kMaxDecodeSmem;
+}
+
 int choose_path(const moe_layer_desc& L, int64_t T) {
     if (L.format == MOE_WEIGHTS_FP8_ROW) return PATH_SEL_PREFILL;   // e4m3 layers run on tensor-core tiles
     if (L.path == MOE_PATH_DECODE) return PATH_SEL_DECODE;
     if (L.path == MOE_PATH_PREFILL) return PATH_SEL_PREFILL;
-    return T * L.k <= 4 * int64_t(L.E) ? PATH_SEL_DECODE : PATH_SEL_PREFILL;
+    return T * L.k <= 4 * int64_t(L.E) && decode_fits(L) ? PATH_SEL_DECODE : PATH_SEL_PREFILL;
 }
 
 moe_status check_layer(const moe_layer_desc* L) {
@@ -157,7 +164,7 @@ struct Marks {
     }
 };
 
-const char* const kDecodeLaunches[] = {"act16_x", "router", "bucket", "decode_gate_up",
+const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up",
                                        "act16_h", "decode_down", "combine"};
 constexpr int32_t kDecodeLaunchCount = 7;
 
@@ -179,15 +186,11 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     float* y_s = at<float>(ws, W.y_s);
     ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
     int32_t* nch = at<int32_t>(ws, W.nchunks);
+    const int64_t S = int64_t(T) * L.k;
 
-    // Launch order: act16_x, router, bucket, gate/up, act16_h, down, combine;
+    // Launch order: router, bucket, act16_x, gate/up, act16_h, down, combine;
     // every launch after the first may start while the one before it runs
     // (programmatic dependent launch) and waits before reading its outputs.
-    mk.mark(st);
-    moe_status s = launch_act16(x, T, L.D, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale),
-                                st, /*after_kernel=*/false);
-    if (s != MOE_OK) return s;
-
     RoutePrep prep;
     memset(&prep, 0, sizeof(prep));
     prep.x_frag = nullptr;
@@ -197,22 +200,27 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     prep.n_zero = 0;
     prep.chunk_tokens = 16;
     prep.routed_chunk_tokens = 8;   // one 8-column n-tile per routed chunk
-    prep.router_after_kernel = true;
+    prep.router_after_kernel = false;
     mk.mark(st);
-    s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                      at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
                      &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
     ++mk.i;
     if (s != MOE_OK) return s;
+    mk.mark(st);
+    s = launch_act16(x, S, L.D, perm, L.k, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale),
+                     st);
+    if (s != MOE_OK) return s;
 
     DecodeMaps m1, m2;
     const uint64_t E = uint64_t(L.E);
-    bool ok = make_tmap_2d(&m1.r0, L.w_gate, false, L.D / 2, E * L.F, 128, 32, true) &&
-              make_tmap_2d(&m1.r1, L.w_up, false, L.D / 2, E * L.F, 128, 32, true) &&
-              make_tmap_2d(&m1.s0, L.ws_gate, true, L.D, L.F_shared, 64, 32, true) &&
-              make_tmap_2d(&m1.s1, L.ws_up, true, L.D, L.F_shared, 64, 32, true) &&
-              make_tmap_2d(&m2.r0, L.w_down, false, L.F / 2, E * L.D, 128, 32, true) &&
-              make_tmap_2d(&m2.s0, L.ws_down, true, L.F_shared, L.D, 64, 32, true);
+    const uint32_t rows = uint32_t(decode_task_rows());
+    bool ok = make_tmap_2d(&m1.r0, L.w_gate, false, L.D / 2, E * L.F, 128, rows, true) &&
+              make_tmap_2d(&m1.r1, L.w_up, false, L.D / 2, E * L.F, 128, rows, true) &&
+              make_tmap_2d(&m1.s0, L.ws_gate, true, L.D, L.F_shared, 64, rows, true) &&
+              make_tmap_2d(&m1.s1, L.ws_up, true, L.D, L.F_shared, 64, rows, true) &&
+              make_tmap_2d(&m2.r0, L.w_down, false, L.F / 2, E * L.D, 128, rows, true) &&
+              make_tmap_2d(&m2.s0, L.ws_down, true, L.F_shared, L.D, 64, rows, true);
     if (!ok) return MOE_ERR_CUDA;
     m2.r1 = m2.r0;
     m2.s1 = m2.s0;
@@ -225,7 +233,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.K_r = L.D;
     p.K_s = L.D;
     p.k_top = L.k;
-    p.scale_buf_floats = 2 * 32 * (L.D / kGroup);
+    p.scale_buf_floats = decode_scale_floats(0, L.D);
     p.chunks = chunks;
     p.n_chunks = nch;
     p.n_shared_chunks = nch + 1;
@@ -250,15 +258,15 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     if (s != MOE_OK) return s;
 
     mk.mark(st);
-    s = launch_act16(h_r, int64_t(T) * L.k, L.F, at<__half>(ws, W.h16), at<float>(ws, W.h_negc),
-                     at<float>(ws, W.h_scale), st, /*after_kernel=*/true);
+    s = launch_act16(h_r, S, L.F, nullptr, 1, at<__half>(ws, W.h16), at<float>(ws, W.h_negc),
+                     at<float>(ws, W.h_scale), st);
     if (s != MOE_OK) return s;
 
     p.n_rows_r = L.D;
     p.n_rows_s = L.D;
     p.K_r = L.F;
     p.K_s = L.F_shared;
-    p.scale_buf_floats = 32 * (L.F / kGroup);
+    p.scale_buf_floats = decode_scale_floats(1, L.F);
     p.b_r = at<bf16>(ws, W.h16);
     p.ldb_r = L.F;
     p.b_s = h_s;
@@ -431,9 +439,7 @@ moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t 
     const int path = choose_path(*layer, T);
     const WsLayout W = ws_layout(*layer, T, path);
     if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (path == PATH_SEL_DECODE && (decode_smem_bytes(2 * 32 * (layer->D / kGroup)) > 227 * 1024 ||
-                                    decode_smem_bytes(32 * (layer->F / kGroup)) > 227 * 1024))
-        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (path == PATH_SEL_DECODE && !decode_fits(*layer)) return MOE_ERR_UNSUPPORTED_SHAPE;
     // the device status word and the zero rows read in place of missing tokens
     if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
         return MOE_ERR_CUDA;
