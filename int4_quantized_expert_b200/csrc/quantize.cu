@@ -44,11 +44,18 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(const float* __restr
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             const float s = fmaxf(m, 1e-6f) * 0.125f;   // exact: division by 8
+            // q = clamp(rint(w / s)) with w / s the IEEE quotient.  |w / s| <= 8,
+            // and y = w * rn(1 / s) lies within 2^-19 of that quotient (two
+            // roundings of at most 2^-24 relative each), so rint gives the same
+            // code unless y is within that distance of a half-integer; those
+            // elements (about 1 in 10^5) take the division itself.
+            const float r = __frcp_rn(s);
             uint32_t packed = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float q = rintf(__fdiv_rn(f[i], s));     // IEEE division, half to even
-                q = fminf(fmaxf(q, -8.0f), 7.0f);
+                float y = f[i] * r;
+                if (fabsf((y - floorf(y)) - 0.5f) < 0x1p-18f) y = __fdiv_rn(f[i], s);
+                const float q = fminf(fmaxf(rintf(y), -8.0f), 7.0f);   // half to even
                 packed |= (uint32_t(int(q)) & 0xFu) << (4 * i);
             }
             reinterpret_cast<uint16_t*>(codes + g * (kGroup / 2))[lane] = uint16_t(packed);

@@ -27,6 +27,38 @@ def test_int4_bit_exact(rows, cols):
     assert np.array_equal(codes.cpu().numpy(), oq.pack_int4(q_ref))
 
 
+def _near_tie_groups(n_groups, seed):
+    """Groups whose quotients w / s sit on or within a few ulps of a
+    half-integer (the places where a quotient one ulp off would round the
+    other way), with scales that are not powers of two."""
+    g = synth.stream(seed, 99)
+    w = np.zeros((n_groups, 128), np.float32)
+    for i in range(n_groups):
+        m = np.float32(g.uniform(0.01, 0.05))
+        s = np.float32(np.maximum(m, np.float32(1e-6)) / np.float32(8.0))
+        k = g.integers(-8, 8, 127).astype(np.float32) + np.float32(0.5)   # half-integers
+        v = (k * s).astype(np.float32)                                     # quotients near k + 1/2
+        steps = g.integers(-3, 4, 127)
+        v = np.array([np.float32(x) for x in v])
+        for j in range(127):                                               # move a few ulps either way
+            for _ in range(abs(int(steps[j]))):
+                v[j] = np.nextafter(v[j], np.float32(np.inf if steps[j] > 0 else -np.inf), dtype=np.float32)
+        v = np.clip(v, -m, m)
+        w[i, 0] = m                                                        # the group maximum
+        w[i, 1:] = v
+    return w
+
+
+def test_int4_bit_exact_near_ties():
+    """Quotients on and a few ulps around half-integers: the GPU's rounding
+    decisions must be those of the IEEE quotient, as in the oracle."""
+    w = _near_tie_groups(512, 5)
+    codes, scales = moe.quantize_int4(torch.from_numpy(w).cuda())
+    q_ref, s_ref = oq.int4_row_quantize(w)
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy(), oq.pack_int4(q_ref))
+
+
 def test_int4_worked_group_on_gpu():
     group = np.zeros((1, 128), np.float32)
     group[0, :6] = [0.3125, 0.4375, -0.0625, 1.0, -1.0, 0.1875]
