@@ -226,19 +226,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                         wrow = (lane < 16 ? p.s0 : p.s1)[int64_t(ce.expert) * p.n_rows + f];
                         tcol = col0 + lane < ce.count ? p.tok_scale[ce.start + col0 + lane] : 0.0f;
                     }
+                    // columns in pairs: lanes 0..15 finish the even column (own
+                    // gate, partner's up), lanes 16..31 the odd one (partner's
+                    // gate, own up) -- one exchange per pair, every lane busy
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float mine = __uint_as_float(v[j]);
-                        if (FP8) mine *= wrow * __shfl_sync(0xffffffffu, tcol, j);
-                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-                        // lanes 0..15 store even columns, lanes 16..31 odd ones
-                        if ((j & 1) == (lane >> 4)) {
-                            const float g = lane < 16 ? mine : other;
-                            const float u = lane < 16 ? other : mine;
-                            const int col = col0 + j;
-                            if (col < ce.count)
-                                p.h_out[int64_t(ce.start + col) * p.n_rows + fpos] = __float2bfloat16_rn(silu_f32(g) * u);
+                    for (int jp = 0; jp < 16; ++jp) {
+                        float a = __uint_as_float(v[2 * jp]), b = __uint_as_float(v[2 * jp + 1]);
+                        if (FP8) {
+                            a *= wrow * __shfl_sync(0xffffffffu, tcol, 2 * jp);
+                            b *= wrow * __shfl_sync(0xffffffffu, tcol, 2 * jp + 1);
                         }
+                        const float recv = __shfl_xor_sync(0xffffffffu, lane < 16 ? b : a, 16);
+                        const float g = lane < 16 ? a : recv;
+                        const float u = lane < 16 ? recv : b;
+                        const int col = col0 + 2 * jp + (lane >> 4);
+                        if (col < ce.count)
+                            p.h_out[int64_t(ce.start + col) * p.n_rows + fpos] = __float2bfloat16_rn(silu_fast(g) * u);
                     }
                 } else if (MODE == TC_DOWN_INT4 || MODE == TC_DOWN_FP8) {
                     const int d = fb * 128 + ew * 32 + lane;
