@@ -38,14 +38,27 @@ constexpr int DC_KPH = 3;                   // K phases
 constexpr int DC_CONSUMERS = DC_RB * DC_KPH;   // 12: 3 warps per SM sub-partition
 // Four warpgroups: warpgroup 0 holds the producer (warp 0, one thread) and
 // gives most of its registers to warpgroups 1 to 3, the 12 consumer warps:
-// 128 x 40 + 384 x 152 <= 512 x 128, the registers the block launches with.
+// 128 x 64 + 384 x 144 <= 512 x 128, the registers the block launches with.
 constexpr int DC_THREADS = 512;
-constexpr int DC_PRODUCER_REGS = 40;
-constexpr int DC_CONSUMER_REGS = 152;
+constexpr int DC_PRODUCER_REGS = 64;
+constexpr int DC_CONSUMER_REGS = 144;
 static_assert(128 * DC_PRODUCER_REGS + 32 * DC_CONSUMERS * DC_CONSUMER_REGS <= DC_THREADS * 128, "register split");
 constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 64 rows x 128 B
-constexpr int DC_STAGE = 2 * DC_CHUNK;      // 16 KB
-constexpr int DC_NSTAGES = 8;               // ring: 128 KB in flight
+constexpr int DC_STAGE = 2 * DC_CHUNK;      // weights of a stage: 16 KB
+constexpr int DC_B_OFF = DC_STAGE;          // then the chunk's token rows for the stage's K range
+// then the rows' int4 group offsets (8 rows x 4 groups) in a 1 KB unit; the
+// token rows take 4 KB (gate/up: 256 K of 8 routed or 64 K of 16 shared rows)
+// or 8 KB (down: 512 K routed, 128 K shared)
+__host__ __device__ constexpr int dc_c_off(int mode) { return DC_B_OFF + (mode == 0 ? 4096 : 8192); }
+__host__ __device__ constexpr int dc_slot(int mode) { return dc_c_off(mode) + 1024; }   // a multiple of 1024
+// Ring depth: a multiple of the K-phase count.  A stage goes to K phase
+// (global stage index) % DC_KPH, so every slot is always consumed by the same
+// phase, in order, and no warp ever waits on a slot's next use while its
+// current one is still in flight (a parity wait one phase too far ahead
+// would return at once).
+__host__ __device__ constexpr int dc_nstages(int mode) { return mode == 0 ? 6 : 6; }
+constexpr int DC_MAX_STAGES = 6;
+static_assert(dc_nstages(0) % DC_KPH == 0 && dc_nstages(1) % DC_KPH == 0, "ring depth vs K phases");
 constexpr int DC_NT = 2;                    // n-tiles of 8 tokens per task
 constexpr int DC_RED_FLOATS = (DC_KPH - 1) * DC_RB * 32 * DC_NT * 8;   // partial sums of K phases 1..2
 
@@ -61,8 +74,8 @@ struct TaskInfo {
 };
 
 struct DecodeSmem {
-    uint64_t full[DC_NSTAGES];
-    uint64_t empty[DC_NSTAGES];
+    uint64_t full[DC_MAX_STAGES];
+    uint64_t empty[DC_MAX_STAGES];
     uint64_t sfull[2];
     uint64_t sempty[2];
     uint64_t red_full;    // K phases 1..2 -> phase 0: partial sums written
@@ -76,170 +89,134 @@ __device__ __forceinline__ uint4 lds128(const unsigned char* p) {
     return *reinterpret_cast<const uint4*>(p);
 }
 
+// The first stage of a task (its stages are it_base, it_base + 1, ...) that
+// belongs to K phase q: phases take stages by their global index.
+__device__ __forceinline__ int first_stage(int q, uint32_t it_base) {
+    return int((uint32_t(q) + DC_KPH - it_base % DC_KPH) % DC_KPH);
+}
+
+// Row pitch (floats) of a task's scale buffer in shared memory.  When a
+// row's K / 128 scales fill whole 16-byte units (ng % 4 == 0), rows are
+// copied one by one to a pitch of 4 x an odd number of floats, which puts
+// the 8 rows a warp reads at once in distinct banks; otherwise the task's
+// rows are one block copy at pitch ng.
+__host__ __device__ __forceinline__ bool scale_rows_padded(int ng) { return ng % 4 == 0; }
+__host__ __device__ __forceinline__ int scale_row_floats(int ng) {
+    return !scale_rows_padded(ng) ? ng : ((ng / 4) % 2 ? ng : ng + 4);
+}
+
 // Address of logical 16-byte chunk j of row r in a 128-byte-swizzled tile.
 __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, int r, int j) {
     return tile + r * 128 + ((j ^ (r & 7)) << 4);
 }
 
 
-// The int4 part of a decode task: the warp's stages q, q + 3, ... of groups
-// of 128 K, NT token tiles.  Returns false if a wait timed out.
+// The int4 part of a decode task: the warp's stages (those of K phase q) of groups
+// of 128 K, one n-tile of 8 tokens.  Returns false if a wait timed out.
 //
 // Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
 // shift and four LOP3s give (k0,k4) and (k2,k6) as 1032 + q and (k1,k5),
-// (k3,k7) as 1152 + 16 q.  The B rows (fp16 tokens, scaled per row by a power
+// (k3,k7) as 1152 + 16 q.  The token rows (fp16, scaled per row by a power
 // of two) store odd positions divided by 16 and every 8-block in the order
 // x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x plus a per-group
 // offset that the partial sum starts from (negc, passed as the MMA's C).
-// Token rows that do not exist point at a zero row, so every load is
-// unconditional; the fragments of the next group are loaded one group ahead.
-template <int MODE, int NT>
+// The stage holds the chunk's 8 token rows for its K range and their group
+// offsets next to the codes; MMA column g is token row sigma8(g).
+template <int MODE>
 __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
                                              const float* sc, uint32_t it_base, int q, int lane, int row_a,
-                                             int row_b, const bf16* const (&brow)[DC_NT],
-                                             const float* const (&crow)[DC_NT][2], float (&acc0)[DC_NT][4],
-                                             float (&acc1)[DC_NT][4], int32_t* status) {
+                                             int row_b, float (&acc0)[4], float (&acc1)[4], int32_t* status) {
     constexpr int GPS = MODE == 0 ? 2 : 4;   // groups per stage
-    const int c = lane & 3;
+    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
+    const int g = lane >> 2, c = lane & 3;
     const int ng = ti.K / kGroup;
-    // byte offsets of this thread's 16-byte chunks in a swizzled 32 x 128 B tile:
-    // chunk 4 gi + c of rows row_a and row_b, for the tile's two groups gi
+    // byte offsets of this thread's 16-byte code chunks in a swizzled 64 x 128 B
+    // tile: chunk 4 gi + c of rows row_a and row_b, for the tile's two groups gi
     uint32_t off_a[2], off_b[2];
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) {
         off_a[gi] = row_a * 128 + (((4 * gi + c) ^ (row_a & 7)) << 4);
         off_b[gi] = row_b * 128 + (((4 * gi + c) ^ (row_b & 7)) << 4);
     }
-    const float* sga_p = sc + row_a * ng;
-    const float* sgb_p = sc + row_b * ng;
-    const float* sua_p = sc + (DC_ROWS + row_a) * ng;
-    const float* sub_p = sc + (DC_ROWS + row_b) * ng;
-    const bf16* xp[NT];
+    const int ldsc = scale_row_floats(ng);   // padded row pitch of the scale buffer
+    const float* sga_p = sc + row_a * ldsc;
+    const float* sgb_p = sc + row_b * ldsc;
+    const float* sua_p = sc + (DC_ROWS + row_a) * ldsc;
+    const float* sub_p = sc + (DC_ROWS + row_b) * ldsc;
+    // token tile: group gl of the stage in boxes 2 gl, 2 gl + 1 (8 rows x 128 B,
+    // 128-byte swizzle); this thread's K chunk 4 c + i of the group is stored
+    // at box i >> 1, chunk c + 4 (i & 1) (see act16_kernel)
+    const int trow = sigma8(g);
+    uint32_t offx[4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) xp[nt] = brow[nt] + 32 * c;
-
-    uint4 xA[NT][4], xB[NT][4];
-    float cA[NT][2], cB[NT][2];
-    auto load = [&](int G, uint4 (&xv)[NT][4], float (&cv)[NT][2]) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) xv[nt][i] = ldg_cached(xp[nt] + G * kGroup + 8 * i);
-            cv[nt][0] = ldg_f32(crow[nt][0] + G);
-            cv[nt][1] = ldg_f32(crow[nt][1] + G);
-        }
-    };
-    auto group = [&](const unsigned char* st, int G, int gi, const unsigned char* tile, int Gn,
-                     uint4 (&xc)[NT][4], float (&cc)[NT][2], uint4 (&xn)[NT][4], float (&cn)[NT][2]) {
-        load(Gn, xn, cn);   // Gn is clamped to a valid group; a final redundant load is harmless
-        const uint4 wa = lds128(tile + off_a[gi]);
-        const uint4 wb = lds128(tile + off_b[gi]);
-        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-        if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
-        const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
-        const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
-        // CH independent accumulation chains per matrix (word jj feeds chain
-        // jj % CH; chain 0 starts from the group offset, the others from
-        // zero).  Every word's even-nibble MMAs are issued before any
-        // odd-nibble one, so consecutive MMAs of a warp do not depend on
-        // each other.
-        constexpr int CH = NT == 1 ? 4 : 2;
-        float pg[CH][NT][4], pu[CH][NT][4];
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
-            const uint32_t ea0 = f16_lo_nibbles(WA[jj]), ea1 = f16_lo_nibbles(WB[jj]);
-            const uint32_t ea2 = f16_lo_nibbles(wa8), ea3 = f16_lo_nibbles(wb8);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float* d = pg[jj % CH][nt];
-                if (jj == 0) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y,
-                                           cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
-                else if (jj < CH) mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
-                else mma_f16_16816(d, ea0, ea1, ea2, ea3, xc[nt][jj].x, xc[nt][jj].y);
-            }
-            if (MODE == 0) {
-                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
-                const uint32_t eu0 = f16_lo_nibbles(VA[jj]), eu1 = f16_lo_nibbles(VB[jj]);
-                const uint32_t eu2 = f16_lo_nibbles(va8), eu3 = f16_lo_nibbles(vb8);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float* d = pu[jj % CH][nt];
-                    if (jj == 0) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y,
-                                               cc[nt][0], cc[nt][1], cc[nt][0], cc[nt][1]);
-                    else if (jj < CH) mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y, 0.f, 0.f, 0.f, 0.f);
-                    else mma_f16_16816(d, eu0, eu1, eu2, eu3, xc[nt][jj].x, xc[nt][jj].y);
-                }
-            }
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
-            const uint32_t oa0 = f16_hi_nibbles(WA[jj]), oa1 = f16_hi_nibbles(WB[jj]);
-            const uint32_t oa2 = f16_hi_nibbles(wa8), oa3 = f16_hi_nibbles(wb8);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                mma_f16_16816(pg[jj % CH][nt], oa0, oa1, oa2, oa3, xc[nt][jj].z, xc[nt][jj].w);
-            if (MODE == 0) {
-                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
-                const uint32_t ou0 = f16_hi_nibbles(VA[jj]), ou1 = f16_hi_nibbles(VB[jj]);
-                const uint32_t ou2 = f16_hi_nibbles(va8), ou3 = f16_hi_nibbles(vb8);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_f16_16816(pu[jj % CH][nt], ou0, ou1, ou2, ou3, xc[nt][jj].z, xc[nt][jj].w);
-            }
-        }
-#pragma unroll
-        for (int k = 1; k < CH; ++k)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    pg[0][nt][r] += pg[k][nt][r];
-                    if (MODE == 0) pu[0][nt][r] += pu[k][nt][r];
-                }
-        const float sga = sga_p[G], sgb = sgb_p[G];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            acc0[nt][0] = fmaf(pg[0][nt][0], sga, acc0[nt][0]);
-            acc0[nt][1] = fmaf(pg[0][nt][1], sga, acc0[nt][1]);
-            acc0[nt][2] = fmaf(pg[0][nt][2], sgb, acc0[nt][2]);
-            acc0[nt][3] = fmaf(pg[0][nt][3], sgb, acc0[nt][3]);
-        }
-        if (MODE == 0) {
-            const float sua = sua_p[G], sub = sub_p[G];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                acc1[nt][0] = fmaf(pu[0][nt][0], sua, acc1[nt][0]);
-                acc1[nt][1] = fmaf(pu[0][nt][1], sua, acc1[nt][1]);
-                acc1[nt][2] = fmaf(pu[0][nt][2], sub, acc1[nt][2]);
-                acc1[nt][3] = fmaf(pu[0][nt][3], sub, acc1[nt][3]);
-            }
-        }
-    };
+    for (int i = 0; i < 4; ++i) offx[i] = (i >> 1) * 1024 + trow * 128 + (((c + 4 * (i & 1)) ^ (trow & 7)) << 4);
+    const int tc0 = sigma8(2 * c), tc1 = sigma8(2 * c + 1);   // token rows of C columns 2c, 2c + 1
 
     bool ok = true;
-    if (q < ti.n_stages) load(q * GPS, xA, cA);
-    for (int s = q; s < ti.n_stages; s += DC_KPH) {
+    for (int s = first_stage(q, it_base); s < ti.n_stages; s += DC_KPH) {
         const uint32_t it = it_base + s;
-        const uint32_t slot = it % DC_NSTAGES;
-        if (!mbar_wait(&sm->full[slot], (it / DC_NSTAGES) & 1, status)) { ok = false; break; }
-        const unsigned char* st = ring + slot * DC_STAGE;
+        const uint32_t slot = it % NST;
+        if (!mbar_wait(&sm->full[slot], (it / NST) & 1, status)) { ok = false; break; }
+        const unsigned char* st = ring + slot * SLOT;
+        const unsigned char* bt = st + DC_B_OFF;
+        const float* ct = reinterpret_cast<const float*>(st + C_OFF);
         const int G0 = s * GPS;
-        const int g_next_stage = min((s + DC_KPH) * GPS, ng - 1);
-        // groups alternate between the A and B fragment buffers; a stage holds
-        // an even number of groups, so every stage starts on A
+        const int cg0 = G0 & 3;   // the offsets tile starts at group G0 rounded down to a multiple of 4
 #pragma unroll
-        for (int gl = 0; gl < GPS; gl += 2) {
-            if (G0 + gl >= ng) break;
+        for (int gl = 0; gl < GPS; ++gl) {
+            const int G = G0 + gl;
+            if (G >= ng) break;
             // MODE 0: both groups in tile 0 (gate) and tile 1 (up);
             // MODE 1: groups 0,1 in tile 0 and 2,3 in tile 1 of the one matrix
             const unsigned char* tile = st + (MODE == 0 ? 0 : (gl >> 1) * DC_CHUNK);
-            group(st, G0 + gl, 0, tile, (gl + 1 < GPS) ? min(G0 + gl + 1, ng - 1) : g_next_stage,
-                  xA, cA, xB, cB);
-            if (G0 + gl + 1 >= ng) break;
-            group(st, G0 + gl + 1, 1, tile, (gl + 2 < GPS) ? min(G0 + gl + 2, ng - 1) : g_next_stage,
-                  xB, cB, xA, cA);
+            const int gi = gl & 1;
+            uint4 xc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xc[i] = lds128(bt + gl * 2048 + offx[i]);
+            const float cc0 = ct[tc0 * 4 + cg0 + gl], cc1 = ct[tc1 * 4 + cg0 + gl];
+            const uint4 wa = lds128(tile + off_a[gi]);
+            const uint4 wb = lds128(tile + off_b[gi]);
+            uint4 va = make_uint4(0, 0, 0, 0), vb = va;
+            if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
+            const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
+            const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
+            // four independent accumulation chains per matrix (word jj feeds
+            // chain jj; chain 0 starts from the group offset, the others from
+            // zero); every word's even-nibble MMAs go before any odd-nibble one
+            float pg[4][4], pu[4][4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
+                const float c0 = jj == 0 ? cc0 : 0.0f, c1 = jj == 0 ? cc1 : 0.0f;
+                mma_f16_16816(pg[jj], f16_lo_nibbles(WA[jj]), f16_lo_nibbles(WB[jj]), f16_lo_nibbles(wa8),
+                              f16_lo_nibbles(wb8), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
+                if (MODE == 0) {
+                    const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                    mma_f16_16816(pu[jj], f16_lo_nibbles(VA[jj]), f16_lo_nibbles(VB[jj]), f16_lo_nibbles(va8),
+                                  f16_lo_nibbles(vb8), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
+                mma_f16_16816(pg[jj], f16_hi_nibbles(WA[jj]), f16_hi_nibbles(WB[jj]), f16_hi_nibbles(wa8),
+                              f16_hi_nibbles(wb8), xc[jj].z, xc[jj].w);
+                if (MODE == 0) {
+                    const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                    mma_f16_16816(pu[jj], f16_hi_nibbles(VA[jj]), f16_hi_nibbles(VB[jj]), f16_hi_nibbles(va8),
+                                  f16_hi_nibbles(vb8), xc[jj].z, xc[jj].w);
+                }
+            }
+            const float sga = sga_p[G], sgb = sgb_p[G];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                acc0[r] = fmaf((pg[0][r] + pg[1][r]) + (pg[2][r] + pg[3][r]), r < 2 ? sga : sgb, acc0[r]);
+            if (MODE == 0) {
+                const float sua = sua_p[G], sub = sub_p[G];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    acc1[r] = fmaf((pu[0][r] + pu[1][r]) + (pu[2][r] + pu[3][r]), r < 2 ? sua : sub, acc1[r]);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->empty[slot]);
@@ -251,19 +228,22 @@ template <int MODE>   // 0 = gate/up with SwiGLU, 1 = down
 __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const __grid_constant__ CUtensorMap tm_r0, const __grid_constant__ CUtensorMap tm_r1,
     const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_s1,
-    DecodeParams p) {
+    const __grid_constant__ CUtensorMap tm_br, const __grid_constant__ CUtensorMap tm_cr,
+    const __grid_constant__ CUtensorMap tm_bs, const __grid_constant__ CUtensorMap tm_g0,
+    const __grid_constant__ CUtensorMap tm_g1, DecodeParams p) {
+    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment of the ring is required by the 128-byte swizzle
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* ring = base;
-    float* sbuf = reinterpret_cast<float*>(ring + DC_NSTAGES * DC_STAGE);      // 2 scale buffers
+    float* sbuf = reinterpret_cast<float*>(ring + NST * SLOT);      // 2 scale buffers
     float* red = sbuf + 2 * p.scale_buf_floats;
     DecodeSmem* sm = reinterpret_cast<DecodeSmem*>(red + DC_RED_FLOATS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < DC_NSTAGES; ++i) { mbar_init(&sm->full[i], 1); mbar_init(&sm->empty[i], DC_RB); }
+        for (int i = 0; i < NST; ++i) { mbar_init(&sm->full[i], 1); mbar_init(&sm->empty[i], DC_RB); }
         for (int i = 0; i < 2; ++i) { mbar_init(&sm->sfull[i], 1); mbar_init(&sm->sempty[i], DC_CONSUMERS); }
         mbar_init(&sm->red_full, (DC_KPH - 1) * DC_RB);
         mbar_init(&sm->red_empty, DC_RB);
@@ -283,6 +263,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(DC_PRODUCER_REGS));
         if (warp == 0 && lane == 0) {
             prefetch_tmap(&tm_r0); prefetch_tmap(&tm_r1); prefetch_tmap(&tm_s0); prefetch_tmap(&tm_s1);
+            prefetch_tmap(&tm_br); prefetch_tmap(&tm_cr); prefetch_tmap(&tm_bs);
+            prefetch_tmap(&tm_g0); prefetch_tmap(&tm_g1);
             uint32_t it = 0;
             bool ok = true, waited = false;
             int n_tasks = n_sh * nbs;   // grows by the routed tasks after the wait
@@ -330,39 +312,57 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const CUtensorMap* m1 = ti.kind ? &tm_r1 : &tm_s1;
                 const int grow = ti.kind ? ti.expert * p.n_rows_r + ti.row0 : ti.row0;   // global tile row
                 if (ti.kind) {
-                    const int ng = ti.K / kGroup;
-                    const uint32_t bytes = uint32_t(DC_ROWS * ng * 4);
+                    // one bulk copy per scale row, rows ldsc floats apart in
+                    // shared memory so a warp's 8 rows fall in distinct banks
+                    const int ng = ti.K / kGroup, ldsc = scale_row_floats(ng);
+                    const uint32_t row_bytes = uint32_t(ng * 4);
                     float* dst = sbuf + b * p.scale_buf_floats;
-                    mbar_arrive_expect_tx(&sm->sfull[b], (MODE == 0 ? 2 : 1) * bytes);
-                    bulk_load(dst, p.sc0 + int64_t(grow) * ng, bytes, &sm->sfull[b]);
-                    if (MODE == 0) bulk_load(dst + DC_ROWS * ng, p.sc1 + int64_t(grow) * ng, bytes, &sm->sfull[b]);
+                    mbar_arrive_expect_tx(&sm->sfull[b], (MODE == 0 ? 2 : 1) * DC_ROWS * uint32_t(ldsc * 4));
+                    for (int m = 0; m < (MODE == 0 ? 2 : 1); ++m) {
+                        float* d = dst + m * DC_ROWS * ldsc;
+                        if (scale_rows_padded(ng))   // one box of ldsc x 64: columns past ng read as zeros
+                            tma_load_2d(d, m ? &tm_g1 : &tm_g0, &sm->sfull[b], 0, grow);
+                        else                         // 64 rows at pitch ng: a multiple of 16 bytes
+                            bulk_load(d, (m ? p.sc1 : p.sc0) + int64_t(grow) * ng, DC_ROWS * row_bytes, &sm->sfull[b]);
+                    }
                 } else {
                     mbar_arrive(&sm->sfull[b]);
                 }
                 const int kbytes = ti.kind ? 128 : 64;   // tile x extent in elements (uint8 codes / bf16)
+                // token rows of the chunk (8 routed, 16 shared) for the stage's K range,
+                // in boxes of 64 K; routed stages also carry the rows' group offsets
+                const int kstage = (MODE == 0 ? 1 : 2) * kchunk;   // K values per stage
+                const int nbox = kstage / 64;
+                const uint32_t box_bytes = ti.kind ? 1024u : 2048u;
+                const uint32_t b_bytes = uint32_t(nbox) * box_bytes + (ti.kind ? 128u : 0u);
+                const CUtensorMap* mb = ti.kind ? &tm_br : &tm_bs;
                 for (int s = 0; s < ti.n_stages; ++s, ++it) {
-                    const uint32_t slot = it % DC_NSTAGES;
-                    if (!mbar_wait(&sm->empty[slot], ((it / DC_NSTAGES) & 1) ^ 1, p.status, 128)) { ok = false; break; }
-                    unsigned char* st = ring + slot * DC_STAGE;
+                    const uint32_t slot = it % NST;
+                    if (!mbar_wait(&sm->empty[slot], ((it / NST) & 1) ^ 1, p.status, 128)) { ok = false; break; }
+                    unsigned char* st = ring + slot * SLOT;
                     if (MODE == 0) {
-                        mbar_arrive_expect_tx(&sm->full[slot], DC_STAGE);
+                        mbar_arrive_expect_tx(&sm->full[slot], DC_STAGE + b_bytes);
                         tma_load_2d(st, m0, &sm->full[slot], s * kbytes, grow);
                         tma_load_2d(st + DC_CHUNK, m1, &sm->full[slot], s * kbytes, grow);
                     } else {
                         // two consecutive K tiles of the one matrix; the second only if in range
                         const bool second = (2 * s + 1) * kchunk < ti.K;
-                        mbar_arrive_expect_tx(&sm->full[slot], second ? DC_STAGE : DC_CHUNK);
+                        mbar_arrive_expect_tx(&sm->full[slot], (second ? DC_STAGE : DC_CHUNK) + b_bytes);
                         tma_load_2d(st, m0, &sm->full[slot], 2 * s * kbytes, grow);
                         if (second) tma_load_2d(st + DC_CHUNK, m0, &sm->full[slot], (2 * s + 1) * kbytes, grow);
                     }
+                    // one 3-D box: nbox 64-K chunks x the chunk's rows (chunks beyond K read zeros)
+                    tma_load_3d(st + DC_B_OFF, mb, &sm->full[slot], 0, ti.start, s * kstage / 64);
+                    if (ti.kind)   // group offsets: 4 groups from the stage's first, rounded down to a multiple of 4
+                        tma_load_2d(st + C_OFF, &tm_cr, &sm->full[slot], (s * kstage / kGroup) & ~3, ti.start);
                 }
             }
             // this grid completes only after the kernels before it
             if (!waited) griddep_wait();
             // wind down: wait (bounded) for every stage still in flight to land
-            for (uint32_t i = 0; i < DC_NSTAGES && i < it; ++i) {
+            for (uint32_t i = 0; i < NST && i < it; ++i) {
                 const uint32_t j = it - 1 - i;
-                mbar_wait(&sm->full[j % DC_NSTAGES], (j / DC_NSTAGES) & 1, nullptr);
+                mbar_wait(&sm->full[j % NST], (j / NST) & 1, nullptr);
             }
         }
         return;
@@ -390,31 +390,15 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         const float* sc = sbuf + b * p.scale_buf_floats;
         const int ng = ti.K / kGroup;
 
-        // B rows (tokens) of this chunk for the two n-tiles: column n = g of each
-        // (16-bit elements: bf16 for the shared expert, fp16 for routed ones).
-        // Routed tasks also need, for the C columns 2c and 2c + 1, the group
-        // offsets (negc) and the rows' power-of-two scales.
-        const bf16* brow[DC_NT];
-        const float* crow[DC_NT][2];
-        float cscale[DC_NT][2];
-#pragma unroll
-        for (int nt = 0; nt < DC_NT; ++nt) {
-            const int i = nt * 8 + g;
-            brow[nt] = p.zero_row;          // tokens beyond the chunk read zeros
-            if (i < ti.count) {
-                if (ti.kind == 0) brow[nt] = p.b_s + int64_t(ti.start + i) * p.ldb_s;
-                else brow[nt] = p.b_r + int64_t(ti.start + i) * p.ldb_r;   // routed rows by position
-            }
+        // MMA column g of n-tile nt is token row nt * 8 + sigma8(g) of the chunk;
+        // routed results are rescaled per token by their row's power of two
+        // (C columns 2c and 2c + 1 of this thread)
+        float cscale[2] = {1.0f, 1.0f};
+        if (ti.kind == 1) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int ic = nt * 8 + 2 * c + h;
-                crow[nt][h] = p.zero_corr;
-                cscale[nt][h] = 1.0f;
-                if (ti.kind == 1 && ic < ti.count) {
-                    const int64_t row = ti.start + ic;
-                    crow[nt][h] = p.corr_r + row * ng;
-                    cscale[nt][h] = p.rscale_r[row];
-                }
+                const int tok = sigma8(2 * c + h);
+                if (tok < ti.count) cscale[h] = p.rscale_r[ti.start + tok];
             }
         }
         const int nt_used = ti.count > 8 ? 2 : 1;
@@ -428,37 +412,30 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         bool ok = true;
         if (ti.kind == 1) {
             // routed chunks hold at most 8 tokens: one n-tile
-            ok = consume_int4<MODE, 1>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, brow, crow, acc0, acc1,
-                                       p.status);
+            ok = consume_int4<MODE>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, acc0[0], acc1[0], p.status);
         } else {
             // ---------------- bf16 weights (shared expert): 64 K per tile ----------------
-            // thread c takes the 8-blocks c and c + 4 of each 64-K tile
+            // thread c takes the 8-blocks c and c + 4 of each 64-K tile, of the
+            // weight rows and of its token rows nt * 8 + sigma8(g) (in the stage)
             constexpr int UPS = MODE == 0 ? 1 : 2;           // 64-K units per stage
             const int n_units = ti.K / 64;
-            uint4 xc[DC_NT][2], xn[DC_NT][2];
-            auto load = [&](int U, uint4 (&xv)[DC_NT][2]) {
-#pragma unroll
-                for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2)
-                        xv[nt][h2] = (nt < nt_used && brow[nt]) ? ldg_cached(brow[nt] + U * 64 + 8 * (c + 4 * h2))
-                                                                : make_uint4(0, 0, 0, 0);
-            };
-            if (q < ti.n_stages) load(q * UPS, xc);
-            for (int s = q; s < ti.n_stages; s += DC_KPH) {
+            const int trow = sigma8(g);
+            for (int s = first_stage(q, it_base); s < ti.n_stages; s += DC_KPH) {
                 const uint32_t it = it_base + s;
-                const uint32_t slot = it % DC_NSTAGES;
-                if (!mbar_wait(&sm->full[slot], (it / DC_NSTAGES) & 1, p.status)) { ok = false; break; }
-                const unsigned char* st = ring + slot * DC_STAGE;
+                const uint32_t slot = it % NST;
+                if (!mbar_wait(&sm->full[slot], (it / NST) & 1, p.status)) { ok = false; break; }
+                const unsigned char* st = ring + slot * SLOT;
 #pragma unroll
                 for (int ul = 0; ul < UPS; ++ul) {
                     const int U = s * UPS + ul;
                     if (U >= n_units) break;
-                    int Un = -1;
-                    if (ul + 1 < UPS) Un = U + 1;
-                    else if (s + DC_KPH < ti.n_stages) Un = (s + DC_KPH) * UPS;
-                    if (Un >= 0 && Un < n_units) load(Un, xn);
                     const unsigned char* ta = st + (MODE == 0 ? 0 : ul * DC_CHUNK);
+                    const unsigned char* tb = st + DC_B_OFF + ul * 2048;   // 16 token rows x 64 K
+                    uint4 xc[DC_NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < DC_NT; ++nt)
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) xc[nt][h2] = lds128(swz(tb, nt * 8 + trow, c + 4 * h2));
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int j = c + 4 * h2;
@@ -492,10 +469,6 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                             }
                         }
                     }
-#pragma unroll
-                    for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) xc[nt][h2] = xn[nt][h2];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->empty[slot]);
@@ -523,17 +496,18 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 #pragma unroll
                     for (int r = 0; r < 4; ++r) { acc0[nt][r] += o[nt * 8 + r]; acc1[nt][r] += o[nt * 8 + 4 + r]; }
             }
-            // ---- epilogue: C rows (row_a, row_b) x token columns (2c, 2c + 1) of each n-tile ----
-            // routed results are rescaled by their B row's power of two;
+            // ---- epilogue: C rows (row_a, row_b) x columns (2c, 2c + 1) of each n-tile,
+            // column n of n-tile nt being token nt * 8 + sigma8(n) of the chunk ----
+            // routed results are rescaled by their token row's power of two;
             // h is stored in natural order (the routed rows' fp16 copy is made next)
 #pragma unroll
             for (int nt = 0; nt < DC_NT; ++nt) {
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const int col = nt * 8 + 2 * c + (r & 1);
+                    const int col = nt * 8 + sigma8(2 * c + (r & 1));
                     if (col >= ti.count) continue;
                     const int n = ti.row0 + (r < 2 ? row_a : row_b);
-                    const float cs = cscale[nt][r & 1];
+                    const float cs = cscale[r & 1];   // 1 for the shared expert (one n-tile for routed chunks)
                     if (MODE == 0) {
                         if (ti.kind == 1) {
                             const float hv = silu_f32(acc0[nt][r] * cs) * (acc1[nt][r] * cs);
@@ -588,11 +562,15 @@ int decode_max_chunks(int T, int k, int E) { return int(ceil_div(T, 16)) + int(c
 
 int decode_task_rows() { return DC_ROWS; }
 
-// floats of one task's int4 scale buffer: gate and up rows (mode 0) or down rows
-int decode_scale_floats(int mode, int K) { return (mode == 0 ? 2 : 1) * DC_ROWS * (K / kGroup); }
+// scale_row_floats(K / 128) if the task scales load as one padded box, else 0
+int decode_scale_pitch(int K) { return scale_rows_padded(K / kGroup) ? scale_row_floats(K / kGroup) : 0; }
 
-size_t decode_smem_bytes(int scale_buf_floats) {
-    return 1024 + size_t(DC_NSTAGES) * DC_STAGE + 2 * size_t(scale_buf_floats) * 4 + DC_RED_FLOATS * 4 +
+// floats of one task's int4 scale buffer: gate and up rows (mode 0) or down
+// rows, each row padded to scale_row_floats(K / 128)
+int decode_scale_floats(int mode, int K) { return (mode == 0 ? 2 : 1) * DC_ROWS * scale_row_floats(K / kGroup); }
+
+size_t decode_smem_bytes(int mode, int scale_buf_floats) {
+    return 1024 + size_t(dc_nstages(mode)) * dc_slot(mode) + 2 * size_t(scale_buf_floats) * 4 + DC_RED_FLOATS * 4 +
            sizeof(DecodeSmem);
 }
 
@@ -615,20 +593,41 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D map over a row-major [rows, inner] matrix; box = box_inner x box_rows.
-bool make_tmap_2d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t inner, uint64_t rows,
+// 2-D map over a row-major [rows, inner] matrix of 1-, 2- or 4-byte elements;
+// box = box_inner x box_rows.
+bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
-    const uint64_t esz = bf16_elems ? 2 : 1;
+    const uint64_t esz = uint64_t(elem_bytes);
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {inner * esz};
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, bf16_elems ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+    const CUtensorMapDataType dt = elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(m, dt, 2,
                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 3-D map over fp16/bf16 token rows [rows, K] seen as (64 K values, row,
+// 64-K chunk): a box of box_rows rows x nbox chunks lands as nbox tiles of
+// box_rows x 128 bytes, each with the 128-byte swizzle.
+bool make_tmap_rows_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+                       uint32_t nbox) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, rows, K / 64};
+    cuuint64_t strides[2] = {K * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, nbox};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -636,12 +635,13 @@ moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParam
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = decode_smem_bytes(prm.scale_buf_floats);
+    const size_t smem = decode_smem_bytes(mode, prm.scale_buf_floats);
     cudaError_t e;
     auto kern = mode == 0 ? decode_ffn_kernel<0> : decode_ffn_kernel<1>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    return launch_pdl(kern, dim3(sms), dim3(DC_THREADS), smem, stream, maps.r0, maps.r1, maps.s0, maps.s1, prm);
+    return launch_pdl(kern, dim3(sms), dim3(DC_THREADS), smem, stream, maps.r0, maps.r1, maps.s0, maps.s1, maps.br,
+                      maps.cr, maps.bs, maps.g0, maps.g1, prm);
 }
 
 moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
@@ -666,10 +666,14 @@ namespace moe {
 //           scaled row stays below 2^15 (fp16 keeps every bf16 value exactly
 //           in that range); rscale[r] = 2^e undoes it on the MMA results;
 //   out16  every 8-block stored as x0 x4 x2 x6 x1/16 x5/16 x3/16 x7/16 (scaled)
-//          -- the K order and the 1/16 factors the int4 unpacking expects;
+//          -- the K order and the 1/16 factors the int4 unpacking expects --
+//          and, inside each group of 128, 8-block 4 c + i (c, i = 0..3) stored
+//          at 8-block 8 (i >> 1) + c + 4 (i & 1), so that the four threads c
+//          of an MMA fragment read distinct shared-memory banks;
 //   negc   per group of 128: -(1032 * sum of the even-position stored values
 //          + 1152 * sum of the odd-position stored values), the offset the
-//          unpacked codes (1032 + q and 1152 + 16 q) add to a dot product.
+//          unpacked codes (1032 + q and 1152 + 16 q) add to a dot product;
+//          rows of act16_negc_pitch(cols) floats.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in, int cols,
                                                     const int32_t* __restrict__ src_perm, int k,
@@ -719,12 +723,14 @@ __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in,
                 h[i] = __float2half_rn(s);
                 if (i < 4) ev += __half2float(h[i]); else od += __half2float(h[i]);
             }
-            *reinterpret_cast<uint4*>(out16 + r * cols + 8 * b) = *reinterpret_cast<const uint4*>(h);
+            const int lc = b & 15, ci = lc >> 2, ii = lc & 3;
+            const int sb = (b & ~15) + 8 * (ii >> 1) + ci + 4 * (ii & 1);
+            *reinterpret_cast<uint4*>(out16 + r * cols + 8 * sb) = *reinterpret_cast<const uint4*>(h);
         }
         float cs = 1032.0f * ev + 1152.0f * od;
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
-        if (b < nblk && (threadIdx.x & 15) == 0) negc[r * (cols / kGroup) + b / 16] = -cs;
+        if (b < nblk && (threadIdx.x & 15) == 0) negc[r * act16_negc_pitch(cols) + b / 16] = -cs;
     }
 }
 

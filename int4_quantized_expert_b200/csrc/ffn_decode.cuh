@@ -26,24 +26,16 @@ struct DecodeParams {
     int32_t scale_buf_floats;
     const ChunkEntry* chunks;
     const int32_t* n_chunks;
-    const int32_t* n_shared_chunks;
     const int32_t* perm;    // sorted position -> slot (t * k + j)
     const float* gates;     // per slot
-    const bf16* b_r;        // B rows, routed, by sorted position (fp16 bits; see act16): tokens or h rows
-    int32_t ldb_r;
-    const bf16* b_s;        // B rows, shared: gate/up: tokens; down: shared h rows
-    int32_t ldb_s;
     const float* sc0;       // routed scales: gate/up: gate; down: down   ([E * rows, K / 128])
     const float* sc1;       // routed scales: gate/up: up
-    const float* corr_r;    // routed B rows (by position): group offsets negc [rows, K_r / 128] (see act16)
-    const float* rscale_r;  // routed B rows (by position): power-of-two scale of each row
-    bf16* h_r;              // gate/up outputs: routed [T*k, F] (natural order), shared [T, F_shared] (fragment order)
+    const float* rscale_r;  // routed token rows (by position): power-of-two scale of each row
+    bf16* h_r;              // gate/up outputs: routed [T*k, F] by position, shared [T, F_shared]
     bf16* h_s;
-    float* y_r;             // down outputs: routed gate * y [T*k, D] (by position), shared [T, D]
+    float* y_r;             // down outputs: routed gate * y [T*k, D] by position, shared [T, D]
     float* y_s;
-    const bf16* zero_row;   // zeros, at least max(K_r, K_s) long: B row of a token that does not exist
-    const float* zero_corr; // zeros, at least K_r / 128 long
-    int32_t* task_counter;  // zeroed by the routing step
+    int32_t* task_counter;  // cleared with the status word
     int32_t* status;        // device status word
 };
 
@@ -59,14 +51,30 @@ struct RoutePrep {
     bool router_after_kernel;   // the router may start while the kernel before it runs
 };
 
+// TMA maps of one weight-streaming launch:
+//   r0, r1  routed int4 codes uint8 [E * rows, K / 2] (gate, up; or down), box 128 B x 64 rows, 128-B swizzle
+//   s0, s1  shared bf16 weights, box 64 x 64, 128-B swizzle
+//   br      routed token rows, fp16 [T * k, K] by position (act16 layout), 3-D box of 8 rows x the
+//           stage's 64-K chunks (make_tmap_rows_3d)
+//   cr      their group offsets, fp32 [T * k, act16_negc_pitch(K)], box 4 x 8
+//   bs      shared-expert token rows, bf16 [T, K] (x, or the shared h), 3-D box of 16 rows x chunks
+//   g0, g1  routed int4 scales fp32 [E * rows, K / 128] (gate, up; or down), box
+//           scale_row_floats(K / 128) x 64 (when K / 128 is a multiple of 4)
 struct DecodeMaps {
-    CUtensorMap r0, r1, s0, s1;   // routed tile maps (int4 codes) and shared maps (bf16)
+    CUtensorMap r0, r1, s0, s1, br, cr, bs, g0, g1;
 };
 
-bool make_tmap_2d(CUtensorMap* m, const void* base, bool bf16_elems, uint64_t inner, uint64_t rows,
+// Row pitch (floats) of act16's group offsets: K / 128 rounded up to 4, so
+// every row starts on 16 bytes.
+__host__ __device__ inline int act16_negc_pitch(int cols) { return int(ceil_div(cols / kGroup, 4) * 4); }
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+bool make_tmap_rows_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+                       uint32_t nbox);
+int decode_scale_pitch(int K);
 int decode_max_chunks(int T, int k, int E);
-size_t decode_smem_bytes(int scale_buf_floats);
+size_t decode_smem_bytes(int mode, int scale_buf_floats);
 int decode_task_rows();
 int decode_scale_floats(int mode, int K);
 moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParams& prm, cudaStream_t stream);

@@ -83,11 +83,11 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
         w.x16 = take(S * L.D * 2);                 // tokens by expert-sorted position
-        w.x_negc = take(S * (L.D / kGroup) * 4);
+        w.x_negc = take(S * act16_negc_pitch(L.D) * 4);
         w.x_scale = take(S * 4);
         w.h_r = take(S * L.F * 2);
         w.h16 = take(S * L.F * 2);
-        w.h_negc = take(S * (L.F / kGroup) * 4);
+        w.h_negc = take(S * act16_negc_pitch(L.F) * 4);
         w.h_scale = take(S * 4);
         w.h_s = take(T * L.F_shared * 2);
         w.y_r = take(S * L.D * 4);
@@ -125,8 +125,8 @@ size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
 
 // The weight-streaming kernels keep a task's int4 scales in shared memory.
 bool decode_fits(const moe_layer_desc& L) {
-    return decode_smem_bytes(decode_scale_floats(0, L.D)) <= kMaxDecodeSmem &&
-           decode_smem_bytes(decode_scale_floats(1, L.F)) <= kMaxDecodeSmem;
+    return decode_smem_bytes(0, decode_scale_floats(0, L.D)) <= kMaxDecodeSmem &&
+           decode_smem_bytes(1, decode_scale_floats(1, L.F)) <= kMaxDecodeSmem;
 }
 
 int choose_path(const moe_layer_desc& L, int64_t T) {
@@ -215,15 +215,30 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     DecodeMaps m1, m2;
     const uint64_t E = uint64_t(L.E);
     const uint32_t rows = uint32_t(decode_task_rows());
-    bool ok = make_tmap_2d(&m1.r0, L.w_gate, false, L.D / 2, E * L.F, 128, rows, true) &&
-              make_tmap_2d(&m1.r1, L.w_up, false, L.D / 2, E * L.F, 128, rows, true) &&
-              make_tmap_2d(&m1.s0, L.ws_gate, true, L.D, L.F_shared, 64, rows, true) &&
-              make_tmap_2d(&m1.s1, L.ws_up, true, L.D, L.F_shared, 64, rows, true) &&
-              make_tmap_2d(&m2.r0, L.w_down, false, L.F / 2, E * L.D, 128, rows, true) &&
-              make_tmap_2d(&m2.s0, L.ws_down, true, L.F_shared, L.D, 64, rows, true);
+    // weights; token rows (8 per routed chunk, 16 per shared chunk) and group offsets
+    bool ok = make_tmap_2d(&m1.r0, L.w_gate, 1, L.D / 2, E * L.F, 128, rows, true) &&
+              make_tmap_2d(&m1.r1, L.w_up, 1, L.D / 2, E * L.F, 128, rows, true) &&
+              make_tmap_2d(&m1.s0, L.ws_gate, 2, L.D, L.F_shared, 64, rows, true) &&
+              make_tmap_2d(&m1.s1, L.ws_up, 2, L.D, L.F_shared, 64, rows, true) &&
+              make_tmap_rows_3d(&m1.br, at<__half>(ws, W.x16), L.D, S, 8, 4) &&
+              make_tmap_2d(&m1.cr, at<float>(ws, W.x_negc), 4, act16_negc_pitch(L.D), S, 4, 8, false) &&
+              make_tmap_rows_3d(&m1.bs, x, L.D, T, 16, 1) &&
+              make_tmap_2d(&m2.r0, L.w_down, 1, L.F / 2, E * L.D, 128, rows, true) &&
+              make_tmap_2d(&m2.s0, L.ws_down, 2, L.F_shared, L.D, 64, rows, true) &&
+              make_tmap_rows_3d(&m2.br, at<__half>(ws, W.h16), L.F, S, 8, 8) &&
+              make_tmap_2d(&m2.cr, at<float>(ws, W.h_negc), 4, act16_negc_pitch(L.F), S, 4, 8, false) &&
+              make_tmap_rows_3d(&m2.bs, h_s, L.F_shared, T, 16, 2);
+    // the task scales: one box per matrix when their rows are whole 16-byte units
+    const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
+    if (pd) ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / kGroup, E * L.F, pd, rows, false) &&
+                 make_tmap_2d(&m1.g1, L.s_up, 4, L.D / kGroup, E * L.F, pd, rows, false);
+    else m1.g0 = m1.g1 = m1.r0;   // unused: the scales come by bulk copy
+    if (pf) ok = ok && make_tmap_2d(&m2.g0, L.s_down, 4, L.F / kGroup, E * L.D, pf, rows, false);
+    else m2.g0 = m2.r0;
     if (!ok) return MOE_ERR_CUDA;
     m2.r1 = m2.r0;
     m2.s1 = m2.s0;
+    m2.g1 = m2.g0;
 
     DecodeParams p;
     memset(&p, 0, sizeof(p));
@@ -236,21 +251,13 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.scale_buf_floats = decode_scale_floats(0, L.D);
     p.chunks = chunks;
     p.n_chunks = nch;
-    p.n_shared_chunks = nch + 1;
     p.perm = perm;
     p.gates = gates;
-    p.b_r = at<bf16>(ws, W.x16);
-    p.ldb_r = L.D;
-    p.b_s = x;   // the shared expert reads the layer input itself
-    p.ldb_s = L.D;
     p.sc0 = L.s_gate;
     p.sc1 = L.s_up;
-    p.corr_r = at<float>(ws, W.x_negc);
     p.rscale_r = at<float>(ws, W.x_scale);
     p.h_r = h_r;
     p.h_s = h_s;
-    p.zero_row = at<bf16>(ws, W.zeros);
-    p.zero_corr = at<float>(ws, W.zero_corr);
     p.task_counter = counters;
     p.status = status;
     mk.mark(st);
@@ -267,13 +274,8 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.K_r = L.F;
     p.K_s = L.F_shared;
     p.scale_buf_floats = decode_scale_floats(1, L.F);
-    p.b_r = at<bf16>(ws, W.h16);
-    p.ldb_r = L.F;
-    p.b_s = h_s;
-    p.ldb_s = L.F_shared;
     p.sc0 = L.s_down;
     p.sc1 = nullptr;
-    p.corr_r = at<float>(ws, W.h_negc);
     p.rscale_r = at<float>(ws, W.h_scale);
     p.y_r = y_r;
     p.y_s = y_s;
@@ -353,22 +355,22 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     TcMaps m_gu, m_dn, m_sgu, m_sdn;
     bool ok;
     if (fp8)
-        ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), false, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D, E * L.F, 128, 16, true) &&
-             make_tmap_2d(&m_gu.a1, L.w_up, false, L.D, E * L.F, 128, 16, true) &&
-             make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), false, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_dn.a0, L.w_down, false, L.F, E * L.D, 128, 16, true);
+        ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), 1, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D, E * L.F, 128, 16, true) &&
+             make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D, E * L.F, 128, 16, true) &&
+             make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), 1, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F, E * L.D, 128, 16, true);
     else
-        ok = make_tmap_2d(&m_gu.b, x_sorted, true, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_gu.a0, L.w_gate, false, L.D / 2, E * L.F, 32, 64, false) &&
-             make_tmap_2d(&m_gu.a1, L.w_up, false, L.D / 2, E * L.F, 32, 64, false) &&
-             make_tmap_2d(&m_dn.b, h_sorted, true, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_dn.a0, L.w_down, false, L.F / 2, E * L.D, 32, 64, false);
-    ok = ok && make_tmap_2d(&m_sgu.b, x_pad, true, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_sgu.a0, L.ws_gate, true, L.D, L.F_shared, 64, 16, true) &&
-              make_tmap_2d(&m_sgu.a1, L.ws_up, true, L.D, L.F_shared, 64, 16, true) &&
-              make_tmap_2d(&m_sdn.b, h_s, true, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_sdn.a0, L.ws_down, true, L.F_shared, L.D, 64, 16, true);
+        ok = make_tmap_2d(&m_gu.b, x_sorted, 2, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D / 2, E * L.F, 32, 64, false) &&
+             make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D / 2, E * L.F, 32, 64, false) &&
+             make_tmap_2d(&m_dn.b, h_sorted, 2, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+             make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
+    ok = ok && make_tmap_2d(&m_sgu.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
+              make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
+              make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+              make_tmap_2d(&m_sdn.a0, L.ws_down, 2, L.F_shared, L.D, 64, 16, true);
     if (!ok) return MOE_ERR_CUDA;
     m_dn.a1 = m_dn.a0;
     m_sdn.a1 = m_sdn.a0;
