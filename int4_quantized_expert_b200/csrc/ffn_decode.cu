@@ -636,10 +636,8 @@ moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParam
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = decode_smem_bytes(mode, prm.scale_buf_floats);
-    cudaError_t e;
     auto kern = mode == 0 ? decode_ffn_kernel<0> : decode_ffn_kernel<1>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (allow_max_smem(kern) != MOE_OK) return MOE_ERR_CUDA;
     return launch_pdl(kern, dim3(sms), dim3(DC_THREADS), smem, stream, maps.r0, maps.r1, maps.s0, maps.s1, maps.br,
                       maps.cr, maps.bs, maps.g0, maps.g1, prm);
 }

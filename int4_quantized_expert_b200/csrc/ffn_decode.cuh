@@ -49,6 +49,8 @@ struct RoutePrep {
     int32_t* zero_words;  // zeroed by the bucketing kernel (or null)
     int32_t n_zero;
     bool router_after_kernel;   // the router may start while the kernel before it runs
+    float* router_part;         // router_partial_floats(T, D, E) floats for a K-split router (or null)
+    int32_t* router_tile_cnt;   // ceil(T / 16) counters, zero on entry (with router_part)
 };
 
 // TMA maps of one weight-streaming launch:
@@ -74,6 +76,8 @@ bool make_tmap_rows_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t ro
                        uint32_t nbox);
 int decode_scale_pitch(int K);
 int decode_max_chunks(int T, int k, int E);
+int router_ksplit(int T, int D);
+size_t router_partial_floats(int T, int D, int E);
 size_t decode_smem_bytes(int mode, int scale_buf_floats);
 int decode_task_rows();
 int decode_scale_floats(int mode, int K);

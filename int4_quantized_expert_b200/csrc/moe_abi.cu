@@ -40,7 +40,7 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
 // are shared by both paths; the rest is laid out per path from there, and a
 // workspace must be large enough for either.
 struct WsLayout {
-    size_t status, zeros, zero_corr, zeros_end, counters, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t status, rt_cnt, zeros_end, counters, rt_part, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
     size_t common_end;
     // weight-streaming path
     size_t x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
@@ -68,10 +68,10 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     const int64_t T_pad = ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
     w.status = take(64);
     w.counters = take(64);   // task counters of the weight-streaming kernels
-    const int maxdim = L.D > L.F ? (L.D > L.F_shared ? L.D : L.F_shared) : (L.F > L.F_shared ? L.F : L.F_shared);
-    w.zeros = take(size_t(maxdim) * 2);
-    w.zero_corr = take(size_t(maxdim / kGroup) * 4);
+    const bool rt_split = router_ksplit(int(T), L.D) > 1;
+    w.rt_cnt = take(rt_split ? size_t(ceil_div(T, 16)) * 4 : 0);   // router tile counters
     w.zeros_end = off;   // [status, zeros_end) is cleared at the start of every call
+    w.rt_part = take(router_partial_floats(int(T), L.D, L.E) * 4);
     w.ids = take(S * 4);
     w.gates = take(S * 4);
     w.counts = take(size_t(L.E) * 4);
@@ -173,6 +173,34 @@ T* at(void* base, size_t off) {
     return reinterpret_cast<T*>(static_cast<unsigned char*>(base) + off);
 }
 
+// A launch's tensor maps depend only on the layer description, the workspace,
+// the input pointer, T and the path; a call with the same ones reuses them.
+struct MapCacheKey {
+    moe_layer_desc L;
+    const void* ws;
+    const void* x;
+    int64_t T;
+    int path;
+    bool valid;
+};
+
+MapCacheKey make_key(const moe_layer_desc& L, const void* ws, const void* x, int64_t T, int path) {
+    MapCacheKey k;
+    memset(&k, 0, sizeof(k));
+    memcpy(&k.L, &L, sizeof(L));
+    k.ws = ws;
+    k.x = x;
+    k.T = T;
+    k.path = path;
+    k.valid = true;
+    return k;
+}
+
+bool same_key(const MapCacheKey& a, const MapCacheKey& b) {
+    return a.valid && b.valid && memcmp(&a.L, &b.L, sizeof(a.L)) == 0 && a.ws == b.ws && a.x == b.x &&
+           a.T == b.T && a.path == b.path;
+}
+
 moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
                            const WsLayout& W, cudaStream_t st, Marks& mk) {
     int32_t* status = at<int32_t>(ws, W.status);
@@ -193,6 +221,10 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     // (programmatic dependent launch) and waits before reading its outputs.
     RoutePrep prep;
     memset(&prep, 0, sizeof(prep));
+    if (W.rt_cnt != W.zeros_end) {   // K-split router (few token tiles)
+        prep.router_part = at<float>(ws, W.rt_part);
+        prep.router_tile_cnt = at<int32_t>(ws, W.rt_cnt);
+    }
     prep.x_frag = nullptr;
     prep.chunks = chunks;
     prep.n_chunks = nch;
@@ -212,33 +244,46 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
                      st);
     if (s != MOE_OK) return s;
 
-    DecodeMaps m1, m2;
-    const uint64_t E = uint64_t(L.E);
-    const uint32_t rows = uint32_t(decode_task_rows());
-    // weights; token rows (8 per routed chunk, 16 per shared chunk) and group offsets
-    bool ok = make_tmap_2d(&m1.r0, L.w_gate, 1, L.D / 2, E * L.F, 128, rows, true) &&
-              make_tmap_2d(&m1.r1, L.w_up, 1, L.D / 2, E * L.F, 128, rows, true) &&
-              make_tmap_2d(&m1.s0, L.ws_gate, 2, L.D, L.F_shared, 64, rows, true) &&
-              make_tmap_2d(&m1.s1, L.ws_up, 2, L.D, L.F_shared, 64, rows, true) &&
-              make_tmap_rows_3d(&m1.br, at<__half>(ws, W.x16), L.D, S, 8, 4) &&
-              make_tmap_2d(&m1.cr, at<float>(ws, W.x_negc), 4, act16_negc_pitch(L.D), S, 4, 8, false) &&
-              make_tmap_rows_3d(&m1.bs, x, L.D, T, 16, 1) &&
-              make_tmap_2d(&m2.r0, L.w_down, 1, L.F / 2, E * L.D, 128, rows, true) &&
-              make_tmap_2d(&m2.s0, L.ws_down, 2, L.F_shared, L.D, 64, rows, true) &&
-              make_tmap_rows_3d(&m2.br, at<__half>(ws, W.h16), L.F, S, 8, 8) &&
-              make_tmap_2d(&m2.cr, at<float>(ws, W.h_negc), 4, act16_negc_pitch(L.F), S, 4, 8, false) &&
-              make_tmap_rows_3d(&m2.bs, h_s, L.F_shared, T, 16, 2);
-    // the task scales: one box per matrix when their rows are whole 16-byte units
-    const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
-    if (pd) ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / kGroup, E * L.F, pd, rows, false) &&
-                 make_tmap_2d(&m1.g1, L.s_up, 4, L.D / kGroup, E * L.F, pd, rows, false);
-    else m1.g0 = m1.g1 = m1.r0;   // unused: the scales come by bulk copy
-    if (pf) ok = ok && make_tmap_2d(&m2.g0, L.s_down, 4, L.F / kGroup, E * L.D, pf, rows, false);
-    else m2.g0 = m2.r0;
-    if (!ok) return MOE_ERR_CUDA;
-    m2.r1 = m2.r0;
-    m2.s1 = m2.s0;
-    m2.g1 = m2.g0;
+    // tensor maps: built once per (layer, workspace, input, T) and thread
+    static thread_local MapCacheKey dkey;
+    static thread_local DecodeMaps dm1, dm2;
+    const MapCacheKey key = make_key(L, ws, x, T, PATH_SEL_DECODE);
+    if (!same_key(key, dkey)) {
+        dkey.valid = false;
+        auto build = [&](DecodeMaps& m1, DecodeMaps& m2) -> bool {
+        const uint64_t E = uint64_t(L.E);
+        const uint32_t rows = uint32_t(decode_task_rows());
+        // weights; token rows (8 per routed chunk, 16 per shared chunk) and group offsets
+        bool ok = make_tmap_2d(&m1.r0, L.w_gate, 1, L.D / 2, E * L.F, 128, rows, true) &&
+                  make_tmap_2d(&m1.r1, L.w_up, 1, L.D / 2, E * L.F, 128, rows, true) &&
+                  make_tmap_2d(&m1.s0, L.ws_gate, 2, L.D, L.F_shared, 64, rows, true) &&
+                  make_tmap_2d(&m1.s1, L.ws_up, 2, L.D, L.F_shared, 64, rows, true) &&
+                  make_tmap_rows_3d(&m1.br, at<__half>(ws, W.x16), L.D, S, 8, 4) &&
+                  make_tmap_2d(&m1.cr, at<float>(ws, W.x_negc), 4, act16_negc_pitch(L.D), S, 4, 8, false) &&
+                  make_tmap_rows_3d(&m1.bs, x, L.D, T, 16, 1) &&
+                  make_tmap_2d(&m2.r0, L.w_down, 1, L.F / 2, E * L.D, 128, rows, true) &&
+                  make_tmap_2d(&m2.s0, L.ws_down, 2, L.F_shared, L.D, 64, rows, true) &&
+                  make_tmap_rows_3d(&m2.br, at<__half>(ws, W.h16), L.F, S, 8, 8) &&
+                  make_tmap_2d(&m2.cr, at<float>(ws, W.h_negc), 4, act16_negc_pitch(L.F), S, 4, 8, false) &&
+                  make_tmap_rows_3d(&m2.bs, h_s, L.F_shared, T, 16, 2);
+        // the task scales: one box per matrix when their rows are whole 16-byte units
+        const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
+        if (pd) ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / kGroup, E * L.F, pd, rows, false) &&
+                     make_tmap_2d(&m1.g1, L.s_up, 4, L.D / kGroup, E * L.F, pd, rows, false);
+        else m1.g0 = m1.g1 = m1.r0;   // unused: the scales come by bulk copy
+        if (pf) ok = ok && make_tmap_2d(&m2.g0, L.s_down, 4, L.F / kGroup, E * L.D, pf, rows, false);
+        else m2.g0 = m2.r0;
+        if (!ok) return false;
+        m2.r1 = m2.r0;
+        m2.s1 = m2.s0;
+        m2.g1 = m2.g0;
+            return true;
+        };
+        if (!build(dm1, dm2)) return MOE_ERR_CUDA;
+        dkey = key;
+    }
+    const DecodeMaps& m1 = dm1;
+    const DecodeMaps& m2 = dm2;
 
     DecodeParams p;
     memset(&p, 0, sizeof(p));
@@ -327,6 +372,10 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
 
     RoutePrep prep;
     memset(&prep, 0, sizeof(prep));
+    if (W.rt_cnt != W.zeros_end) {   // K-split router (few token tiles)
+        prep.router_part = at<float>(ws, W.rt_part);
+        prep.router_tile_cnt = at<int32_t>(ws, W.rt_cnt);
+    }
     memset(&prep, 0, sizeof(prep));
     prep.chunks = chunks;
     prep.n_chunks = nch;
@@ -351,29 +400,43 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     if (cudaMemcpyAsync(x_pad, x, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return MOE_ERR_CUDA;
 
-    const uint64_t E = uint64_t(L.E);
-    TcMaps m_gu, m_dn, m_sgu, m_sdn;
-    bool ok;
-    if (fp8)
-        ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), 1, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D, E * L.F, 128, 16, true) &&
-             make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D, E * L.F, 128, 16, true) &&
-             make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), 1, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F, E * L.D, 128, 16, true);
-    else
-        ok = make_tmap_2d(&m_gu.b, x_sorted, 2, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D / 2, E * L.F, 32, 64, false) &&
-             make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D / 2, E * L.F, 32, 64, false) &&
-             make_tmap_2d(&m_dn.b, h_sorted, 2, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
-             make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
-    ok = ok && make_tmap_2d(&m_sgu.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
-              make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
-              make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
-              make_tmap_2d(&m_sdn.a0, L.ws_down, 2, L.F_shared, L.D, 64, 16, true);
-    if (!ok) return MOE_ERR_CUDA;
-    m_dn.a1 = m_dn.a0;
-    m_sdn.a1 = m_sdn.a0;
+    static thread_local MapCacheKey pkey;
+    static thread_local TcMaps pm[4];
+    const MapCacheKey key = make_key(L, ws, x, T, PATH_SEL_PREFILL);
+    if (!same_key(key, pkey)) {
+        pkey.valid = false;
+        auto build = [&](TcMaps& m_gu, TcMaps& m_dn, TcMaps& m_sgu, TcMaps& m_sdn) -> bool {
+        const uint64_t E = uint64_t(L.E);
+        bool ok;
+        if (fp8)
+            ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), 1, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D, E * L.F, 128, 16, true) &&
+                 make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D, E * L.F, 128, 16, true) &&
+                 make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), 1, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F, E * L.D, 128, 16, true);
+        else
+            ok = make_tmap_2d(&m_gu.b, x_sorted, 2, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D / 2, E * L.F, 32, 64, false) &&
+                 make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D / 2, E * L.F, 32, 64, false) &&
+                 make_tmap_2d(&m_dn.b, h_sorted, 2, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
+        ok = ok && make_tmap_2d(&m_sgu.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                  make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
+                  make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
+                  make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                  make_tmap_2d(&m_sdn.a0, L.ws_down, 2, L.F_shared, L.D, 64, 16, true);
+        if (!ok) return false;
+        m_dn.a1 = m_dn.a0;
+        m_sdn.a1 = m_sdn.a0;
+            return true;
+        };
+        if (!build(pm[0], pm[1], pm[2], pm[3])) return MOE_ERR_CUDA;
+        pkey = key;
+    }
+    TcMaps& m_gu = pm[0];
+    TcMaps& m_dn = pm[1];
+    TcMaps& m_sgu = pm[2];
+    TcMaps& m_sdn = pm[3];
 
     TcParams p;
     memset(&p, 0, sizeof(p));

@@ -38,18 +38,27 @@ inline int router_warps(int D, int E) {
     return 1;
 }
 
+// grid (token tiles, ksplit): CTA (i, j) takes tokens 16 i .. 16 i + 15 and
+// the j-th of ksplit equal K ranges.  With ksplit > 1 each CTA stores its
+// partial logits (summed over its warps) to part_g and the last CTA of a
+// tile to arrive (counted in tile_cnt, zeroed beforehand) sums them in
+// K-range order -- the same order whichever CTA is last -- and takes the
+// top-k.  No CTA waits for another.
 __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     const bf16* __restrict__ x, int T, int D, const bf16* __restrict__ wr,
     const float* __restrict__ bias, int E, int k, int32_t* __restrict__ ids,
-    float* __restrict__ gates, bf16* __restrict__ x_frag) {
+    float* __restrict__ gates, bf16* __restrict__ x_frag, int ksplit, float* __restrict__ part_g,
+    int32_t* __restrict__ tile_cnt) {
     extern __shared__ __align__(16) float part[];     // [nw][RT_TOK][E]
+    __shared__ int s_last;
     griddep_launch_dependents();
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int t0 = blockIdx.x * RT_TOK;
-    const int groups_per_warp = (D / kGroup) / nw;
-    const int k_begin = warp * groups_per_warp * kGroup;
+    const int groups_per_cta = (D / kGroup) / ksplit;
+    const int groups_per_warp = groups_per_cta / nw;
+    const int k_begin = (blockIdx.y * groups_per_cta + warp * groups_per_warp) * kGroup;
     const int k_end = k_begin + groups_per_warp * kGroup;
     const bool row_a = t0 + g < T, row_b = t0 + g + 8 < T;
     const bf16* xa_row = x + int64_t(t0 + g) * D;
@@ -118,6 +127,37 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     }
     __syncthreads();
 
+    if (ksplit > 1) {
+        // this K range's logits to global memory; the tile's last CTA goes on
+        float* mine = part_g + (int64_t(blockIdx.x) * ksplit + blockIdx.y) * RT_TOK * E;
+        for (int i = threadIdx.x; i < RT_TOK * E; i += blockDim.x) {
+            float a = 0.0f;
+            for (int w = 0; w < nw; ++w) a += part[w * RT_TOK * E + i];
+            mine[i] = a;
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) s_last = atomicAdd(&tile_cnt[blockIdx.x], 1) == ksplit - 1;
+        __syncthreads();
+        if (!s_last) {
+            griddep_wait();
+            return;
+        }
+        __threadfence();
+    }
+    // logit of token row r, expert e: the sum over warps (one CTA) or over
+    // the K ranges in order (split)
+    auto logit = [&](int r, int e) {
+        float a = 0.0f;
+        if (ksplit > 1) {
+            const float* base = part_g + int64_t(blockIdx.x) * ksplit * RT_TOK * E + r * E + e;
+            for (int j = 0; j < ksplit; ++j) a += __ldcg(base + int64_t(j) * RT_TOK * E);
+        } else {
+            for (int w = 0; w < nw; ++w) a += part[(w * RT_TOK + r) * E + e];
+        }
+        return a;
+    };
+
     // top-k per token; lane holds experts lane + 32 i
     for (int r = warp; r < RT_TOK; r += nw) {
         const int t = t0 + r;
@@ -128,8 +168,7 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
             const int e = lane + 32 * i;
             float s = -INFINITY;
             if (e < E) {
-                s = 0.0f;
-                for (int w = 0; w < nw; ++w) s += part[(w * RT_TOK + r) * E + e];
+                s = logit(r, e);
                 if (bias) s += bias[e];
             }
             v[i] = s;
@@ -265,22 +304,41 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
 
 size_t router_smem_bytes(int D, int E) { return size_t(router_warps(D, E)) * RT_TOK * E * sizeof(float); }
 
+// K ranges per token tile: with few tiles (a decode batch) the router would
+// run on a handful of SMs, so K is split over up to 32 CTAs per tile, each
+// with at least two groups of 128.
+int router_ksplit(int T, int D) {
+    const int tiles = int(ceil_div(T, RT_TOK)), groups = D / kGroup;
+    if (tiles >= 37) return 1;
+    for (int ks = 32; ks > 1; --ks)
+        if (groups % ks == 0 && groups / ks >= 2) return ks;
+    return 1;
+}
+
+size_t router_partial_floats(int T, int D, int E) {
+    const int ks = router_ksplit(T, D);
+    return ks > 1 ? size_t(ks) * ceil_div(T, RT_TOK) * RT_TOK * E : 0;
+}
+
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between) {
-    const int nw = router_warps(D, E);
-    const size_t smem = router_smem_bytes(D, E);
-    if (cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(RT_SMEM_MAX)) !=
-        cudaSuccess)
-        return MOE_ERR_CUDA;
+    // K split only with scratch for the partial logits (the layer's workspace)
+    const int ks = (prep && prep->router_part) ? router_ksplit(T, D) : 1;
+    const int nw = router_warps(D / ks, E);
+    const size_t smem = router_smem_bytes(D / ks, E);
+    if (allow_max_smem(router_kernel) != MOE_OK) return MOE_ERR_CUDA;
     moe_status st;
     bf16* x_frag = prep ? prep->x_frag : nullptr;
+    float* part_g = ks > 1 ? prep->router_part : nullptr;
+    int32_t* tile_cnt = ks > 1 ? prep->router_tile_cnt : nullptr;
+    const dim3 grid(unsigned(ceil_div(T, RT_TOK)), unsigned(ks));
     if (prep && prep->router_after_kernel)   // may overlap the kernel before it (it reads only x and W_r)
-        st = launch_pdl(router_kernel, dim3(unsigned(ceil_div(T, RT_TOK))), dim3(nw * 32), smem, stream, x, T, D,
-                        wr, bias, E, k, ids, gates, x_frag);
+        st = launch_pdl(router_kernel, grid, dim3(nw * 32), smem, stream, x, T, D, wr, bias, E, k, ids, gates, x_frag,
+                        ks, part_g, tile_cnt);
     else {
-        router_kernel<<<unsigned(ceil_div(T, RT_TOK)), nw * 32, smem, stream>>>(x, T, D, wr, bias, E, k, ids,
-                                                                               gates, x_frag);
+        router_kernel<<<grid, nw * 32, smem, stream>>>(x, T, D, wr, bias, E, k, ids, gates, x_frag, ks, part_g,
+                                                       tile_cnt);
         st = launch_status();
     }
     if (st != MOE_OK) return st;

@@ -471,9 +471,7 @@ moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cud
     const size_t smem = tc_smem_bytes();
 #define TC_LAUNCH(M)                                                                                     \
     do {                                                                                                 \
-        if (cudaFuncSetAttribute(tc_gemm_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
-                                 int(smem)) != cudaSuccess)                                              \
-            return MOE_ERR_CUDA;                                                                         \
+        if (allow_max_smem(tc_gemm_kernel<M>) != MOE_OK) return MOE_ERR_CUDA;                         \
         tc_gemm_kernel<M><<<sms, TC_THREADS, smem, stream>>>(maps.b, maps.a0, maps.a1, prm);           \
     } while (0)
     switch (mode) {
