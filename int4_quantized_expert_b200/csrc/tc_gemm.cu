@@ -32,7 +32,12 @@
 
 namespace moe {
 
-constexpr int TC_THREADS = 384;
+// Four warpgroups: 0 -- TMA producer (warp 0), MMA issuer (warp 1); 1 --
+// epilogue; 2 and 3 -- int4 converters (idle in the bf16 / e4m3 modes).
+// Registers: 128 x 64 + 128 x 192 + 256 x 96 <= 512 x 128 (setmaxnreg).
+constexpr int TC_THREADS = 512;
+constexpr int TC_CTRL_REGS = 64, TC_EPI_REGS = 192, TC_CONV_REGS = 96;
+static_assert(128 * TC_CTRL_REGS + 128 * TC_EPI_REGS + 256 * TC_CONV_REGS <= TC_THREADS * 128, "register split");
 constexpr int TC_STAGES = 4;
 constexpr int TC_B_BYTES = TC_BLOCK_TOKENS * 64 * 2;   // 32 KB
 constexpr int TC_A_BYTES = 128 * 64 * 2;               // 16 KB
@@ -90,7 +95,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     if (threadIdx.x == 0) {
         for (int i = 0; i < TC_STAGES; ++i) {
             mbar_init(&sm->full[i], 1);
-            mbar_init(&sm->a_ready[i], 4);
+            mbar_init(&sm->a_ready[i], 8);   // the 8 converter warps
             mbar_init(&sm->empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) { mbar_init(&sm->acc_full[i], 1); mbar_init(&sm->acc_empty[i], 4); }
@@ -105,11 +110,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
+
     const int n_all = p.n_chunks[0], n_sh = p.n_chunks[1];
     const int c_begin = p.routed ? n_sh : 0, c_end = p.routed ? n_all : n_sh;
     const int n_tiles = (c_end - c_begin) * p.n_fblocks;
     const int nk = p.K / KSTEP;
 
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(TC_CTRL_REGS));
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
@@ -199,7 +207,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             // wind down: wait (bounded) for the last MMAs
             if (it > 0) mbar_wait(&sm->empty[(it - 1) % TC_STAGES], ((it - 1) / TC_STAGES) & 1, nullptr);
         }
-    } else if (warp >= 4 && warp < 8) {
+    }
+    } else if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(TC_EPI_REGS));
         // ------------------------------ epilogue ------------------------------
         const int ew = warp & 3;                 // TMEM lanes 32 ew .. 32 ew + 31
         uint32_t n = 0;
@@ -293,9 +303,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm->acc_empty[acc]);
         }
-    } else if (INT4 && warp >= 8) {
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(TC_CONV_REGS));
+    if (INT4) {
         // ------------------------------ int4 -> bf16 converters ------------------------------
-        const int i = threadIdx.x - 256;                     // A row 0..127
+        // thread: A row i, half hh of the stage's 64 K (4 of its 8 code words)
+        const int i = (threadIdx.x - 256) & 127, hh = (threadIdx.x - 256) >> 7;
         int code_row, srow_off;
         const float* sbase;
         if (MODE == TC_GATEUP_INT4) {
@@ -330,16 +343,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 unsigned char* st = base + slot * TC_STAGE_BYTES;
                 unsigned char* sa = st + TC_B_BYTES;
                 const unsigned char* sc = sa + TC_A_BYTES;
-                const uint4 c0 = *reinterpret_cast<const uint4*>(sc + code_row * 32);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(sc + code_row * 32 + 16);
-                const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const uint4 c0 = *reinterpret_cast<const uint4*>(sc + code_row * 32 + hh * 16);
+                const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = 4 * hh + jj;   // 16-byte chunk of the A row (8 K values)
                     // 8 codes k0..k7 -> (k0,k4) (k1,k5) (k2,k6) (k3,k7), each (q * s) in bf16
                     uint32_t o[4];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        uint32_t t = ((w[j] >> (4 * h)) & 0x000F000Fu) ^ 0x43084308u;   // bf16 136 + q
+                        uint32_t t = ((w[jj] >> (4 * h)) & 0x000F000Fu) ^ 0x43084308u;   // bf16 136 + q
                         __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&t), k136);
                         __nv_bfloat162 r = __hmul2(q, s2);
                         o[h] = *reinterpret_cast<uint32_t*>(&r);
@@ -354,6 +367,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         }
     }
 
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
