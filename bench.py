@@ -61,10 +61,10 @@ def peaks():
 KERNEL_SOURCES = {   # the files a kernel's code comes from (a change invalidates its ncu numbers)
     "decode_gate_up": ["ffn_decode.cu", "ffn_decode.cuh", "common.cuh"],
     "decode_down": ["ffn_decode.cu", "ffn_decode.cuh", "common.cuh"],
-    "tc_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
-    "tc_down": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
-    "tc_shared_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
-    "tc_shared_down": ["tc_gemm.cu", "tc_gemm.cuh", "common.cuh"],
+    "tc_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "tcgen05.cuh", "common.cuh"],
+    "tc_down": ["tc_gemm.cu", "tc_gemm.cuh", "tcgen05.cuh", "common.cuh"],
+    "tc_shared_gate_up": ["tc_gemm.cu", "tc_gemm.cuh", "tcgen05.cuh", "common.cuh"],
+    "tc_shared_down": ["tc_gemm.cu", "tc_gemm.cuh", "tcgen05.cuh", "common.cuh"],
 }
 
 
@@ -632,7 +632,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scout_decode",
-                    choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8", "quantize"])
+                    choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8", "maverick_fp8_e16",
+                             "quantize"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

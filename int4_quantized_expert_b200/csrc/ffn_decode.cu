@@ -9,22 +9,29 @@
 //
 // With a handful of tokens per expert every weight byte is used by only a few
 // multiply-adds, so the kernels are bound by HBM bandwidth.  Design:
-//   * one persistent CTA per SM; a producer warp takes tasks (32 output rows of
-//     one matrix pair x one chunk of <= 16 tokens) from a global counter, shared
-//     expert first, and streams the task's weights with 2-D TMA loads
-//     (64 rows x 128 bytes, 128-byte swizzle) through a ring of 16 KB stages;
-//     the task's int4 scales arrive with one 1-D bulk copy.
-//   * 12 consumer warps: 4 row blocks of 16 rows x 3 K phases (stage s goes
-//     to phase s % 3), three per SM sub-partition to hide each one's MMA and
-//     load latencies.  Each converts int4 codes to exact bf16 integers in
-//     registers (no scale multiply per element), runs m16n8k16 tensor-core
-//     MMAs against the tokens (fp32 accumulate), and applies the group's scale
-//     to the 128-K partial sum.  The 3 K phases are summed through shared
-//     memory, then the epilogue applies SwiGLU (gate/up pass) or the gate
-//     (down pass).
-//   * Tokens are the MMA's N operand (8 per n-tile).  Their rows are read with
-//     L1-cached global loads in a layout where every 8 values are stored
-//     x0 x4 x1 x5 x2 x6 x3 x7, which is the order the int4 unpacking yields.
+//   * one persistent CTA per SM (512 threads); a producer thread takes tasks
+//     (64 output rows of one matrix pair x one chunk of <= 16 tokens x the
+//     whole K) from a global counter, shared expert first, and streams each
+//     task through a ring of 6 stages.  A stage holds 16 KB of weights (2-D
+//     TMA, 64 rows x 128 bytes, 128-byte swizzle), the chunk's token rows for
+//     the stage's K range (one 3-D TMA box) and, for int4, the rows' group
+//     offsets (one 2-D box).  The benchmark's fp32 scales arrive first, one padded
+//     2-D box per matrix.
+//   * 12 consumer warps: 4 row blocks of 16 rows x 3 K phases (a stage goes to
+//     phase (global stage index) % 3), three per SM sub-partition to hide each
+//     one's MMA and load latencies.  Each converts int4 codes to exact fp16
+//     integers in registers (no scale multiply per element), runs m16n8k16
+//     tensor-core MMAs against the tokens (fp32 accumulate), and applies the
+//     group's scale to the 128-K partial sum.  The 3 K phases are summed
+//     through shared memory, then the epilogue applies SwiGLU (gate/up pass)
+//     or the gate (down pass).
+//   * Tokens are the MMA's N operand (8 per n-tile), written by act16_kernel as
+//     fp16 rows in the order the int4 unpacking yields.
+//   * Every wait is bounded; a timeout sets the status word and the CTA
+//     drains its copies in flight and returns.
+//   * Launches chain by programmatic dependent launch: each kernel's setup
+//     (barriers, tensor-map prefetch, shared-expert tasks) overlaps the tail
+//     of the kernel before it.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -270,8 +277,12 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             int n_tasks = n_sh * nbs;   // grows by the routed tasks after the wait
             for (uint32_t tn = 0; ok; ++tn) {
                 const int t = atomicAdd(p.task_counter, 1);
-                if (t >= n_sh * nbs && !waited) {
-                    griddep_wait();   // the routing step's chunk list is complete
+                // Wait for the kernels before this one before the first load of
+                // anything they write: the chunk list (routed tasks) and, in the
+                // down pass, every task's input rows.  Only the gate/up pass's
+                // shared-expert tasks (rows of the layer input) start before it.
+                if (!waited && (MODE == 1 || t >= n_sh * nbs)) {
+                    griddep_wait();
                     n_tasks += (*p.n_chunks - n_sh) * nbr;
                     waited = true;
                 }
@@ -388,7 +399,6 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             waited = true;
         }
         const float* sc = sbuf + b * p.scale_buf_floats;
-        const int ng = ti.K / kGroup;
 
         // MMA column g of n-tile nt is token row nt * 8 + sigma8(g) of the chunk;
         // routed results are rescaled per token by their row's power of two

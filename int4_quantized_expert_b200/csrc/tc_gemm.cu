@@ -11,13 +11,15 @@
 //   shared memory with the 128-byte swizzle, K step 64; D = fp32 in tensor
 //   memory (TMEM), two 256-column accumulators so a tile's epilogue overlaps
 //   the next tile's MMAs.
-// Warp roles (12 warps):
+// Warp roles (16 warps):
 //   warp 0      TMA producer (one thread) and TMEM allocator
-//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 inputs
+//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16 (bf16) or
+//               kind::f8f6f4 (e4m3)
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
 //               lanes 32 (w % 4) ..), SwiGLU / gate scaling / combine, stores
-//   warps 8-11  int4 modes only: dequantize the stage's codes (w = q * s, s
-//               rounded to bf16) into the swizzled A tile, one thread per row
+//   warps 8-15  int4 modes only: dequantize the stage's codes (w = q * s, s
+//               rounded to bf16) into the swizzled A tile; two threads per
+//               row, each taking 32 of the stage's 64 K
 // Gate/up tiles hold 64 features: A rows alternate 16 gate rows and the same
 // 16 up rows, so each epilogue warp finds g (lanes 0..15) and u (lanes 16..31)
 // of its 16 features together.  Routed activations are stored with every 8
@@ -42,7 +44,12 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_B_BYTES = TC_BLOCK_TOKENS * 64 * 2;   // 32 KB
 constexpr int TC_A_BYTES = 128 * 64 * 2;               // 16 KB
 constexpr int TC_C_BYTES = 128 * 32;                   // int4 codes of the A tile: 4 KB
-constexpr int TC_STAGE_BYTES = TC_B_BYTES + TC_A_BYTES + TC_C_BYTES;
+constexpr int TC_STAGE_BYTES = TC_B_BYTES + TC_A_BYTES;
+// The int4 codes have a ring of their own, twice as deep as the stages: they
+// are loaded (by warp 2) well ahead, so the converters can fill a stage's A
+// tile as soon as its previous MMAs complete, while its token tile is still
+// in flight.
+constexpr int TC_CSTAGES = 2 * TC_STAGES;
 constexpr int TC_TMEM_COLS = 512;
 static_assert(TC_STAGE_BYTES % 1024 == 0, "stage alignment");
 
@@ -50,6 +57,8 @@ struct TcSmem {
     uint64_t full[TC_STAGES];      // TMA data of the stage landed (tx counted)
     uint64_t a_ready[TC_STAGES];   // converter warps wrote the A tile
     uint64_t empty[TC_STAGES];     // the stage's MMAs completed
+    uint64_t cfull[TC_CSTAGES];    // int4 codes of a code slot landed
+    uint64_t cempty[TC_CSTAGES];   // converter warps read the code slot
     uint64_t acc_full[2];          // accumulator holds a finished tile
     uint64_t acc_empty[2];         // epilogue finished reading the accumulator
     uint32_t tmem_base;
@@ -89,7 +98,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    TcSmem* sm = reinterpret_cast<TcSmem*>(base + TC_STAGES * TC_STAGE_BYTES);
+    unsigned char* cring = base + TC_STAGES * TC_STAGE_BYTES;   // int4 code ring
+    TcSmem* sm = reinterpret_cast<TcSmem*>(cring + TC_CSTAGES * TC_C_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -98,6 +108,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             mbar_init(&sm->a_ready[i], 8);   // the 8 converter warps
             mbar_init(&sm->empty[i], 1);
         }
+        for (int i = 0; i < TC_CSTAGES; ++i) { mbar_init(&sm->cfull[i], 1); mbar_init(&sm->cempty[i], 8); }
         for (int i = 0; i < 2; ++i) { mbar_init(&sm->acc_full[i], 1); mbar_init(&sm->acc_empty[i], 4); }
         fence_barrier_init();
     }
@@ -134,17 +145,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status, 64)) { ok = false; break; }
                     unsigned char* st = base + slot * TC_STAGE_BYTES;
                     unsigned char* sa = st + TC_B_BYTES;
-                    unsigned char* sc = sa + TC_A_BYTES;
-                    mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES + (INT4 ? TC_C_BYTES : TC_A_BYTES));
+                    mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES + (INT4 ? 0 : TC_A_BYTES));
                     tma_load_2d(st, &tm_b, &sm->full[slot], kk * KSTEP, ce.start);
-                    if (MODE == TC_GATEUP_INT4) {
-                        const int row = e * p.n_rows + fb * 64;
-                        tma_load_2d(sc, &tm_a0, &sm->full[slot], kk * 32, row);
-                        tma_load_2d(sc + 64 * 32, &tm_a1, &sm->full[slot], kk * 32, row);
-                    } else if (MODE == TC_DOWN_INT4) {
-                        const int row = e * p.n_rows + fb * 128;
-                        tma_load_2d(sc, &tm_a0, &sm->full[slot], kk * 32, row);
-                        tma_load_2d(sc + 64 * 32, &tm_a0, &sm->full[slot], kk * 32, row + 64);
+                    if (INT4) {
+                        // the codes come through the code ring (warp 2)
                     } else if (MODE == TC_GATEUP_BF16) {
                         // 16-row boxes: gate rows, up rows, gate rows, ... (same features)
 #pragma unroll
@@ -172,6 +176,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             for (uint32_t i = 0; i < TC_STAGES && i < it; ++i) {
                 const uint32_t j = it - 1 - i;
                 mbar_wait(&sm->full[j % TC_STAGES], (j / TC_STAGES) & 1, nullptr);
+            }
+        }
+    } else if (warp == 2 && INT4) {
+        // ------------------------------ int4 code producer ------------------------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                int ci, fb;
+                tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
+                const ChunkEntry ce = p.chunks[c_begin + ci];
+                const int e = ce.expert < 0 ? 0 : ce.expert;
+                const int row = e * p.n_rows + fb * (GATEUP ? 64 : 128);
+                for (int kk = 0; kk < nk; ++kk, ++it) {
+                    const uint32_t cs = it % TC_CSTAGES;
+                    if (!mbar_wait(&sm->cempty[cs], ((it / TC_CSTAGES) & 1) ^ 1, p.status, 64)) { ok = false; break; }
+                    unsigned char* sc = cring + cs * TC_C_BYTES;
+                    mbar_arrive_expect_tx(&sm->cfull[cs], TC_C_BYTES);
+                    if (GATEUP) {   // gate rows, then the same features' up rows
+                        tma_load_2d(sc, &tm_a0, &sm->cfull[cs], kk * 32, row);
+                        tma_load_2d(sc + 64 * 32, &tm_a1, &sm->cfull[cs], kk * 32, row);
+                    } else {
+                        tma_load_2d(sc, &tm_a0, &sm->cfull[cs], kk * 32, row);
+                        tma_load_2d(sc + 64 * 32, &tm_a0, &sm->cfull[cs], kk * 32, row + 64);
+                    }
+                }
+            }
+            // wind down: wait (bounded) for the code loads still in flight to land
+            for (uint32_t i = 0; i < TC_CSTAGES && i < it; ++i) {
+                const uint32_t j = it - 1 - i;
+                mbar_wait(&sm->cfull[j % TC_CSTAGES], (j / TC_CSTAGES) & 1, nullptr);
             }
         }
     } else if (warp == 1) {
@@ -307,8 +342,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(TC_CONV_REGS));
     if (INT4) {
         // ------------------------------ int4 -> bf16 converters ------------------------------
-        // thread: A row i, half hh of the stage's 64 K (4 of its 8 code words)
-        const int i = (threadIdx.x - 256) & 127, hh = (threadIdx.x - 256) >> 7;
+        // thread: A row i, half hh of the stage's 64 K (4 of its 8 code words);
+        // a warp reads 16 consecutive code rows, 512 contiguous bytes
+        const int i = (threadIdx.x - 256) >> 1, hh = threadIdx.x & 1;
         int code_row, srow_off;
         const float* sbase;
         if (MODE == TC_GATEUP_INT4) {
@@ -338,12 +374,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     const int gn = kk / 2 + 1;
                     if (gn < ng) s_next = ldg_f32(srow + gn);
                 }
-                const uint32_t slot = it % TC_STAGES;
-                if (!mbar_wait(&sm->full[slot], (it / TC_STAGES) & 1, p.status)) { ok = false; break; }
-                unsigned char* st = base + slot * TC_STAGE_BYTES;
-                unsigned char* sa = st + TC_B_BYTES;
-                const unsigned char* sc = sa + TC_A_BYTES;
+                const uint32_t slot = it % TC_STAGES, cs = it % TC_CSTAGES;
+                if (!mbar_wait(&sm->cfull[cs], (it / TC_CSTAGES) & 1, p.status)) { ok = false; break; }
+                const unsigned char* sc = cring + cs * TC_C_BYTES;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(sc + code_row * 32 + hh * 16);
+                // the A tile is free once the slot's previous MMAs completed
+                if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status)) { ok = false; break; }
+                unsigned char* sa = base + slot * TC_STAGE_BYTES + TC_B_BYTES;
                 const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
@@ -361,7 +398,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->a_ready[slot]);
+                // the code slot is released only after its codes have been used
+                // (released right after the load, it was sometimes refilled
+                // before the load had read it)
+                if (lane == 0) {
+                    mbar_arrive(&sm->a_ready[slot]);
+                    mbar_arrive(&sm->cempty[cs]);
+                }
             }
             if (!ok) break;
         }
@@ -476,7 +519,9 @@ moe_status launch_combine_slots(const float* y_s, const float* y, int64_t T, int
     return launch_status();
 }
 
-size_t tc_smem_bytes() { return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + sizeof(TcSmem); }
+size_t tc_smem_bytes() {
+    return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + size_t(TC_CSTAGES) * TC_C_BYTES + sizeof(TcSmem);
+}
 
 moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream) {
     int dev = 0, sms = 148;

@@ -62,15 +62,20 @@ class LayerShape:
                           self.F_shared, self.fmt, self.skewed)
 
 
-# The five workloads: a tiny layer, the Scout-shaped decode and prefill layers
-# (16 experts, top-1), the Maverick-shaped FP8 layer (128 experts, top-8) and
-# a Scout-shaped layer with a Zipf-like router bias.
+# The workloads: a tiny layer, the Scout-shaped decode and prefill layers
+# (16 experts, top-1), the Maverick-shaped FP8 layer (128 experts, top-8), a
+# Scout-shaped layer with a Zipf-like router bias, and a 16-expert cut of the
+# FP8 layer.
 SHAPES = {
     "tiny": LayerShape("tiny", 64, 256, 512, 4, 1, 512, "int4"),
     "scout_decode": LayerShape("scout_decode", 16, 5120, 8192, 16, 1, 8192, "int4"),
     "scout_prefill": LayerShape("scout_prefill", 8192, 5120, 8192, 16, 1, 8192, "int4"),
     "maverick_fp8": LayerShape("maverick_fp8", 4096, 5120, 8192, 128, 8, 8192, "fp8"),
     "skewed": LayerShape("skewed", 32768, 5120, 8192, 16, 1, 8192, "int4", skewed=True),
+    # the Maverick-shaped FP8 layer cut to 16 experts and 512 tokens (the same
+    # 256 slots per expert on average, 2.3 GB of weights): a case small enough
+    # for profiling captures of the FP8 kernels
+    "maverick_fp8_e16": LayerShape("maverick_fp8_e16", 512, 5120, 8192, 16, 8, 8192, "fp8"),
 }
 
 # Stream ids.  Routed expert e uses ids 16 + 3e + {0: gate, 1: up, 2: down}.
