@@ -208,9 +208,20 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
         quant = lambda w, out: moe.quantize_fp8_rows(w, out=out)
         fmt = moe.FMT_FP8
     gate, up, down = alloc(F, D), alloc(F, D), alloc(D, F)
-    for e, g, u, d in synth.iter_expert_weights(seed, range(E), D, F, workers=min(16, os.cpu_count() or 1)):
-        for w, (c, s) in ((g, gate), (u, up), (d, down)):
-            quant(torch.from_numpy(w).to(dev), (c[e], s[e]))
+    # Routed experts: N(0, 0.02) fp32 drawn on the device by torch's seeded
+    # Philox generator (the same distribution as the parity tests' PCG64
+    # draws, without minutes of host work for 128 experts), then quantized by
+    # the library.  Routing depends only on x and the router, drawn as in the
+    # tests.
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    wbuf = torch.empty(max(F * D, D * F), dtype=torch.float32, device=dev)
+    for e in range(E):
+        for (n, kk), (c, s) in (((F, D), gate), ((F, D), up), ((D, F), down)):
+            w = wbuf[:n * kk].view(n, kk)
+            torch.randn(n, kk, generator=gen, out=w).mul_(synth.WEIGHT_STD)
+            quant(w, (c[e], s[e]))
+    del wbuf
     torch.cuda.synchronize()
     layer = moe.MoELayer(E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr, router_bias=bias, gate=gate,
                          up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T)
@@ -380,7 +391,8 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16" if shape.fmt == "int4" else "e4m3 (routed experts), bf16 (shared expert)",
-        "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
+        "data": ("synthetic (seeded; no dataset, random-init weights of the stated shapes: x, router and "
+                 "shared expert from PCG64, routed experts N(0, 0.02) from torch's device generator)"),
         "config": {
             "workload": workload_text(shape),
             "weights": weights_text(shape),

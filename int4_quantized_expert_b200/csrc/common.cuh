@@ -228,22 +228,33 @@ __device__ __forceinline__ int32_t ld_volatile(const int32_t* p) {
     return *reinterpret_cast<const volatile int32_t*>(p);
 }
 
-// Bounded wait for the phase with the given parity to complete.  Gives up
-// at once if another wait of this launch already timed out (status set).
-// With backoff_ns > 0 the thread sleeps between polls, leaving the issue
-// slots of its SM sub-partition to the warps doing the arithmetic.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
-                                          uint32_t backoff_ns = 0) {
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes (or about hint_ns pass), so a waiter wakes as
+// soon as its data lands and issues nothing meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete.  The
+// device status word (another wait of this launch timed out) and the clock
+// are checked only every 64 sleeps, so a wait that misses its first try
+// costs no global-memory round trip.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (status && ld_volatile(status) != DEV_OK) return false;
     const long long t0 = clock64();
     for (uint32_t i = 1;; ++i) {
-        if (backoff_ns) __nanosleep(backoff_ns);
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 0 && status && ld_volatile(status) != DEV_OK) return false;
-        if (clock64() - t0 > kWaitCycles) {
-            if (status) atomicExch(status, DEV_TIMEOUT);
-            return false;
+        if (mbar_try_wait_sleep(bar, parity, 10000u)) return true;
+        if ((i & 63u) == 0) {
+            if (status && ld_volatile(status) != DEV_OK) return false;
+            if (clock64() - t0 > kWaitCycles) {
+                if (status) atomicExch(status, DEV_TIMEOUT);
+                return false;
+            }
         }
     }
 }

@@ -132,7 +132,8 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 template <int MODE>
 __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
                                              const float* sc, uint32_t it_base, int q, int lane, int row_a,
-                                             int row_b, float (&acc0)[4], float (&acc1)[4], int32_t* status) {
+                                             int row_b, float (&acc0)[4], float (&acc1)[4],
+                                             int32_t* status) {
     constexpr int GPS = MODE == 0 ? 2 : 4;   // groups per stage
     constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
     const int g = lane >> 2, c = lane & 3;
@@ -159,6 +160,64 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
     for (int i = 0; i < 4; ++i) offx[i] = (i >> 1) * 1024 + trow * 128 + (((c + 4 * (i & 1)) ^ (trow & 7)) << 4);
     const int tc0 = sigma8(2 * c), tc1 = sigma8(2 * c + 1);   // token rows of C columns 2c, 2c + 1
 
+    // One group of 128 K (group G of the task, gl of the stage).  gl is a
+    // compile-time constant at every call, so the register arrays above are
+    // indexed statically.
+    auto group = [&](const unsigned char* st, const unsigned char* bt, const float* ct, int cg0, int G, int gl) {
+        // MODE 0: both groups in tile 0 (gate) and tile 1 (up);
+        // MODE 1: groups 0,1 in tile 0 and 2,3 in tile 1 of the one matrix
+        const unsigned char* tile = st + (MODE == 0 ? 0 : (gl >> 1) * DC_CHUNK);
+        const int gi = gl & 1;
+        uint4 xc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xc[i] = lds128(bt + gl * 2048 + offx[i]);
+        const float cc0 = ct[tc0 * 4 + cg0 + gl], cc1 = ct[tc1 * 4 + cg0 + gl];
+        const uint4 wa = lds128(tile + off_a[gi]);
+        const uint4 wb = lds128(tile + off_b[gi]);
+        uint4 va = make_uint4(0, 0, 0, 0), vb = va;
+        if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
+        const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
+        const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
+        // four independent accumulation chains per matrix (word jj feeds
+        // chain jj; chain 0 starts from the group offset, the others from
+        // zero); every word's even-nibble MMAs go before any odd-nibble one
+        float pg[4][4], pu[4][4];
+        uint32_t wa8[4], wb8[4], va8[4], vb8[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            wa8[jj] = WA[jj] >> 8;
+            wb8[jj] = WB[jj] >> 8;
+            if (MODE == 0) { va8[jj] = VA[jj] >> 8; vb8[jj] = VB[jj] >> 8; }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const float c0 = jj == 0 ? cc0 : 0.0f, c1 = jj == 0 ? cc1 : 0.0f;
+            mma_f16_16816(pg[jj], f16_lo_nibbles(WA[jj]), f16_lo_nibbles(WB[jj]), f16_lo_nibbles(wa8[jj]),
+                          f16_lo_nibbles(wb8[jj]), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
+            if (MODE == 0)
+                mma_f16_16816(pu[jj], f16_lo_nibbles(VA[jj]), f16_lo_nibbles(VB[jj]), f16_lo_nibbles(va8[jj]),
+                              f16_lo_nibbles(vb8[jj]), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            mma_f16_16816(pg[jj], f16_hi_nibbles(WA[jj]), f16_hi_nibbles(WB[jj]), f16_hi_nibbles(wa8[jj]),
+                          f16_hi_nibbles(wb8[jj]), xc[jj].z, xc[jj].w);
+            if (MODE == 0)
+                mma_f16_16816(pu[jj], f16_hi_nibbles(VA[jj]), f16_hi_nibbles(VB[jj]), f16_hi_nibbles(va8[jj]),
+                              f16_hi_nibbles(vb8[jj]), xc[jj].z, xc[jj].w);
+        }
+        const float sga = sga_p[G], sgb = sgb_p[G];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            acc0[r] = fmaf((pg[0][r] + pg[1][r]) + (pg[2][r] + pg[3][r]), r < 2 ? sga : sgb, acc0[r]);
+        if (MODE == 0) {
+            const float sua = sua_p[G], sub = sub_p[G];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                acc1[r] = fmaf((pu[0][r] + pu[1][r]) + (pu[2][r] + pu[3][r]), r < 2 ? sua : sub, acc1[r]);
+        }
+    };
+
     bool ok = true;
     for (int s = first_stage(q, it_base); s < ti.n_stages; s += DC_KPH) {
         const uint32_t it = it_base + s;
@@ -169,61 +228,15 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
         const float* ct = reinterpret_cast<const float*>(st + C_OFF);
         const int G0 = s * GPS;
         const int cg0 = G0 & 3;   // the offsets tile starts at group G0 rounded down to a multiple of 4
+        if (G0 + GPS <= ng) {
+            // a full stage: straight-line code, so the groups' loads and
+            // unpacking interleave
 #pragma unroll
-        for (int gl = 0; gl < GPS; ++gl) {
-            const int G = G0 + gl;
-            if (G >= ng) break;
-            // MODE 0: both groups in tile 0 (gate) and tile 1 (up);
-            // MODE 1: groups 0,1 in tile 0 and 2,3 in tile 1 of the one matrix
-            const unsigned char* tile = st + (MODE == 0 ? 0 : (gl >> 1) * DC_CHUNK);
-            const int gi = gl & 1;
-            uint4 xc[4];
+            for (int gl = 0; gl < GPS; ++gl) group(st, bt, ct, cg0, G0 + gl, gl);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xc[i] = lds128(bt + gl * 2048 + offx[i]);
-            const float cc0 = ct[tc0 * 4 + cg0 + gl], cc1 = ct[tc1 * 4 + cg0 + gl];
-            const uint4 wa = lds128(tile + off_a[gi]);
-            const uint4 wb = lds128(tile + off_b[gi]);
-            uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-            if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
-            const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
-            const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
-            // four independent accumulation chains per matrix (word jj feeds
-            // chain jj; chain 0 starts from the group offset, the others from
-            // zero); every word's even-nibble MMAs go before any odd-nibble one
-            float pg[4][4], pu[4][4];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
-                const float c0 = jj == 0 ? cc0 : 0.0f, c1 = jj == 0 ? cc1 : 0.0f;
-                mma_f16_16816(pg[jj], f16_lo_nibbles(WA[jj]), f16_lo_nibbles(WB[jj]), f16_lo_nibbles(wa8),
-                              f16_lo_nibbles(wb8), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
-                if (MODE == 0) {
-                    const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
-                    mma_f16_16816(pu[jj], f16_lo_nibbles(VA[jj]), f16_lo_nibbles(VB[jj]), f16_lo_nibbles(va8),
-                                  f16_lo_nibbles(vb8), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
-                mma_f16_16816(pg[jj], f16_hi_nibbles(WA[jj]), f16_hi_nibbles(WB[jj]), f16_hi_nibbles(wa8),
-                              f16_hi_nibbles(wb8), xc[jj].z, xc[jj].w);
-                if (MODE == 0) {
-                    const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
-                    mma_f16_16816(pu[jj], f16_hi_nibbles(VA[jj]), f16_hi_nibbles(VB[jj]), f16_hi_nibbles(va8),
-                                  f16_hi_nibbles(vb8), xc[jj].z, xc[jj].w);
-                }
-            }
-            const float sga = sga_p[G], sgb = sgb_p[G];
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-                acc0[r] = fmaf((pg[0][r] + pg[1][r]) + (pg[2][r] + pg[3][r]), r < 2 ? sga : sgb, acc0[r]);
-            if (MODE == 0) {
-                const float sua = sua_p[G], sub = sub_p[G];
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    acc1[r] = fmaf((pu[0][r] + pu[1][r]) + (pu[2][r] + pu[3][r]), r < 2 ? sua : sub, acc1[r]);
-            }
+            for (int gl = 0; gl < GPS; ++gl)
+                if (G0 + gl < ng) group(st, bt, ct, cg0, G0 + gl, gl);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->empty[slot]);
@@ -287,7 +300,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     waited = true;
                 }
                 const int b = tn & 1;
-                if (!mbar_wait(&sm->sempty[b], ((tn >> 1) & 1) ^ 1, p.status, 128)) break;
+                if (!mbar_wait(&sm->sempty[b], ((tn >> 1) & 1) ^ 1, p.status)) break;
                 TaskInfo ti;
                 ti.pad = 0;
                 if (t >= n_tasks) {
@@ -349,7 +362,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const CUtensorMap* mb = ti.kind ? &tm_br : &tm_bs;
                 for (int s = 0; s < ti.n_stages; ++s, ++it) {
                     const uint32_t slot = it % NST;
-                    if (!mbar_wait(&sm->empty[slot], ((it / NST) & 1) ^ 1, p.status, 128)) { ok = false; break; }
+                    if (!mbar_wait(&sm->empty[slot], ((it / NST) & 1) ^ 1, p.status)) { ok = false; break; }
                     unsigned char* st = ring + slot * SLOT;
                     if (MODE == 0) {
                         mbar_arrive_expect_tx(&sm->full[slot], DC_STAGE + b_bytes);

@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 const int e = ce.expert < 0 ? 0 : ce.expert;
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const uint32_t slot = it % TC_STAGES;
-                    if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status, 64)) { ok = false; break; }
+                    if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status)) { ok = false; break; }
                     unsigned char* st = base + slot * TC_STAGE_BYTES;
                     unsigned char* sa = st + TC_B_BYTES;
                     mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES + (INT4 ? 0 : TC_A_BYTES));
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 const int row = e * p.n_rows + fb * (GATEUP ? 64 : 128);
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const uint32_t cs = it % TC_CSTAGES;
-                    if (!mbar_wait(&sm->cempty[cs], ((it / TC_CSTAGES) & 1) ^ 1, p.status, 64)) { ok = false; break; }
+                    if (!mbar_wait(&sm->cempty[cs], ((it / TC_CSTAGES) & 1) ^ 1, p.status)) { ok = false; break; }
                     unsigned char* sc = cring + cs * TC_C_BYTES;
                     mbar_arrive_expect_tx(&sm->cfull[cs], TC_C_BYTES);
                     if (GATEUP) {   // gate rows, then the same features' up rows
