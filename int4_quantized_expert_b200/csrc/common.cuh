@@ -171,9 +171,31 @@ __device__ __forceinline__ void mma_f16_16816(float d[4], uint32_t a0, uint32_t 
 // int4 codes -> exact fp16 integers, two per instruction.  0x6400 is 1024.0
 // in fp16, whose mantissa step is 1; a nibble placed in mantissa bits 0..3
 // with its top bit flipped (two's-complement q -> q + 8) reads 1032 + q, and
-// one in bits 4..7 reads 1024 + 16 (q + 8) = 1152 + 16 q.
-__device__ __forceinline__ uint32_t f16_lo_nibbles(uint32_t w) { return (w & 0x000F000Fu) ^ 0x64086408u; }
-__device__ __forceinline__ uint32_t f16_hi_nibbles(uint32_t w) { return (w & 0x00F000F0u) ^ 0x64806480u; }
+// one in bits 4..7 reads 1024 + 16 (q + 8) = 1152 + 16 q.  Each is one LOP3
+// (w & mask) ^ magic with the mask as the immediate and the magic in a
+// register: kF16MagicLo / kF16MagicHi, which the caller passes in as a run-
+// time value.  Written with both as compile-time constants the expression
+// takes two ALU instructions, since one LOP3 holds one immediate.
+// The same for bf16 (mantissa step 1 at 128.0 = 0x4300): nibbles in bits
+// 0..3 of each half read 136 + q.
+constexpr uint32_t kBf16Magic = 0x43084308u;
+__device__ __forceinline__ uint32_t bf16_lo_nibbles(uint32_t w, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(w), "n"(0x000F000F), "r"(magic));
+    return d;
+}
+constexpr uint32_t kF16MagicLo = 0x64086408u;
+constexpr uint32_t kF16MagicHi = 0x64806480u;
+__device__ __forceinline__ uint32_t f16_lo_nibbles(uint32_t w, uint32_t magic_lo) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(w), "n"(0x000F000F), "r"(magic_lo));   // (a & b) ^ c
+    return d;
+}
+__device__ __forceinline__ uint32_t f16_hi_nibbles(uint32_t w, uint32_t magic_hi) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(w), "n"(0x00F000F0), "r"(magic_hi));
+    return d;
+}
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 

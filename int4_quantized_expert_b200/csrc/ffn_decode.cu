@@ -123,17 +123,18 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 //
 // Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
 // shift and four LOP3s give (k0,k4) and (k2,k6) as 1032 + q and (k1,k5),
-// (k3,k7) as 1152 + 16 q.  The token rows (fp16, scaled per row by a power
-// of two) store odd positions divided by 16 and every 8-block in the order
-// x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x plus a per-group
-// offset that the partial sum starts from (negc, passed as the MMA's C).
-// The stage holds the chunk's 8 token rows for its K range and their group
+// (k3,k7) as 1152 + 16 q (f16_lo_nibbles / f16_hi_nibbles, the magic numbers
+// held in registers klo, khi).  The token rows (fp16, scaled per row by a
+// power of two) store odd positions divided by 16 and every 8-block in the
+// order x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x plus a
+// per-group offset (negc) that is added to the group's partial sum.  The
+// stage holds the chunk's 8 token rows for its K range and their group
 // offsets next to the codes; MMA column g is token row sigma8(g).
 template <int MODE>
 __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
                                              const float* sc, uint32_t it_base, int q, int lane, int row_a,
-                                             int row_b, float (&acc0)[4], float (&acc1)[4],
-                                             int32_t* status) {
+                                             int row_b, uint32_t klo, uint32_t khi, float (&acc0)[4],
+                                             float (&acc1)[4], int32_t* status) {
     constexpr int GPS = MODE == 0 ? 2 : 4;   // groups per stage
     constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
     const int g = lane >> 2, c = lane & 3;
@@ -178,43 +179,45 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
         if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
         const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
         const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
-        // four independent accumulation chains per matrix (word jj feeds
-        // chain jj; chain 0 starts from the group offset, the others from
-        // zero); every word's even-nibble MMAs go before any odd-nibble one
-        float pg[4][4], pu[4][4];
-        uint32_t wa8[4], wb8[4], va8[4], vb8[4];
+        // one accumulation chain per matrix over the group's 8 MMAs, started
+        // at zero; the group offset is added to its sum in fp32
+        float pg[4], pu[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            wa8[jj] = WA[jj] >> 8;
-            wb8[jj] = WB[jj] >> 8;
-            if (MODE == 0) { va8[jj] = VA[jj] >> 8; vb8[jj] = VB[jj] >> 8; }
+            const uint32_t wa8 = WA[jj] >> 8, wb8 = WB[jj] >> 8;
+            if (jj == 0)
+                mma_f16_16816(pg, f16_lo_nibbles(WA[jj], klo), f16_lo_nibbles(WB[jj], klo),
+                              f16_lo_nibbles(wa8, klo), f16_lo_nibbles(wb8, klo), xc[jj].x, xc[jj].y,
+                              0.0f, 0.0f, 0.0f, 0.0f);
+            else
+                mma_f16_16816(pg, f16_lo_nibbles(WA[jj], klo), f16_lo_nibbles(WB[jj], klo),
+                              f16_lo_nibbles(wa8, klo), f16_lo_nibbles(wb8, klo), xc[jj].x, xc[jj].y);
+            if (MODE == 0) {
+                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                if (jj == 0)
+                    mma_f16_16816(pu, f16_lo_nibbles(VA[jj], klo), f16_lo_nibbles(VB[jj], klo),
+                                  f16_lo_nibbles(va8, klo), f16_lo_nibbles(vb8, klo), xc[jj].x, xc[jj].y,
+                                  0.0f, 0.0f, 0.0f, 0.0f);
+                else
+                    mma_f16_16816(pu, f16_lo_nibbles(VA[jj], klo), f16_lo_nibbles(VB[jj], klo),
+                                  f16_lo_nibbles(va8, klo), f16_lo_nibbles(vb8, klo), xc[jj].x, xc[jj].y);
+            }
+            mma_f16_16816(pg, f16_hi_nibbles(WA[jj], khi), f16_hi_nibbles(WB[jj], khi),
+                          f16_hi_nibbles(wa8, khi), f16_hi_nibbles(wb8, khi), xc[jj].z, xc[jj].w);
+            if (MODE == 0) {
+                const uint32_t va8 = VA[jj] >> 8, vb8 = VB[jj] >> 8;
+                mma_f16_16816(pu, f16_hi_nibbles(VA[jj], khi), f16_hi_nibbles(VB[jj], khi),
+                              f16_hi_nibbles(va8, khi), f16_hi_nibbles(vb8, khi), xc[jj].z, xc[jj].w);
+            }
         }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const float c0 = jj == 0 ? cc0 : 0.0f, c1 = jj == 0 ? cc1 : 0.0f;
-            mma_f16_16816(pg[jj], f16_lo_nibbles(WA[jj]), f16_lo_nibbles(WB[jj]), f16_lo_nibbles(wa8[jj]),
-                          f16_lo_nibbles(wb8[jj]), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
-            if (MODE == 0)
-                mma_f16_16816(pu[jj], f16_lo_nibbles(VA[jj]), f16_lo_nibbles(VB[jj]), f16_lo_nibbles(va8[jj]),
-                              f16_lo_nibbles(vb8[jj]), xc[jj].x, xc[jj].y, c0, c1, c0, c1);
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            mma_f16_16816(pg[jj], f16_hi_nibbles(WA[jj]), f16_hi_nibbles(WB[jj]), f16_hi_nibbles(wa8[jj]),
-                          f16_hi_nibbles(wb8[jj]), xc[jj].z, xc[jj].w);
-            if (MODE == 0)
-                mma_f16_16816(pu[jj], f16_hi_nibbles(VA[jj]), f16_hi_nibbles(VB[jj]), f16_hi_nibbles(va8[jj]),
-                              f16_hi_nibbles(vb8[jj]), xc[jj].z, xc[jj].w);
-        }
+        // C columns 2c and 2c + 1 (r & 1) are token rows tc0 and tc1
         const float sga = sga_p[G], sgb = sgb_p[G];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-            acc0[r] = fmaf((pg[0][r] + pg[1][r]) + (pg[2][r] + pg[3][r]), r < 2 ? sga : sgb, acc0[r]);
+        for (int r = 0; r < 4; ++r) acc0[r] = fmaf(pg[r] + ((r & 1) ? cc1 : cc0), r < 2 ? sga : sgb, acc0[r]);
         if (MODE == 0) {
             const float sua = sua_p[G], sub = sub_p[G];
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                acc1[r] = fmaf((pu[0][r] + pu[1][r]) + (pu[2][r] + pu[3][r]), r < 2 ? sua : sub, acc1[r]);
+            for (int r = 0; r < 4; ++r) acc1[r] = fmaf(pu[r] + ((r & 1) ? cc1 : cc0), r < 2 ? sua : sub, acc1[r]);
         }
     };
 
@@ -435,7 +438,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         bool ok = true;
         if (ti.kind == 1) {
             // routed chunks hold at most 8 tokens: one n-tile
-            ok = consume_int4<MODE>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, acc0[0], acc1[0], p.status);
+            ok = consume_int4<MODE>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, p.f16_magic_lo, p.f16_magic_hi,
+                                   acc0[0], acc1[0], p.status);
         } else {
             // ---------------- bf16 weights (shared expert): 64 K per tile ----------------
             // thread c takes the 8-blocks c and c + 4 of each 64-K tile, of the

@@ -24,6 +24,8 @@ struct DecodeParams {
     int32_t K_r, K_s;       // reduction lengths (routed, shared)
     int32_t k_top;
     int32_t scale_buf_floats;
+    uint32_t f16_magic_lo;  // kF16MagicLo, kF16MagicHi: passed at run time so the int4 unpacking
+    uint32_t f16_magic_hi;  // holds them in registers (one LOP3 per two codes)
     const ChunkEntry* chunks;
     const int32_t* n_chunks;
     const int32_t* perm;    // sorted position -> slot (t * k + j)

@@ -294,6 +294,8 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.K_s = L.D;
     p.k_top = L.k;
     p.scale_buf_floats = decode_scale_floats(0, L.D);
+    p.f16_magic_lo = kF16MagicLo;
+    p.f16_magic_hi = kF16MagicHi;
     p.chunks = chunks;
     p.n_chunks = nch;
     p.perm = perm;
@@ -446,6 +448,7 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.perm = perm;
     p.inv_perm = inv;
     p.k_top = L.k;
+    p.bf16_magic = kBf16Magic;
     p.status = status;
     float* y_shared = at<float>(ws, W.y_shared);
 

@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         }
         const int ng = p.K / kGroup;
         const __nv_bfloat162 k136 = __floats2bfloat162_rn(136.0f, 136.0f);
+        const uint32_t magic = p.bf16_magic;
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             int ci, fb;
@@ -389,7 +390,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                     uint32_t o[4];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        uint32_t t = ((w[jj] >> (4 * h)) & 0x000F000Fu) ^ 0x43084308u;   // bf16 136 + q
+                        uint32_t t = bf16_lo_nibbles(w[jj] >> (4 * h), magic);   // bf16 136 + q
                         __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&t), k136);
                         __nv_bfloat162 r = __hmul2(q, s2);
                         o[h] = *reinterpret_cast<uint32_t*>(&r);

@@ -36,6 +36,7 @@ struct TcParams {
     const float* y_r;          // ... and the shared expert's y_s it adds
     const int32_t* inv_perm;   // slot -> position
     int32_t k_top;
+    uint32_t bf16_magic;       // kBf16Magic, passed at run time so the int4 converters hold it in a register
     int32_t* status;
 };
 
