@@ -134,30 +134,71 @@ def workload_text(s: synth.LayerShape) -> str:
 # clocks sampled while the timed loop runs
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled every ~20 ms by
+    NVML in a thread (nvidia-smi every 50 ms if NVML is unavailable), so
+    that even a timed region of a fraction of a second gets samples."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, device_index: int):
         self.proc = None
-        self.lines = []
+        self.samples = []          # (time, sm_mhz, max_mhz, reasons)
+        self.stop_flag = threading.Event()
+        self.t = None
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.reasons_fn = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                               or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.t.start()
+            return
+        except Exception as e:  # no NVML: fall back to nvidia-smi
+            log("NVML clock sampling unavailable (%s); using nvidia-smi" % e)
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "--id=" + uuid, "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
             self.t.start()
-        except Exception as e:  # no nvidia-smi: report no clocks
+        except Exception as e:
             log("clock sampling unavailable:", e)
             self.proc = None
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = int(self.reasons_fn(self.h))
+                reasons = {n for n, b in self.REASON_BITS.items() if bits & b}
+                self.samples.append((time.time(), sm, self.max_mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def _read_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [p.strip() for p in line.strip().split(",")]
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except (ValueError, IndexError):
+                continue
+            reasons = {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}
+            self.samples.append((time.time(), sm, mx, reasons))
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -166,25 +207,14 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0: float, t1: float):
-        if not self.proc or not self.lines:
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:
             return None
-        inside = [l for t, l in self.lines if t0 <= t <= t1] or [l for _, l in self.lines]
-        sm, mx, reasons = [], None, set()
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in inside:
-            parts = [p.strip() for p in l.split(",")]
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names[1:], parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for s in inside:
+            reasons |= s[3]
+        return {"sm_mhz": float(np.median([s[1] for s in inside])), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside)}
 
 
 # ---------------------------------------------------------------------------
