@@ -102,9 +102,9 @@ def quant_matrices():
     return [("gate", E * F, D), ("up", E * F, D), ("down", E * D, F)]
 
 
-def quant_bytes(rows: int, cols: int) -> int:
+def quant_bytes(rows: int, cols: int, group: int = 128) -> int:
     """Algorithmic bytes of int4_row_quantize: fp32 in, codes + scales out."""
-    return rows * cols * 4 + rows * cols // 2 + rows * (cols // 128) * 4
+    return rows * cols * 4 + rows * cols // 2 + rows * (cols // group) * 4
 
 
 def max_over_ranks(values, dev, world: int):
@@ -116,14 +116,14 @@ def max_over_ranks(values, dev, world: int):
     return [float(v) for v in t.tolist()]
 
 
-def weights_text(s: synth.LayerShape) -> str:
+def weights_text(s: synth.LayerShape, group: int = 128) -> str:
     if s.fmt == "int4":
-        return "routed int4 g128 (fp32 scales, zero point 0); router and shared bf16"
+        return "routed int4 g%d (fp32 scales, zero point 0); router and shared bf16" % group
     return "routed e4m3 rows (fp32 row scales), e4m3 per-row activations; router and shared bf16"
 
 
-def workload_text(s: synth.LayerShape) -> str:
-    w = "int4 g128" if s.fmt == "int4" else "fp8 e4m3 rows"
+def workload_text(s: synth.LayerShape, group: int = 128) -> str:
+    w = ("int4 g%d" % group) if s.fmt == "int4" else "fp8 e4m3 rows"
     gate = "sigmoid" if s.k == 1 else "softmax over top-%d" % s.k
     return ("%s: T=%d tokens, d_model=%d, expert d_ff=%d, E=%d routed experts (%s), top-%d %s gate, "
             "bf16 shared expert d_ff=%d%s" % (s.name, s.T, s.D, s.F, s.E, w, s.k, gate, s.F_shared,
@@ -220,7 +220,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
+def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device, group: int = 128):
     import int4_quantized_expert_b200 as moe
     E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
     wr = synth.router_weight(seed, E, D).to(dev)
@@ -229,8 +229,8 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
     sg, su, sd = (t.to(dev) for t in synth.shared_weights(seed, D, Fs))
     if shape.fmt == "int4":
         alloc = lambda n, kk: (torch.empty(E, n, kk // 2, dtype=torch.uint8, device=dev),
-                               torch.empty(E, n, kk // 128, dtype=torch.float32, device=dev))
-        quant = lambda w, out: moe.quantize_int4(w, out=out)
+                               torch.empty(E, n, kk // group, dtype=torch.float32, device=dev))
+        quant = lambda w, out: moe.quantize_int4(w, group_size=group, out=out)
         fmt = moe.FMT_INT4
     else:
         alloc = lambda n, kk: (torch.empty(E, n, kk, dtype=torch.uint8, device=dev),
@@ -254,12 +254,12 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device):
     del wbuf
     torch.cuda.synchronize()
     layer = moe.MoELayer(E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr, router_bias=bias, gate=gate,
-                         up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T)
+                         up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T, group_size=group)
     x = synth.tokens(seed, shape.T, D).to(dev)
     return layer, x, (wr, bias)
 
 
-def kernel_work(shape: synth.LayerShape, n_touched: int) -> dict:
+def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> dict:
     """Algorithmic work per launch of each kernel, as (kind, amount):
     ("bytes", HBM bytes with every weight byte of a touched expert and of the
     shared expert read once and every activation read and written once) for
@@ -268,9 +268,9 @@ def kernel_work(shape: synth.LayerShape, n_touched: int) -> dict:
     T, D, F, Fs, E, k = shape.T, shape.D, shape.F, shape.F_shared, shape.E, shape.k
     S = T * k
     codes_gu = 2 * F * D // 2
-    scales_gu = 2 * F * (D // 128) * 4
+    scales_gu = 2 * F * (D // group) * 4
     codes_d = D * F // 2
-    scales_d = D * (F // 128) * 4
+    scales_d = D * (F // group) * 4
     if shape.fmt == "fp8":   # e4m3 routed experts: one tensor-core pass each, bf16-equivalent flop count
         return {
             "router": ("flops", 2 * T * D * E),
@@ -309,7 +309,7 @@ def layer_flops(shape: synth.LayerShape) -> int:
 def run_ours(args, rank: int, world: int, dev: torch.device):
     import int4_quantized_expert_b200 as moe
     shape = synth.SHAPES[args.workload]
-    layer, x, (wr, bias) = build_layer(shape, args.seed + 0, dev)
+    layer, x, (wr, bias) = build_layer(shape, args.seed + 0, dev, args.group_size)
     r = moe.route(x, wr, bias, shape.k)
     n_touched = int((r["counts"] > 0).sum().item())
     names = layer.launch_names(shape.T)
@@ -389,7 +389,7 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         e2e_ms += e0.elapsed_time(e1)
     e2e_ms = max_over_ranks([e2e_ms / n_e2e], dev, world)[0]
 
-    work = kernel_work(shape, n_touched)
+    work = kernel_work(shape, n_touched, args.group_size)
     dom = int(np.argmax(per_kernel))
     dom_name = names[dom]
     hbm_peak, tc_peak, peak_src = peaks()
@@ -424,8 +424,8 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         "data": ("synthetic (seeded; no dataset, random-init weights of the stated shapes: x, router and "
                  "shared expert from PCG64, routed experts N(0, 0.02) from torch's device generator)"),
         "config": {
-            "workload": workload_text(shape),
-            "weights": weights_text(shape),
+            "workload": workload_text(shape, args.group_size),
+            "weights": weights_text(shape, args.group_size),
             "parallelism": "replicas" if world > 1 else "single GPU",
             "experts_touched": n_touched,
             "l2": "flushed between steps (256 MB write)",
@@ -462,14 +462,14 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
     for name, rows, cols in quant_matrices():
         w = torch.randn(rows, cols, generator=gen, device=dev, dtype=torch.float32).mul_(synth.WEIGHT_STD)
         codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
-        scales = torch.empty(rows, cols // 128, dtype=torch.float32, device=dev)
+        scales = torch.empty(rows, cols // args.group_size, dtype=torch.float32, device=dev)
         mats.append((name, w, codes, scales))
-    step_bytes = sum(quant_bytes(w.shape[0], w.shape[1]) for _, w, _, _ in mats)
+    step_bytes = sum(quant_bytes(w.shape[0], w.shape[1], args.group_size) for _, w, _, _ in mats)
     stream = torch.cuda.current_stream()
 
     def step():
         for _, w, c, sc in mats:
-            moe.quantize_int4(w, out=(c, sc))
+            moe.quantize_int4(w, group_size=args.group_size, out=(c, sc))
 
     for _ in range(args.warmup):
         step()
@@ -504,7 +504,7 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
         e0.record(stream)
         for (_, w, c, sc), (wh, ch, sh) in zip(mats, host):
             w.copy_(wh, non_blocking=True)
-            moe.quantize_int4(w, out=(c, sc))
+            moe.quantize_int4(w, group_size=args.group_size, out=(c, sc))
             ch.copy_(c, non_blocking=True)
             sh.copy_(sc, non_blocking=True)
         e1.record(stream)
@@ -531,7 +531,7 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
         "dtype": "f32 -> int4 (fp32 scales)",
         "data": "synthetic (N(0, 0.02) fp32 weights from torch's seeded device generator)",
         "config": {
-            "workload": "quantize: int4_row_quantize (group 128) of 16 experts x {gate [8192, 5120], "
+            "workload": "quantize: int4_row_quantize (group %d) of 16 experts x {gate [8192, 5120], " % args.group_size +
                         "up [8192, 5120], down [5120, 8192]} fp32 = 2.01 G weights, 3 calls per step",
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": "inputs (8.05 GB) larger than L2; no flush",
@@ -547,26 +547,26 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
     return result
 
 
-def time_oracle_quantize(seed: int, budget_s: float, n_steps: int, n_warm: int):
+def time_oracle_quantize(seed: int, budget_s: float, n_steps: int, n_warm: int, group: int = 128):
     """The oracle's int4_row_quantize (then packing) on row blocks of the gate
     projection's shape, sized so a step takes about budget_s; returns (GB/s
     of algorithmic bytes, sample text, seconds per step)."""
     from oracle import quant as oq
     w = synth.expert_weights(seed, 0, QUANT_D, QUANT_F)[0]       # [8192, 5120] fp32
     t = time.perf_counter()
-    oq.pack_int4(oq.int4_row_quantize(w[:64])[0])
+    oq.pack_int4(oq.int4_row_quantize(w[:64], group_size=group)[0])
     c64 = max(time.perf_counter() - t, 1e-4)
     rows = int(min(w.shape[0], max(64, budget_s / c64 * 64 // 64 * 64)))
     blk = np.ascontiguousarray(w[:rows])
     for _ in range(n_warm):
-        oq.pack_int4(oq.int4_row_quantize(blk)[0])
+        oq.pack_int4(oq.int4_row_quantize(blk, group_size=group)[0])
     t = time.perf_counter()
     for _ in range(n_steps):
-        oq.pack_int4(oq.int4_row_quantize(blk)[0])
+        oq.pack_int4(oq.int4_row_quantize(blk, group_size=group)[0])
     el = (time.perf_counter() - t) / max(n_steps, 1)
     sample = ("the first %d of 8192 rows of expert 0's gate projection [8192, 5120] per step (%.2f%% of "
               "the 2.01 G-weight set); GB/s of algorithmic bytes" % (rows, 100.0 * rows * QUANT_D / 2.01e9))
-    return quant_bytes(rows, QUANT_D) / el / 1e9, sample, el
+    return quant_bytes(rows, QUANT_D, group) / el / 1e9, sample, el
 
 
 # ---------------------------------------------------------------------------
@@ -583,7 +583,7 @@ def oracle_cores() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_sample_layer(shape: synth.LayerShape, seed: int, f_sub: int, token: int, x):
+def oracle_sample_layer(shape: synth.LayerShape, seed: int, f_sub: int, token: int, x, group: int = 128):
     """The oracle's layer restricted to the first f_sub hidden units of every
     expert (and of the shared expert): a layer of the same kind whose work per
     token is f_sub / F of the full one.  Weights are quantized before timing."""
@@ -596,25 +596,27 @@ def oracle_sample_layer(shape: synth.LayerShape, seed: int, f_sub: int, token: i
     experts = {}
     for e in ids:
         g, u, d = synth.expert_weights(seed, int(e), shape.D, shape.F)
-        quant = oq.int4_row_quantize if shape.fmt == "int4" else oq.fp8_row_quantize
+        quant = ((lambda w: oq.int4_row_quantize(w, group_size=group)) if shape.fmt == "int4"
+                 else oq.fp8_row_quantize)
         experts[int(e)] = tuple(quant(np.ascontiguousarray(w))
                                 for w in (g[:f_sub], u[:f_sub], d[:, :f_sub]))
     return offn.Layer(shape.fmt, shape.k, wr, bias, experts.__getitem__,
-                      (sg[:fs_sub], su[:fs_sub], sd[:, :fs_sub].contiguous())), fs_sub
+                      (sg[:fs_sub], su[:fs_sub], sd[:, :fs_sub].contiguous()), group_size=group), fs_sub
 
 
-def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: int, n_warm: int):
+def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: int, n_warm: int,
+                group: int = 128):
     """Runs the oracle for one token per step on a hidden-width slice sized so
     a step takes about budget_s; returns (tokens/s, sample text, per-step s)."""
     from oracle import ffn as offn
     x = synth.tokens(seed, shape.T, shape.D)
     probe_f = 128
-    lay, fs = oracle_sample_layer(shape, seed, probe_f, 0, x)
+    lay, fs = oracle_sample_layer(shape, seed, probe_f, 0, x, group)
     t = time.perf_counter()
     offn.moe_forward(lay, x, tokens=[0])
     c128 = max(time.perf_counter() - t, 1e-4)
     f_sub = int(min(shape.F, max(128, (budget_s / c128) * 128 // 128 * 128)))
-    lay, fs = oracle_sample_layer(shape, seed, f_sub, 0, x)
+    lay, fs = oracle_sample_layer(shape, seed, f_sub, 0, x, group)
     for _ in range(n_warm):
         offn.moe_forward(lay, x, tokens=[0])
     t = time.perf_counter()
@@ -632,7 +634,7 @@ def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: in
 def run_reference(args):
     budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
     if args.workload == "quantize":
-        v, sample, per_step = time_oracle_quantize(args.seed, budget, args.steps, args.warmup)
+        v, sample, per_step = time_oracle_quantize(args.seed, budget, args.steps, args.warmup, args.group_size)
         return {
             "impl": "reference", "metric": QUANT_METRIC, "value": v, "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
@@ -644,7 +646,7 @@ def run_reference(args):
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
     shape = synth.SHAPES[args.workload]
-    v, sample, per_step = time_oracle(shape, args.seed, budget, args.steps, args.warmup)
+    v, sample, per_step = time_oracle(shape, args.seed, budget, args.steps, args.warmup, args.group_size)
     cores = oracle_cores()
     return {
         "impl": "reference",
@@ -660,7 +662,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded; no dataset, random-init weights of the stated shapes)",
-        "config": {"workload": workload_text(shape), "weights": weights_text(shape),
+        "config": {"workload": workload_text(shape, args.group_size), "weights": weights_text(shape, args.group_size),
                    "parallelism": "CPU oracle on the host cores"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -678,6 +680,8 @@ def main(argv=None):
                              "quantize"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--group-size", type=int, default=128, choices=[128, 64, 32],
+                    help="int4 group size of the routed experts (and of the quantize workload)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -703,13 +707,13 @@ def main(argv=None):
     if args.workload == "quantize":
         result = run_quantize(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            v, sample, _ = time_oracle_quantize(args.seed, budget_s=5.0, n_steps=2, n_warm=0)
+            v, sample, _ = time_oracle_quantize(args.seed, budget_s=5.0, n_steps=2, n_warm=0, group=args.group_size)
             result["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": 1,   # element-wise numpy: one thread
                                       "kind": "oracle", "sample": sample}
     else:
         result, shape = run_ours(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            v, sample, _ = time_oracle(shape, args.seed, budget_s=10.0, n_steps=2, n_warm=0)
+            v, sample, _ = time_oracle(shape, args.seed, budget_s=10.0, n_steps=2, n_warm=0, group=args.group_size)
             result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle_cores(),
                                       "kind": "oracle", "sample": sample}
     if world > 1:

@@ -11,7 +11,8 @@
  *   [P2] "Meta Llama Models Llama 4 单卡量化推理与选型指南" (lshu.cn):
  *        "量化环节做了什么" (bmm_nt: FP8 row-wise weights with per-row
  *        activation quantization, or int4 group-128 weights with zero points
- *        equal to zero; activations stay bf16).
+ *        equal to zero; activations stay bf16; a smaller group_size named as
+ *        the int4 path's likely next step).
  *   [P5] "Llama 开源模型系列" (docs.ifdog.com): "MoE 架构详解" (router =
  *        linear layer, top-1 of 16 / top-8 of 128) and "SwiGLU：门控激活的数学".
  *
@@ -58,7 +59,8 @@ typedef enum {
 typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP32 = 1 } moe_dtype;
 
 typedef enum {
-    MOE_WEIGHTS_INT4_G128 = 0,  /* int4 codes, two per byte, fp32 scale per 128 K */
+    MOE_WEIGHTS_INT4_G128 = 0,  /* int4 codes, two per byte, fp32 scale per group of K
+                                   (128 by default; 64 or 32 per moe_layer_desc.group_size) */
     MOE_WEIGHTS_FP8_ROW = 1     /* e4m3 codes, fp32 scale per row */
 } moe_weight_format;
 
@@ -83,7 +85,8 @@ MOE_API int32_t moe_abi_version(void);
  *   w       device, fp32 [rows, cols]
  *   codes   device, uint8 [rows, cols / 2]       (output)
  *   scales  device, fp32 [rows, cols / group_size] (output)
- * Requires group_size == 128, cols % 128 == 0, rows >= 0 (0 = no-op).
+ * Requires group_size 128, 64 or 32 (the smaller groups: [P2]'s next step),
+ * cols % 128 == 0, rows >= 0 (0 = no-op).
  */
 MOE_API moe_status moe_quantize_int4(const float* w, int64_t rows, int64_t cols, int32_t group_size,
                              uint8_t* codes, float* scales, void* stream);
@@ -134,9 +137,12 @@ MOE_API moe_status moe_route(const void* x, int32_t T, int32_t D,
  * Description of one MoE FFN layer.  All pointers are device pointers.
  *   E routed experts, k experts per token, D model width, F routed hidden
  *   width, F_shared shared-expert hidden width.
- *   INT4_G128: w_gate, w_up uint8 [E, F, D/2]; s_gate, s_up fp32 [E, F, D/128];
- *              w_down uint8 [E, D, F/2]; s_down fp32 [E, D, F/128]
+ *   INT4_G128: w_gate, w_up uint8 [E, F, D/2]; s_gate, s_up fp32 [E, F, D/G];
+ *              w_down uint8 [E, D, F/2]; s_down fp32 [E, D, F/G], G = group_size
  *              (the layout moe_quantize_int4 writes, one expert after another).
+ *              G = 128, 64 or 32; groups of 64 and 32 run on the tensor-core
+ *              tiles only (AUTO takes PREFILL for them; DECODE is refused with
+ *              MOE_ERR_UNSUPPORTED_SHAPE).
  *   FP8_ROW:   w_gate, w_up uint8 [E, F, D]; s_gate, s_up fp32 [E, F];
  *              w_down uint8 [E, D, F]; s_down fp32 [E, D]
  *              (the layout moe_quantize_fp8_rows writes); every expert matmul
@@ -148,7 +154,7 @@ MOE_API moe_status moe_route(const void* x, int32_t T, int32_t D,
 typedef struct moe_layer_desc {
     int32_t E, k, D, F, F_shared;
     int32_t format;        /* moe_weight_format */
-    int32_t group_size;    /* 128 for INT4_G128; ignored for FP8_ROW */
+    int32_t group_size;    /* INT4_G128: 128, 64 or 32; ignored for FP8_ROW */
     int32_t path;          /* moe_path */
     const void* w_router;      /* bf16 [E, D] */
     const float* router_bias;  /* fp32 [E] or NULL */

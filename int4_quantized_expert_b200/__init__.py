@@ -179,17 +179,19 @@ class MoELayer:
     """One MoE FFN layer on the GPU: holds the (already quantized) weights,
     a workspace for up to ``T_max`` tokens, and the ``moe_layer_desc``.
 
-    Routed weights: int4 -- (codes uint8 [E, N, K/2], scales fp32 [E, N, K/128])
-    per projection; fp8 -- (codes uint8 [E, N, K], scales fp32 [E, N]).
+    Routed weights: int4 -- (codes uint8 [E, N, K/2], scales fp32 [E, N, K/group_size])
+    per projection, group_size 128, 64 or 32; fp8 -- (codes uint8 [E, N, K],
+    scales fp32 [E, N]).
     """
 
     def __init__(self, *, E: int, k: int, D: int, F: int, F_shared: int, w_router: torch.Tensor,
                  router_bias: Optional[torch.Tensor], gate, up, down, shared, fmt: int = FMT_INT4,
-                 act_scale_ub: float = math.inf, T_max: int = 16, path: int = PATH_AUTO):
+                 act_scale_ub: float = math.inf, T_max: int = 16, path: int = PATH_AUTO,
+                 group_size: int = 128):
         self.tensors = [w_router, router_bias, *gate, *up, *down, *shared]   # keep alive
         d = LayerDesc()
         d.E, d.k, d.D, d.F, d.F_shared = E, k, D, F, F_shared
-        d.format, d.group_size, d.path = fmt, 128, path
+        d.format, d.group_size, d.path = fmt, group_size, path
         d.w_router, d.router_bias = _ptr(w_router), _ptr(router_bias)
         d.w_gate, d.s_gate = _ptr(gate[0]), _ptr(gate[1])
         d.w_up, d.s_up = _ptr(up[0]), _ptr(up[1])

@@ -10,8 +10,8 @@
 #include "tc_gemm.cuh"
 
 namespace moe {
-moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, uint8_t* codes, float* scales,
-                                cudaStream_t stream);
+moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, int group_size, uint8_t* codes,
+                                float* scales, cudaStream_t stream);
 moe_status launch_quantize_fp8_rows(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
                                     int64_t num_valid, float scale_ub, uint8_t* q, float* scales,
                                     cudaStream_t stream);
@@ -51,6 +51,8 @@ struct WsLayout {
     size_t x_in, out;
     size_t total;
 };
+
+inline bool int4_group_ok(int g) { return g == 128 || g == 64 || g == 32; }
 
 enum { PATH_SEL_DECODE = 1, PATH_SEL_PREFILL = 2 };
 
@@ -113,18 +115,24 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     return w;
 }
 
+bool decode_fits(const moe_layer_desc& L);
+
 // Workspace for every call with this descriptor and at most T tokens: the
 // fixed path's layout, or the larger of the two when the path depends on T.
 size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
     const size_t a = ws_layout(L, T, PATH_SEL_DECODE).total;
     const size_t b = ws_layout(L, T, PATH_SEL_PREFILL).total;
     if (L.format == MOE_WEIGHTS_FP8_ROW || L.path == MOE_PATH_PREFILL) return b;
+    if (L.path == MOE_PATH_AUTO && !decode_fits(L)) return b;   // AUTO never takes the decode path
     if (L.path == MOE_PATH_DECODE) return a;
     return a > b ? a : b;
 }
 
-// The weight-streaming kernels keep a task's int4 scales in shared memory.
+// The weight-streaming kernels keep a task's int4 scales in shared memory,
+// and their MMAs sum whole groups of 128 K before scaling: smaller groups
+// run on the tensor-core tiles only.
 bool decode_fits(const moe_layer_desc& L) {
+    if (L.format == MOE_WEIGHTS_INT4_G128 && L.group_size != 128) return false;
     return decode_smem_bytes(0, decode_scale_floats(0, L.D)) <= kMaxDecodeSmem &&
            decode_smem_bytes(1, decode_scale_floats(1, L.F)) <= kMaxDecodeSmem;
 }
@@ -141,7 +149,7 @@ moe_status check_layer(const moe_layer_desc* L) {
     if (L->E < 1 || L->E > 256 || L->k < 1 || L->k > L->E || L->k > 8) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!valid_dim(L->D) || !valid_dim(L->F) || !valid_dim(L->F_shared)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (L->format != MOE_WEIGHTS_INT4_G128 && L->format != MOE_WEIGHTS_FP8_ROW) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (L->format == MOE_WEIGHTS_INT4_G128 && L->group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->format == MOE_WEIGHTS_INT4_G128 && !int4_group_ok(L->group_size)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (L->format == MOE_WEIGHTS_FP8_ROW && !(L->act_scale_ub > 0.0f)) return MOE_ERR_INVALID_ARG;
     if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
     const void* ptrs[] = {L->w_router, L->w_gate, L->s_gate, L->w_up, L->s_up, L->w_down, L->s_down,
@@ -448,6 +456,7 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.perm = perm;
     p.inv_perm = inv;
     p.k_top = L.k;
+    p.group_shift = L.group_size == 32 ? 5 : L.group_size == 64 ? 6 : 7;   // int4: log2 of the group
     p.bf16_magic = kBf16Magic;
     p.status = status;
     float* y_shared = at<float>(ws, W.y_shared);
@@ -536,12 +545,12 @@ int32_t moe_abi_version(void) { return 1; }
 
 moe_status moe_quantize_int4(const float* w, int64_t rows, int64_t cols, int32_t group_size, uint8_t* codes,
                              float* scales, void* stream) {
-    if (group_size != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!int4_group_ok(group_size)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (rows < 0 || cols <= 0 || cols % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (rows == 0) return MOE_OK;
     if (!w || !codes || !scales || !aligned16(w) || !aligned16(codes) || !aligned16(scales))
         return MOE_ERR_INVALID_ARG;
-    return launch_quantize_int4(w, rows, cols, codes, scales, as_stream(stream));
+    return launch_quantize_int4(w, rows, cols, group_size, codes, scales, as_stream(stream));
 }
 
 moe_status moe_quantize_fp8_rows(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,

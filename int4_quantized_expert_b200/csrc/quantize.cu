@@ -1,8 +1,11 @@
-// Quantization kernels: int4 groups of 128 and e4m3 rows.
+// Quantization kernels: int4 groups (of 128, or 64 or 32) and e4m3 rows.
 //
 // int4_row_quantize, from "1 卡跑通 Llama 4" (discosf.com), section
 // "FP8 / Int4 混合量化": per group of 128 consecutive K values,
 // scale = max(max|w|, 1e-6) / 8 and q = clamp(round(w / scale), -8, 7).
+// Groups of 64 and 32 follow the same rule: "Meta Llama Models Llama 4 单卡
+// 量化推理与选型指南" (lshu.cn) names a smaller group_size as the likely next
+// step of the int4 path.
 // FP8 row quantization, from "Meta Llama Models Llama 4 单卡量化推理与选型指南"
 // (lshu.cn), section "量化环节做了什么" (quantize_fp8_per_row).
 //
@@ -15,34 +18,39 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// int4: one warp quantizes one group per step (128 fp32 = 32 lanes x float4),
-// UNROLL groups in flight per warp to keep enough bytes in flight.
+// int4: one warp quantizes one block of 128 consecutive values per step
+// (32 lanes x float4), UNROLL blocks in flight per warp to keep enough bytes
+// in flight.  A block holds 128 / G groups of G = 4 * LPG values; the group
+// maximum is reduced over its LPG lanes (G = 128, 64 or 32: 32, 16 or 8
+// lanes), whose first lane writes the scale.  Groups never straddle rows
+// (the row length is a multiple of 128), so group g covers elements
+// g * G .. g * G + G - 1 of the flattened matrix and its scale is scales[g].
 // ---------------------------------------------------------------------------
-template <int UNROLL>
+template <int UNROLL, int LPG>
 __global__ void __launch_bounds__(256) quantize_int4_kernel(const float* __restrict__ w,
-                                                            int64_t n_groups,
+                                                            int64_t n_blocks,
                                                             uint8_t* __restrict__ codes,
                                                             float* __restrict__ scales) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
 
-    for (int64_t g0 = warp * UNROLL; g0 < n_groups; g0 += n_warps * UNROLL) {
+    for (int64_t b0 = warp * UNROLL; b0 < n_blocks; b0 += n_warps * UNROLL) {
         uint4 v[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t g = g0 + u;
-            if (g < n_groups) v[u] = ldg_stream(w + g * kGroup + lane * 4);
+            const int64_t b = b0 + u;
+            if (b < n_blocks) v[u] = ldg_stream(w + b * 128 + lane * 4);
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t g = g0 + u;
-            if (g >= n_groups) break;
+            const int64_t b = b0 + u;
+            if (b >= n_blocks) break;
             float f[4] = {__uint_as_float(v[u].x), __uint_as_float(v[u].y),
                           __uint_as_float(v[u].z), __uint_as_float(v[u].w)};
             float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            for (int o = LPG / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             const float s = fmaxf(m, 1e-6f) * 0.125f;   // exact: division by 8
             // q = clamp(rint(w / s)) with w / s the IEEE quotient.  |w / s| <= 8,
             // and y = w * rn(1 / s) lies within 2^-19 of that quotient (two
@@ -58,8 +66,8 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(const float* __restr
                 const float q = fminf(fmaxf(rintf(y), -8.0f), 7.0f);   // half to even
                 packed |= (uint32_t(int(q)) & 0xFu) << (4 * i);
             }
-            reinterpret_cast<uint16_t*>(codes + g * (kGroup / 2))[lane] = uint16_t(packed);
-            if (lane == 0) scales[g] = s;
+            reinterpret_cast<uint16_t*>(codes + b * 64)[lane] = uint16_t(packed);
+            if (lane % LPG == 0) scales[b * (32 / LPG) + lane / LPG] = s;
         }
     }
 }
@@ -155,19 +163,24 @@ __global__ void __launch_bounds__(256) quantize_fp8_rows_kernel(const T* __restr
     }
 }
 
-moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, uint8_t* codes,
+moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, int group_size, uint8_t* codes,
                                 float* scales, cudaStream_t stream) {
-    const int64_t n_groups = rows * (cols / kGroup);
-    if (n_groups == 0) return MOE_OK;
+    const int64_t n_blocks = rows * (cols / 128);
+    if (n_blocks == 0) return MOE_OK;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     constexpr int UNROLL = 4;
-    const int64_t warps_needed = ceil_div(n_groups, UNROLL);
+    const int64_t warps_needed = ceil_div(n_blocks, UNROLL);
     int64_t blocks = ceil_div(warps_needed, 8);
     const int64_t cap = int64_t(sms) * 8;    // 8 CTAs x 256 threads per SM, grid-stride beyond
     if (blocks > cap) blocks = cap;
-    quantize_int4_kernel<UNROLL><<<unsigned(blocks), 256, 0, stream>>>(w, n_groups, codes, scales);
+    switch (group_size) {
+        case 128: quantize_int4_kernel<UNROLL, 32><<<unsigned(blocks), 256, 0, stream>>>(w, n_blocks, codes, scales); break;
+        case 64: quantize_int4_kernel<UNROLL, 16><<<unsigned(blocks), 256, 0, stream>>>(w, n_blocks, codes, scales); break;
+        case 32: quantize_int4_kernel<UNROLL, 8><<<unsigned(blocks), 256, 0, stream>>>(w, n_blocks, codes, scales); break;
+        default: return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
     return launch_status();
 }
 

@@ -357,7 +357,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             srow_off = i;
             sbase = p.s0;
         }
-        const int ng = p.K / kGroup;
+        // groups of 128, 64 or 32 K: this thread's 32 K of stage kk lie in
+        // group (64 kk + 32 hh) >> gsh, a new one every spg stages; a
+        // group's scale is loaded two groups ahead
+        const int gsh = p.group_shift;
+        const int spg = gsh == 7 ? 2 : 1;
+        const int ng = p.K >> gsh;
         const __nv_bfloat162 k136 = __floats2bfloat162_rn(136.0f, 136.0f);
         const uint32_t magic = p.bf16_magic;
         uint32_t it = 0;
@@ -366,14 +371,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
             const ChunkEntry ce = p.chunks[c_begin + ci];
             const float* srow = sbase + int64_t(ce.expert * p.n_rows + fb * (GATEUP ? 64 : 128) + srow_off) * ng;
-            float s_next = ldg_f32(srow);
-            bool ok = true;
+            auto scale_of = [&](int kq) { return ldg_f32(srow + ((64 * kq + 32 * hh) >> gsh)); };
+            float s_a = scale_of(0), s_b = spg < nk ? scale_of(spg) : 0.0f;
             __nv_bfloat162 s2 = __floats2bfloat162_rn(0.f, 0.f);
+            bool ok = true;
             for (int kk = 0; kk < nk; ++kk, ++it) {
-                if ((kk & 1) == 0) {                           // a new group of 128 K
-                    s2 = __floats2bfloat162_rn(s_next, s_next);
-                    const int gn = kk / 2 + 1;
-                    if (gn < ng) s_next = ldg_f32(srow + gn);
+                if ((kk & (spg - 1)) == 0) {                  // this thread enters a new group
+                    s2 = __floats2bfloat162_rn(s_a, s_a);
+                    s_a = s_b;
+                    if (kk + 2 * spg < nk) s_b = scale_of(kk + 2 * spg);
                 }
                 const uint32_t slot = it % TC_STAGES, cs = it % TC_CSTAGES;
                 if (!mbar_wait(&sm->cfull[cs], (it / TC_CSTAGES) & 1, p.status)) { ok = false; break; }

@@ -25,7 +25,7 @@ struct TcParams {
     const ChunkEntry* chunks;  // token chunks of <= 256 (shared expert's first)
     const int32_t* n_chunks;   // [0] all chunks, [1] the shared expert's
     int32_t routed;            // 1: chunks [n_shared, n_all); 0: chunks [0, n_shared)
-    const float* s0;           // weight scales (gate or down): int4 [E * rows, K / 128]; e4m3 [E * rows]
+    const float* s0;           // weight scales (gate or down): int4 [E * rows, K / group]; e4m3 [E * rows]
     const float* s1;           // weight scales (up)
     const float* tok_scale;    // e4m3 modes: row scale of each token row of B (by slot position)
     bf16* h_out;               // gate/up output rows [*, n_rows] (row = slot position or token)
@@ -36,6 +36,7 @@ struct TcParams {
     const float* y_r;          // ... and the shared expert's y_s it adds
     const int32_t* inv_perm;   // slot -> position
     int32_t k_top;
+    int32_t group_shift;       // int4 modes: log2 of the group size (7, 6 or 5: groups of 128, 64, 32)
     uint32_t bf16_magic;       // kBf16Magic, passed at run time so the int4 converters hold it in a register
     int32_t* status;
 };

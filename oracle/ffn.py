@@ -64,7 +64,8 @@ class Layer:
 
     ``expert(e)`` returns the stored weights of routed expert e as three
     (codes, scales) pairs (gate [F, D], up [F, D], down [D, F]): for "int4"
-    unpacked int8 codes with fp32 group-128 scales, for "fp8" e4m3 codes
+    unpacked int8 codes with fp32 scales, one per ``group_size`` (128, or
+    the smaller 64 / 32) values along K, for "fp8" e4m3 codes
     (uint8) with fp32 row scales.  Router and shared weights are the bf16
     values (any array type; converted to fp64).
     """

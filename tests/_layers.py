@@ -37,7 +37,7 @@ def margin_tokens(shape: synth.LayerShape, w_router, bias, seed: int, margin: bo
 
 
 def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int = moe.PATH_AUTO,
-          device: str = "cuda") -> Built:
+          device: str = "cuda", group_size: int = 128) -> Built:
     E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
     wr = synth.router_weight(seed, E, D)
     bias = synth.router_bias(shape)
@@ -47,8 +47,8 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
 
     if shape.fmt == "int4":
         alloc = lambda n, kk: (torch.empty(E, n, kk // 2, dtype=torch.uint8, device=dev),
-                               torch.empty(E, n, kk // 128, dtype=torch.float32, device=dev))
-        quant = lambda w, out: moe.quantize_int4(w, out=out)
+                               torch.empty(E, n, kk // group_size, dtype=torch.float32, device=dev))
+        quant = lambda w, out: moe.quantize_int4(w, group_size=group_size, out=out)
         fmt = moe.FMT_INT4
     else:
         alloc = lambda n, kk: (torch.empty(E, n, kk, dtype=torch.uint8, device=dev),
@@ -65,16 +65,16 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
         E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr.to(dev),
         router_bias=None if bias is None else torch.from_numpy(bias).to(dev),
         gate=gate, up=up, down=down, shared=(sg.to(dev), su.to(dev), sd.to(dev)),
-        fmt=fmt, T_max=shape.T, path=path)
+        fmt=fmt, T_max=shape.T, path=path, group_size=group_size)
 
     @functools.lru_cache(maxsize=4)
     def expert(e):
         ws = synth.expert_weights(seed, e, D, F)
         if shape.fmt == "int4":
-            return tuple(oq.int4_row_quantize(w) for w in ws)
+            return tuple(oq.int4_row_quantize(w, group_size=group_size) for w in ws)
         return tuple(oq.fp8_row_quantize(w) for w in ws)
 
-    olayer = offn.Layer(shape.fmt, k, wr, bias, expert, (sg, su, sd))
+    olayer = offn.Layer(shape.fmt, k, wr, bias, expert, (sg, su, sd), group_size=group_size)
     return Built(shape, x, layer, olayer, wr, bias)
 
 

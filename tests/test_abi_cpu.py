@@ -41,7 +41,10 @@ def test_version_and_status_strings(lib):
 def test_quantize_rejects_bad_arguments(lib):
     S = moe.Status
     fake = 1 << 20           # an aligned non-null address that is never dereferenced
-    assert lib.moe_quantize_int4(fake, 4, 256, 64, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_int4(fake, 4, 256, 16, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_int4(fake, 4, 256, 96, fake, fake, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_quantize_int4(None, 4, 256, 64, fake, fake, None) == S.INVALID_ARG   # 64: accepted size
+    assert lib.moe_quantize_int4(None, 4, 256, 32, fake, fake, None) == S.INVALID_ARG   # 32: accepted size
     assert lib.moe_quantize_int4(fake, 4, 100, 128, fake, fake, None) == S.UNSUPPORTED_SHAPE
     assert lib.moe_quantize_int4(None, 4, 256, 128, fake, fake, None) == S.INVALID_ARG
     assert lib.moe_quantize_int4(fake + 4, 4, 256, 128, fake, fake, None) == S.INVALID_ARG
@@ -88,7 +91,13 @@ def test_workspace_size_and_layer_checks(lib):
     assert 0 < n16 < n64 and n16 % 256 == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(D=200)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(k=5)), 16) == 0
-    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=64)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=16)), 16) == 0
+    # groups of 64 / 32 run on the tensor-core tiles only: AUTO sizes that
+    # path's workspace, and a forced weight-streaming path is refused
+    g64 = _desc(group_size=64)
+    pre = _desc(path=moe.PATH_PREFILL)
+    assert lib.moe_ffn_workspace_size(ctypes.byref(g64), 16) == lib.moe_ffn_workspace_size(ctypes.byref(pre), 16)
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=32)), 16) > 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(w_up=None)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(d), 0) == 0
 
@@ -107,6 +116,18 @@ def test_forward_rejects_small_workspace_and_bad_pointers(lib):
     assert lib.moe_ffn_device_status(None, None) == S.INVALID_ARG
     ev = (ctypes.c_void_p * 2)(f, f)
     assert lib.moe_ffn_forward_timed(ctypes.byref(d), f, 16, f, f, need, None, ev, 2) == S.INVALID_ARG
+
+
+def test_small_groups_refuse_the_weight_streaming_path(lib):
+    S = moe.Status
+    f = 1 << 20
+    d = _desc(group_size=64, path=moe.PATH_DECODE)
+    need = lib.moe_ffn_workspace_size(ctypes.byref(d), 16)
+    assert need > 0
+    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f, need, None) == S.UNSUPPORTED_SHAPE
+    names = (ctypes.c_char_p * 16)()
+    n = lib.moe_ffn_launch_names(ctypes.byref(_desc(group_size=32)), 16, names, 16)
+    assert "tc_gate_up" in [names[i].decode() for i in range(n)]
 
 
 def test_launch_names(lib):

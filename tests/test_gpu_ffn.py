@@ -112,6 +112,20 @@ def test_skewed_full_size_sampled():
     assert rel_err(got, ref) <= TOL
 
 
+@pytest.mark.parametrize("G", [64, 32])
+@pytest.mark.parametrize("T,D,F,Fs,E,k", [(64, 256, 512, 512, 4, 1), (37, 384, 640, 384, 5, 2),
+                                          (300, 256, 256, 128, 3, 2), (1, 256, 512, 512, 4, 1)])
+def test_small_int4_groups(T, D, F, Fs, E, k, G):
+    """int4 experts quantized in groups of 64 or 32 (AUTO runs them on the
+    tensor-core tiles; the weight-streaming kernels refuse them)."""
+    b = build(synth.LayerShape("g%d" % G, T, D, F, E, k, Fs), group_size=G)
+    got, ref = _run(b, moe.PATH_AUTO)
+    assert rel_err(got, ref) <= TOL
+    b.gpu.set_path(moe.PATH_DECODE)
+    with pytest.raises(moe.MoEError):
+        b.gpu(b.x.cuda())
+
+
 FP8_SHAPES = [
     synth.LayerShape("fp8_tiny", 64, 256, 512, 8, 2, 256, "fp8"),
     synth.LayerShape("fp8_ragged", 37, 384, 640, 5, 3, 384, "fp8"),

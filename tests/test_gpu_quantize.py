@@ -27,6 +27,36 @@ def test_int4_bit_exact(rows, cols):
     assert np.array_equal(codes.cpu().numpy(), oq.pack_int4(q_ref))
 
 
+@pytest.mark.parametrize("G", [64, 32])
+@pytest.mark.parametrize("rows,cols", [(1, 128), (37, 512), (130, 5120)])
+def test_int4_small_groups_bit_exact(rows, cols, G):
+    """Groups of 64 and 32 (the smaller group_size the lshu.cn page names as
+    the int4 path's next step): codes and scales bit-exact."""
+    g = synth.stream(13, rows * 7 + cols + G)
+    w = (g.standard_normal((rows, cols), dtype=np.float32) * np.float32(0.02))
+    w[0, :G] = 0.0                                        # all-zero group
+    w[0, G:2 * G] = np.linspace(-1, 1, G, dtype=np.float32)
+    codes, scales = moe.quantize_int4(torch.from_numpy(w).cuda(), group_size=G)
+    q_ref, s_ref = oq.int4_row_quantize(w, group_size=G)
+    assert scales.shape == (rows, cols // G)
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy(), oq.pack_int4(q_ref))
+
+
+def test_int4_small_groups_worked_example_on_gpu():
+    """The hand-worked row of tests/golden/int4_small_groups_worked_example.txt
+    (padded to 128 columns with zeros) on the GPU quantizer."""
+    row = np.zeros((1, 128), np.float32)
+    idx = [0, 1, 3, 5, 33, 34, 40, 41, 42, 63]
+    row[0, idx] = [0.3125, 0.4375, 1.0, -0.1875, 0.15625, 0.21875, -0.5, 0.46875, -0.03125, 0.09375]
+    expect = {32: [2, 4, 7, -2, 2, 4, -8, 7, 0, 2], 64: [2, 4, 7, -2, 1, 2, -4, 4, 0, 1]}
+    for G in (32, 64):
+        codes, scales = moe.quantize_int4(torch.from_numpy(row).cuda(), group_size=G)
+        q = oq.unpack_int4(codes.cpu().numpy())
+        assert q[0, idx].tolist() == expect[G]
+        assert scales.cpu().numpy()[0, :64 // G].tolist() == ([0.125, 0.0625] if G == 32 else [0.125])
+
+
 def _near_tie_groups(n_groups, seed):
     """Groups whose quotients w / s sit on or within a few ulps of a
     half-integer (the places where a quotient one ulp off would round the

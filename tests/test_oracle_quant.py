@@ -44,17 +44,52 @@ def test_int4_worked_example():
     assert (codes[0, rest] == 0).all()
 
 
-def test_int4_brute_force_nearest_code():
+def _load_small_groups_example():
+    idx, w, q32, q64, sc = [], [], [], [], {}
+    with open(os.path.join(GOLDEN, "int4_small_groups_worked_example.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            parts = line.split()
+            if parts[0].startswith("scales"):
+                sc[int(parts[0][6:])] = [float(v) for v in parts[1:]]
+                continue
+            idx.append(int(parts[0]))
+            w.append(float(parts[1]))
+            q32.append(int(parts[2]))
+            q64.append(int(parts[3]))
+    return idx, w, {32: q32, 64: q64}, sc
+
+
+@pytest.mark.parametrize("G", [32, 64])
+def test_int4_small_groups_worked_example(G):
+    idx, w, q, sc = _load_small_groups_example()
+    row = np.zeros(64, np.float32)
+    row[idx] = w
+    codes, scales = quant.int4_row_quantize(row[None, :], group_size=G)
+    assert scales.shape == (1, 64 // G)
+    assert scales[0].tolist() == sc[G]
+    assert codes[0, idx].tolist() == q[G]
+    rest = np.setdiff1d(np.arange(64), idx)
+    assert (codes[0, rest] == 0).all()
+    # dequantization repeats each group's scale over exactly its G values
+    wh = quant.dequant_int4(codes, scales, group_size=G)
+    assert wh[0, 40] == q[G][idx.index(40)] * sc[G][40 // G]
+
+
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_int4_brute_force_nearest_code(G):
     """q must be the code in [-8, 7] nearest to fl32(w / s), ties to even."""
     rng = np.random.default_rng(1)
     w = (rng.standard_normal((6, 256)) * rng.uniform(1e-4, 3, (6, 1))).astype(np.float32)
     w[0, :128] = 0.0                         # an all-zero group
     w[1, 5] = 7.5 * np.abs(w[1, :128]).max() / 8  # exactly x.5 quotients occur below
-    q, s = quant.int4_row_quantize(w)
+    q, s = quant.int4_row_quantize(w, group_size=G)
     cand = np.arange(-8, 8, dtype=np.float64)
     for r in range(w.shape[0]):
         for c in range(w.shape[1]):
-            sc = s[r, c // 128]
+            sc = s[r, c // G]
             v = float(np.float32(w[r, c]) / np.float32(sc))
             d = np.abs(v - cand)
             best = np.flatnonzero(d == d.min())
@@ -63,17 +98,18 @@ def test_int4_brute_force_nearest_code():
             assert q[r, c] == int(cand[best[0]]), (r, c, v)
 
 
-def test_int4_invariants():
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_int4_invariants(G):
     rng = np.random.default_rng(2)
     w = (rng.standard_normal((32, 512)) * 0.02).astype(np.float32)
-    q, s = quant.int4_row_quantize(w)
+    q, s = quant.int4_row_quantize(w, group_size=G)
     assert q.dtype == np.int8 and q.min() >= -8 and q.max() <= 7
-    groups = w.reshape(-1, 128)
+    groups = w.reshape(-1, G)
     sg = s.reshape(-1)
     amax = np.abs(groups).max(axis=1)
     # scale * 8 recovers max(amax, 1e-6) exactly (division by 8 is exact)
     assert (sg * np.float32(8) == np.maximum(amax, np.float32(1e-6))).all()
-    qg = q.reshape(-1, 128)
+    qg = q.reshape(-1, G)
     for g in range(groups.shape[0]):
         i = np.argmax(np.abs(groups[g]))
         if groups[g, i] > 0:
@@ -81,7 +117,7 @@ def test_int4_invariants():
         else:
             assert qg[g, i] == -8                    # w/s = -8 exactly, no error
     # round trip: error <= s/2 while w/s < 7.5, else <= w - 7 s (<= s)
-    wh = quant.dequant_int4(q, s).reshape(-1, 128)
+    wh = quant.dequant_int4(q, s, group_size=G).reshape(-1, G)
     err = np.abs(groups.astype(np.float64) - wh)
     ratio = groups.astype(np.float64) / sg[:, None].astype(np.float64)
     lim = np.where(ratio < 7.5, sg[:, None] / 2.0, groups - 7.0 * sg[:, None])
