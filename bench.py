@@ -220,7 +220,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device, group: int = 128):
+def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device, group: int = 128, rms: bool = False):
     import int4_quantized_expert_b200 as moe
     E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
     wr = synth.router_weight(seed, E, D).to(dev)
@@ -237,6 +237,7 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device, group: in
                                torch.empty(E, n, dtype=torch.float32, device=dev))
         quant = lambda w, out: moe.quantize_fp8_rows(w, out=out)
         fmt = moe.FMT_FP8
+    gamma = synth.rms_weight(seed, D).to(dev) if rms else None
     gate, up, down = alloc(F, D), alloc(F, D), alloc(D, F)
     # Routed experts: N(0, 0.02) fp32 drawn on the device by torch's seeded
     # Philox generator (the same distribution as the parity tests' PCG64
@@ -254,9 +255,10 @@ def build_layer(shape: synth.LayerShape, seed: int, dev: torch.device, group: in
     del wbuf
     torch.cuda.synchronize()
     layer = moe.MoELayer(E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr, router_bias=bias, gate=gate,
-                         up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T, group_size=group)
+                         up=up, down=down, shared=(sg, su, sd), fmt=fmt, T_max=shape.T, group_size=group,
+                         rms_weight=gamma, rms_eps=1e-5)
     x = synth.tokens(seed, shape.T, D).to(dev)
-    return layer, x, (wr, bias)
+    return layer, x, (wr, bias, gamma)
 
 
 def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> dict:
@@ -273,6 +275,7 @@ def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> di
     scales_d = D * (F // group) * 4
     if shape.fmt == "fp8":   # e4m3 routed experts: one tensor-core pass each, bf16-equivalent flop count
         return {
+            "rmsnorm": ("bytes", T * D * 2 * 2 + D * 2),
             "router": ("flops", 2 * T * D * E),
             "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
             "quantize_x": ("bytes", T * D * 2 + S * D),
@@ -284,6 +287,7 @@ def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> di
             "combine": ("bytes", (S + T) * D * 4 + T * D * 2),
         }
     return {
+        "rmsnorm": ("bytes", T * D * 2 * 2 + D * 2),
         "router": ("flops", 2 * T * D * E),
         "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
         "act16_x": ("bytes", T * D * 2 * 2),
@@ -309,8 +313,9 @@ def layer_flops(shape: synth.LayerShape) -> int:
 def run_ours(args, rank: int, world: int, dev: torch.device):
     import int4_quantized_expert_b200 as moe
     shape = synth.SHAPES[args.workload]
-    layer, x, (wr, bias) = build_layer(shape, args.seed + 0, dev, args.group_size)
-    r = moe.route(x, wr, bias, shape.k)
+    layer, x, (wr, bias, gamma) = build_layer(shape, args.seed + 0, dev, args.group_size, args.rmsnorm)
+    # the experts the layer's routing touches (it routes RMSNorm(x) when the layer has the norm)
+    r = moe.route(x if gamma is None else moe.rmsnorm(x, gamma, 1e-5), wr, bias, shape.k)
     n_touched = int((r["counts"] > 0).sum().item())
     names = layer.launch_names(shape.T)
     out = torch.empty(shape.T, shape.D, dtype=torch.bfloat16, device=dev)
@@ -424,7 +429,8 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
         "data": ("synthetic (seeded; no dataset, random-init weights of the stated shapes: x, router and "
                  "shared expert from PCG64, routed experts N(0, 0.02) from torch's device generator)"),
         "config": {
-            "workload": workload_text(shape, args.group_size),
+            "workload": workload_text(shape, args.group_size) + (
+                ", RMSNorm (eps 1e-5) of x in front" if args.rmsnorm else ""),
             "weights": weights_text(shape, args.group_size),
             "parallelism": "replicas" if world > 1 else "single GPU",
             "experts_touched": n_touched,
@@ -680,6 +686,8 @@ def main(argv=None):
                              "quantize"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rmsnorm", action="store_true",
+                    help="run the layer with its RMSNorm prologue (gamma ~ 1 + N(0, 0.1), eps 1e-5)")
     ap.add_argument("--group-size", type=int, default=128, choices=[128, 64, 32],
                     help="int4 group size of the routed experts (and of the quantize workload)")
     args = ap.parse_args(argv)

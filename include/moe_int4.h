@@ -14,7 +14,8 @@
  *        equal to zero; activations stay bf16; a smaller group_size named as
  *        the int4 path's likely next step).
  *   [P5] "Llama 开源模型系列" (docs.ifdog.com): "MoE 架构详解" (router =
- *        linear layer, top-1 of 16 / top-8 of 128) and "SwiGLU：门控激活的数学".
+ *        linear layer, top-1 of 16 / top-8 of 128), "SwiGLU：门控激活的数学"
+ *        and "RMSNorm：为什么去掉减均值也能工作" (the block's normalization).
  *
  * Conventions for every entry point:
  *   - Pointers named as device pointers must point to device memory of the
@@ -165,7 +166,25 @@ typedef struct moe_layer_desc {
     const void* ws_gate;       /* bf16 [F_shared, D] */
     const void* ws_up;         /* bf16 [F_shared, D] */
     const void* ws_down;       /* bf16 [D, F_shared] */
+    /* Optional RMSNorm applied to x before everything else ([P5] "RMSNorm：
+     * 为什么去掉减均值也能工作"): x[t,:] -> bf16(x[t,:] / sqrt(mean(x[t,:]^2) +
+     * rms_eps) * rms_weight), as moe_rmsnorm computes it.  NULL: none. */
+    const void* rms_weight;    /* bf16 [D] (gamma), or NULL */
+    float rms_eps;             /* >= 0 (and <= 1); ignored when rms_weight is NULL */
 } moe_layer_desc;
+
+/*
+ * moe_rmsnorm -- RMSNorm ([P5] "RMSNorm：为什么去掉减均值也能工作"):
+ *   out[t, d] = bf16( x[t, d] / sqrt((1/D) sum_i x[t, i]^2 + eps) * gamma[d] )
+ * in fp32: the sum of squares in a fixed order, IEEE division and square
+ * root, the two products rounded to fp32 and the result to bf16 (nearest
+ * even).  The same kernel is the prologue of a layer with rms_weight set.
+ *   x      device, bf16 [T, D];  gamma  device, bf16 [D];  out  device, bf16 [T, D]
+ * Requires 1 <= T <= 1048576, D a multiple of 128 in [128, 16384],
+ * 0 <= eps <= 1.
+ */
+MOE_API moe_status moe_rmsnorm(const void* x, int32_t T, int32_t D, const void* gamma, float eps, void* out,
+                               void* stream);
 
 /*
  * Bytes of device workspace moe_ffn_forward needs for up to T_max tokens
@@ -180,6 +199,7 @@ MOE_API size_t moe_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max
 /*
  * moe_ffn_forward -- the whole layer ([P1] "混合专家路由", MoE.forward):
  *   out[t] = bf16( sum_j gate[t,j] * expert_{ids[t,j]}(x[t]) + shared(x[t]) )
+ *   (with layer->rms_weight set, x is first replaced by moe_rmsnorm(x)),
  *   expert_e(x) = (silu(x We_gate^T) * (x We_up^T)) We_down^T  ([P5] SwiGLU),
  *   with int4 (zero point 0) or FP8 row-wise weights ([P2] bmm_nt), fp32
  *   accumulation, and the hidden activation rounded to bf16.

@@ -17,7 +17,7 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "LIB_PATH", "lib", "MoEError", "Status", "LayerDesc", "quantize_int4", "quantize_fp8_rows",
+    "LIB_PATH", "lib", "MoEError", "Status", "LayerDesc", "quantize_int4", "quantize_fp8_rows", "rmsnorm",
     "route", "MoELayer", "FMT_INT4", "FMT_FP8", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
 ]
 
@@ -50,6 +50,7 @@ class LayerDesc(ctypes.Structure):
         ("w_down", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
         ("act_scale_ub", ctypes.c_float),
         ("ws_gate", ctypes.c_void_p), ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p),
+        ("rms_weight", ctypes.c_void_p), ("rms_eps", ctypes.c_float),
     ]
 
 
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_launch_names.restype = i32
         L.moe_ffn_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp]
         L.moe_ffn_forward_noalloc.restype = ctypes.c_int
+        L.moe_rmsnorm.argtypes = [vp, i32, i32, vp, f32, vp, vp]
+        L.moe_rmsnorm.restype = ctypes.c_int
         L.moe_ffn_device_status.argtypes = [vp, vp]
         L.moe_ffn_device_status.restype = ctypes.c_int
         _lib = L
@@ -159,6 +162,17 @@ def quantize_fp8_rows(x: torch.Tensor, num_valid_rows: Optional[int] = None,
     return q, s
 
 
+def rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float, stream=None, out=None) -> torch.Tensor:
+    """RMSNorm of bf16 ``x[T, D]`` with bf16 ``gamma[D]`` (see ``moe_rmsnorm``)."""
+    if x.dtype != torch.bfloat16 or gamma.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor and gamma bf16")
+    T, D = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _check("moe_rmsnorm", lib().moe_rmsnorm(_ptr(x), T, D, _ptr(gamma), ctypes.c_float(eps), _ptr(out),
+                                            _stream(stream)))
+    return out
+
+
 def route(x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Tensor], k: int, stream=None) -> dict:
     """Router + top-k + gate + bucketing (see ``moe_route``)."""
     T, D = x.shape
@@ -187,8 +201,8 @@ class MoELayer:
     def __init__(self, *, E: int, k: int, D: int, F: int, F_shared: int, w_router: torch.Tensor,
                  router_bias: Optional[torch.Tensor], gate, up, down, shared, fmt: int = FMT_INT4,
                  act_scale_ub: float = math.inf, T_max: int = 16, path: int = PATH_AUTO,
-                 group_size: int = 128):
-        self.tensors = [w_router, router_bias, *gate, *up, *down, *shared]   # keep alive
+                 group_size: int = 128, rms_weight: Optional[torch.Tensor] = None, rms_eps: float = 1e-5):
+        self.tensors = [w_router, router_bias, *gate, *up, *down, *shared, rms_weight]   # keep alive
         d = LayerDesc()
         d.E, d.k, d.D, d.F, d.F_shared = E, k, D, F, F_shared
         d.format, d.group_size, d.path = fmt, group_size, path
@@ -198,6 +212,7 @@ class MoELayer:
         d.w_down, d.s_down = _ptr(down[0]), _ptr(down[1])
         d.act_scale_ub = act_scale_ub
         d.ws_gate, d.ws_up, d.ws_down = (_ptr(t) for t in shared)
+        d.rms_weight, d.rms_eps = _ptr(rms_weight), rms_eps
         self.desc = d
         self.D = D
         self.device = w_router.device

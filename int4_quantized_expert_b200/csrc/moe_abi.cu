@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "ffn_decode.cuh"
 #include "tc_gemm.cuh"
+#include "norm.cuh"
 
 namespace moe {
 moe_status launch_quantize_int4(const float* w, int64_t rows, int64_t cols, int group_size, uint8_t* codes,
@@ -41,6 +42,7 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
 // workspace must be large enough for either.
 struct WsLayout {
     size_t status, rt_cnt, zeros_end, counters, rt_part, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t xn;   // RMSNorm of x (layers with rms_weight)
     size_t common_end;
     // weight-streaming path
     size_t x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
@@ -82,6 +84,7 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.inv_perm = take(S * 4);
     w.chunks = take(size_t(decode_max_chunks(int(T), L.k, L.E)) * sizeof(ChunkEntry));
     w.nchunks = take(16);
+    w.xn = take(L.rms_weight ? size_t(T) * L.D * 2 : 0);
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
         w.x16 = take(S * L.D * 2);                 // tokens by expert-sorted position
@@ -157,6 +160,8 @@ moe_status check_layer(const moe_layer_desc* L) {
     for (const void* p : ptrs)
         if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
     if (L->router_bias && !aligned16(L->router_bias)) return MOE_ERR_INVALID_ARG;
+    if (L->rms_weight && (!aligned16(L->rms_weight) || !(L->rms_eps >= 0.0f) || L->rms_eps > 1.0f))
+        return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -363,6 +368,21 @@ int prefill_launches(const moe_layer_desc& L, const char** names, int max_names)
     return n;
 }
 
+// The kernels one forward launches, in order: the RMSNorm (if the layer has
+// one), then the path's kernels.
+int32_t layer_launch_names(const moe_layer_desc& L, int64_t T, const char** names, int32_t max_names) {
+    int32_t n = 0;
+    if (L.rms_weight) {
+        if (names && max_names > 0) names[0] = "rmsnorm";
+        n = 1;
+    }
+    const char** rest = (names && max_names > n) ? names + n : nullptr;
+    const int32_t max_rest = max_names > n ? max_names - n : 0;
+    if (choose_path(L, T) != PATH_SEL_DECODE) return n + prefill_launches(L, rest, max_rest);
+    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_rest && rest; ++i) rest[i] = kDecodeLaunches[i];
+    return n + kDecodeLaunchCount;
+}
+
 moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
                             const WsLayout& W, cudaStream_t st, Marks& mk) {
     int32_t* status = at<int32_t>(ws, W.status);
@@ -520,9 +540,17 @@ moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t 
     // the device status word and the zero rows read in place of missing tokens
     if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
         return MOE_ERR_CUDA;
+    const bf16* xin = static_cast<const bf16*>(x);
+    if (layer->rms_weight) {   // the block's RMSNorm first; the layer reads its result
+        mk.mark(st);
+        s = launch_rmsnorm(xin, T, layer->D, static_cast<const bf16*>(layer->rms_weight), layer->rms_eps,
+                           at<bf16>(workspace, W.xn), st);
+        if (s != MOE_OK) return s;
+        xin = at<bf16>(workspace, W.xn);
+    }
     if (path == PATH_SEL_DECODE)
-        return ffn_decode_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
-    return ffn_prefill_path(*layer, static_cast<const bf16*>(x), T, static_cast<bf16*>(out), workspace, W, st, mk);
+        return ffn_decode_path(*layer, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
+    return ffn_prefill_path(*layer, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
 }
 
 }  // namespace
@@ -541,7 +569,7 @@ const char* moe_status_string(moe_status status) {
     return "unknown status";
 }
 
-int32_t moe_abi_version(void) { return 1; }
+int32_t moe_abi_version(void) { return 2; }
 
 moe_status moe_quantize_int4(const float* w, int64_t rows, int64_t cols, int32_t group_size, uint8_t* codes,
                              float* scales, void* stream) {
@@ -614,8 +642,7 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
                                  void* workspace, size_t workspace_bytes, void* stream, void* const* events,
                                  int32_t n_events) {
     if (!layer) return MOE_ERR_INVALID_ARG;
-    const int32_t need = choose_path(*layer, T) == PATH_SEL_DECODE ? kDecodeLaunchCount
-                                                                   : prefill_launches(*layer, nullptr, 0);
+    const int32_t need = layer_launch_names(*layer, T, nullptr, 0);
     if (!events || n_events < need + 1) return MOE_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_events; ++i)
         if (!events[i]) return MOE_ERR_INVALID_ARG;
@@ -627,9 +654,16 @@ moe_status moe_ffn_forward_timed(const moe_layer_desc* layer, const void* x, int
 
 int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, const char** names, int32_t max_names) {
     if (check_layer(layer) != MOE_OK || T < 1) return 0;
-    if (choose_path(*layer, T) != PATH_SEL_DECODE) return prefill_launches(*layer, names, max_names);
-    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
-    return kDecodeLaunchCount;
+    return layer_launch_names(*layer, T, names, max_names);
+}
+
+moe_status moe_rmsnorm(const void* x, int32_t T, int32_t D, const void* gamma, float eps, void* out,
+                       void* stream) {
+    if (T < 1 || T > kMaxT || !valid_dim(D)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !gamma || !out || !aligned16(x) || !aligned16(gamma) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || eps > 1.0f) return MOE_ERR_INVALID_ARG;
+    return launch_rmsnorm(static_cast<const bf16*>(x), T, D, static_cast<const bf16*>(gamma), eps,
+                          static_cast<bf16*>(out), as_stream(stream));
 }
 
 moe_status moe_ffn_device_status(const void* workspace, void* stream) {

@@ -16,7 +16,8 @@ Sources (web pages; cited by title and section):
   [P4] "Llama" (illegalscreed.cn), introduction (16 experts; 128 routed + 1
        shared experts).
   [P5] "Llama 开源模型系列" (docs.ifdog.com), sections "MoE 架构详解" (router =
-       linear layer + softmax, top-1 / top-8) and "SwiGLU：门控激活的数学".
+       linear layer + softmax, top-1 / top-8), "SwiGLU：门控激活的数学" and
+       "RMSNorm：为什么去掉减均值也能工作".
 
 Where the pages are silent or ambiguous the oracle takes the readings listed in
 the design doc; every function states the reading it uses.
@@ -25,4 +26,4 @@ Parity status: every function here is pinned by CPU tests against worked
 examples, brute force, closed forms, library special cases or invariants
 (tests/test_oracle_*.py).  No function is "parity unpinned".
 """
-from . import quant, route, ffn  # noqa: F401
+from . import quant, route, ffn, norm  # noqa: F401

@@ -77,6 +77,8 @@ class Layer:
     shared: tuple
     act_scale_ub: float = float("inf")
     group_size: int = 128
+    rms_weight: object = None      # gamma [D] of an RMSNorm applied to x first, or None
+    rms_eps: float = 1e-5
 
     def expert_output(self, e: int, x_rows: np.ndarray) -> np.ndarray:
         """y = expert e applied to x_rows[n, D] (fp64 values of bf16 inputs)."""
@@ -104,9 +106,15 @@ def moe_forward(layer: Layer, x, tokens: Optional[Sequence[int]] = None) -> dict
     by their scores, back into their tokens -> plus the shared expert:
         out[t] = bf16( sum_j gate[t, j] * y_{ids[t, j]}(x[t]) + shared(x[t]) ).
     The routing is computed for the whole batch (it is per token anyway).
+    With ``layer.rms_weight`` set, x is first replaced by its RMSNorm
+    (norm.rmsnorm: the block's normalization in front of the FFN, [P5]
+    "RMSNorm：为什么去掉减均值也能工作"), rounded to bf16.
     Returns the routing dict plus ``out`` (fp64 values of the bf16 outputs,
     one row per selected token) and ``tokens``.
     """
+    if layer.rms_weight is not None:
+        from .norm import rmsnorm
+        x = rmsnorm(x, layer.rms_weight, layer.rms_eps)
     xf = _f64(x)
     r = route(x, layer.w_router, layer.bias, layer.k)
     T = xf.shape[0]
@@ -128,6 +136,9 @@ def moe_forward(layer: Layer, x, tokens: Optional[Sequence[int]] = None) -> dict
 def moe_forward_dense(layer: Layer, x, E: int) -> np.ndarray:
     """Brute force: every expert on every token, weighted by a gate vector
     that is zero off each token's top-k; must equal :func:`moe_forward`."""
+    if layer.rms_weight is not None:
+        from .norm import rmsnorm
+        x = rmsnorm(x, layer.rms_weight, layer.rms_eps)
     xf = _f64(x)
     r = route(x, layer.w_router, layer.bias, layer.k)
     T = xf.shape[0]

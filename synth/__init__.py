@@ -32,7 +32,7 @@ import torch
 
 __all__ = [
     "LayerShape", "SHAPES", "stream", "tokens", "router_weight", "router_bias",
-    "shared_weights", "expert_weights", "iter_expert_weights", "to_bf16",
+    "shared_weights", "expert_weights", "iter_expert_weights", "to_bf16", "rms_weight",
     "WEIGHT_STD",
 ]
 
@@ -79,7 +79,7 @@ SHAPES = {
 }
 
 # Stream ids.  Routed expert e uses ids 16 + 3e + {0: gate, 1: up, 2: down}.
-_X, _ROUTER, _SHARED_GATE, _SHARED_UP, _SHARED_DOWN = 0, 1, 2, 3, 4
+_X, _ROUTER, _SHARED_GATE, _SHARED_UP, _SHARED_DOWN, _RMS = 0, 1, 2, 3, 4, 5
 
 
 def _routed_stream_id(e: int, which: int) -> int:
@@ -128,6 +128,12 @@ def tokens(seed: int, T: int, D: int,
 def router_weight(seed: int, E: int, D: int) -> torch.Tensor:
     """W_r [E, D] bf16."""
     return to_bf16(_normal(stream(seed, _ROUTER), (E, D), WEIGHT_STD))
+
+
+def rms_weight(seed: int, D: int) -> torch.Tensor:
+    """gamma [D] bf16 of an RMSNorm in front of the layer: 1 + N(0, 0.1)
+    (trained norm weights sit around 1; the pages give no values)."""
+    return to_bf16(np.float32(1.0) + _normal(stream(seed, _RMS), (D,), 0.1))
 
 
 def router_bias(shape: LayerShape) -> Optional[np.ndarray]:

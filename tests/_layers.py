@@ -15,6 +15,7 @@ import int4_quantized_expert_b200 as moe
 import synth
 from oracle import ffn as offn
 from oracle import quant as oq
+from oracle import norm as onorm
 from oracle import route as oroute
 
 
@@ -28,21 +29,24 @@ class Built:
     bias: Optional[np.ndarray]
 
 
-def margin_tokens(shape: synth.LayerShape, w_router, bias, seed: int, margin: bool = True):
+def margin_tokens(shape: synth.LayerShape, w_router, bias, seed: int, margin: bool = True, gamma=None,
+                  eps: float = 1e-5):
     accept = None
     if margin:
         def accept(x):
-            return oroute.topk_margin_ok(oroute.router_logits(x, w_router, bias), shape.k)
+            xr = x if gamma is None else onorm.rmsnorm(x, gamma, eps)   # the router sees RMSNorm(x)
+            return oroute.topk_margin_ok(oroute.router_logits(xr, w_router, bias), shape.k)
     return synth.tokens(seed, shape.T, shape.D, accept=accept)
 
 
 def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int = moe.PATH_AUTO,
-          device: str = "cuda", group_size: int = 128) -> Built:
+          device: str = "cuda", group_size: int = 128, rms: bool = False, rms_eps: float = 1e-5) -> Built:
     E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
     wr = synth.router_weight(seed, E, D)
     bias = synth.router_bias(shape)
     sg, su, sd = synth.shared_weights(seed, D, Fs)
-    x = margin_tokens(shape, wr, bias, seed, margin)
+    gamma = synth.rms_weight(seed, D) if rms else None
+    x = margin_tokens(shape, wr, bias, seed, margin, gamma, rms_eps)
     dev = torch.device(device)
 
     if shape.fmt == "int4":
@@ -65,7 +69,8 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
         E=E, k=k, D=D, F=F, F_shared=Fs, w_router=wr.to(dev),
         router_bias=None if bias is None else torch.from_numpy(bias).to(dev),
         gate=gate, up=up, down=down, shared=(sg.to(dev), su.to(dev), sd.to(dev)),
-        fmt=fmt, T_max=shape.T, path=path, group_size=group_size)
+        fmt=fmt, T_max=shape.T, path=path, group_size=group_size,
+        rms_weight=None if gamma is None else gamma.to(dev), rms_eps=rms_eps)
 
     @functools.lru_cache(maxsize=4)
     def expert(e):
@@ -74,7 +79,8 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
             return tuple(oq.int4_row_quantize(w, group_size=group_size) for w in ws)
         return tuple(oq.fp8_row_quantize(w) for w in ws)
 
-    olayer = offn.Layer(shape.fmt, k, wr, bias, expert, (sg, su, sd), group_size=group_size)
+    olayer = offn.Layer(shape.fmt, k, wr, bias, expert, (sg, su, sd), group_size=group_size,
+                        rms_weight=gamma, rms_eps=rms_eps)
     return Built(shape, x, layer, olayer, wr, bias)
 
 

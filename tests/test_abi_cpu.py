@@ -26,13 +26,13 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 12
+    assert len(names) == 13
     for n in names:
         assert hasattr(lib, n), n
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     assert lib.moe_status_string(0) == b"ok"
     assert lib.moe_status_string(3) == b"workspace too small"
     assert lib.moe_status_string(99) == b"unknown status"
@@ -128,6 +128,27 @@ def test_small_groups_refuse_the_weight_streaming_path(lib):
     names = (ctypes.c_char_p * 16)()
     n = lib.moe_ffn_launch_names(ctypes.byref(_desc(group_size=32)), 16, names, 16)
     assert "tc_gate_up" in [names[i].decode() for i in range(n)]
+
+
+def test_rmsnorm_checks_and_layer_prologue(lib):
+    S = moe.Status
+    f = 1 << 20
+    assert lib.moe_rmsnorm(f, 0, 256, f, 1e-5, f, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_rmsnorm(f, 4, 200, f, 1e-5, f, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_rmsnorm(f, 4, 256, None, 1e-5, f, None) == S.INVALID_ARG
+    assert lib.moe_rmsnorm(f, 4, 256, f, -1.0, f, None) == S.INVALID_ARG
+    assert lib.moe_rmsnorm(f, 4, 256, f, float("nan"), f, None) == S.INVALID_ARG
+    # a layer with an RMSNorm: the norm is its first launch and needs T x D x 2 more bytes
+    plain, normed = _desc(), _desc(rms_weight=f, rms_eps=1e-5)
+    n0 = lib.moe_ffn_workspace_size(ctypes.byref(plain), 16)
+    n1 = lib.moe_ffn_workspace_size(ctypes.byref(normed), 16)
+    assert n1 >= n0 + 16 * 256 * 2
+    names = (ctypes.c_char_p * 16)()
+    n = lib.moe_ffn_launch_names(ctypes.byref(normed), 16, names, 16)
+    assert n == lib.moe_ffn_launch_names(ctypes.byref(plain), 16, None, 0) + 1
+    assert names[0] == b"rmsnorm" and names[1] == b"router"
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f, rms_eps=-1.0)), 16) == 0
+    assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f + 4, rms_eps=1e-5)), 16) == 0
 
 
 def test_launch_names(lib):
