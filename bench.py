@@ -458,6 +458,119 @@ def run_ours(args, rank: int, world: int, dev: torch.device):
 
 
 # ---------------------------------------------------------------------------
+# the dense SwiGLU layer (the FFN of the dense layers between the MoE layers)
+# ---------------------------------------------------------------------------
+DENSE_SHAPES = {   # (T, D, F): the pages give no dense-layer width; F = twice the expert d_ff
+    "dense_decode": (16, 5120, 16384),
+    "dense_prefill": (8192, 5120, 16384),
+}
+
+
+def run_dense(args, rank: int, world: int, dev: torch.device):
+    import int4_quantized_expert_b200 as moe
+    T, D, F = DENSE_SHAPES[args.workload]
+    g, u, d = (t.to(dev) for t in synth.shared_weights(args.seed, D, F))
+    gamma = synth.rms_weight(args.seed, D).to(dev) if args.rmsnorm else None
+    layer = moe.DenseLayer(D=D, F=F, w_gate=g, w_up=u, w_down=d, T_max=T, rms_weight=gamma)
+    x = synth.tokens(args.seed, T, D).to(dev)
+    out = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer(x, out)
+    torch.cuda.synchronize()
+    assert layer.device_status() == moe.Status.OK
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        layer(x, out)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.summary(t0, t1) if sampler else None
+    if sampler:
+        sampler.stop()
+    if layer.device_status() != moe.Status.OK:
+        raise RuntimeError("device status after the timed loop")
+    ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in evs]))], dev, world)[0]
+    # end to end: pinned host x in, host out, both copies inside the events
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e, e2e_ms = max(3, min(args.steps, 100)), 0.0
+    xd = torch.empty_like(x)
+    for i in range(n_e2e + 1):
+        flush.zero_()
+        e0.record(stream)
+        xd.copy_(xh, non_blocking=True)
+        layer(xd, out)
+        oh.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i > 0:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks([e2e_ms / n_e2e], dev, world)[0]
+    hbm_peak, tc_peak, peak_src = peaks()
+    wbytes = 3 * D * F * 2
+    if T <= 64:   # weight streaming: HBM-bound
+        amount = wbytes + T * D * 2 * 2
+        roof = {"bound": "hbm", "kernel": "dense layer (all launches)", "achieved": amount / (ms * 1e-3) / 1e9,
+                "peak": hbm_peak, "peak_source": peak_src + " copy bandwidth", "unit": "GB/s",
+                "traffic": None, "algorithmic_bytes": amount}
+    else:
+        amount = 2 * T * D * 3 * F
+        roof = {"bound": "tensor", "kernel": "dense layer (all launches)", "achieved": amount / (ms * 1e-3) / 1e12,
+                "peak": tc_peak, "peak_source": peak_src + " sustained dense bf16", "unit": "TFLOP/s",
+                "traffic": None, "algorithmic_flops": amount}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return {
+        "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 x and bf16 weights N(0, 0.02); no dataset)",
+        "config": {"workload": "%s: dense SwiGLU FFN layer, T=%d tokens, d_model=%d, d_ff=%d, bf16 weights%s"
+                               % (args.workload, T, D, F, ", RMSNorm (eps 1e-5) of x in front" if args.rmsnorm else ""),
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (256 MB write)"},
+        "roofline": roof,
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
+                "d2h_bytes_per_step": T * D * 2, "ms_per_step": e2e_ms},
+        "gpu_launches": (4 + (1 if args.rmsnorm else 0)) * args.steps,   # [rmsnorm,] prep, gate/up, down, combine
+        "clocks": clocks,
+    }
+
+
+def time_oracle_dense(workload: str, seed: int, budget_s: float, n_steps: int, rms: bool):
+    """The oracle's dense layer on single tokens, repeated to fill about
+    budget_s per step; returns (tokens/s, sample text, seconds per step)."""
+    from oracle import ffn as offn
+    T, D, F = DENSE_SHAPES[workload]
+    g, u, d = synth.shared_weights(seed, D, F)
+    g, u, d = (t.float().numpy().astype(np.float64) for t in (g, u, d))
+    gamma = synth.rms_weight(seed, D) if rms else None
+    x = synth.tokens(seed, min(T, 64), D)
+    t = time.perf_counter()
+    offn.dense_forward(x[:1], g, u, d, rms_weight=gamma)
+    c1 = max(time.perf_counter() - t, 1e-4)
+    n = int(max(1, min(x.shape[0], budget_s / c1)))
+    t = time.perf_counter()
+    for _ in range(n_steps):
+        for i in range(n):
+            offn.dense_forward(x[i:i + 1], g, u, d, rms_weight=gamma)
+    el = (time.perf_counter() - t) / max(n_steps, 1)
+    return n / el, "%d single tokens of %s per step (the full layer for each)" % (n, workload), el
+
+
+# ---------------------------------------------------------------------------
 # the quantize workload (int4_row_quantize of a 16-expert weight set)
 # ---------------------------------------------------------------------------
 def run_quantize(args, rank: int, world: int, dev: torch.device):
@@ -639,6 +752,20 @@ def time_oracle(shape: synth.LayerShape, seed: int, budget_s: float, n_steps: in
 
 def run_reference(args):
     budget = min(20.0, 150.0 / max(args.steps + args.warmup, 1))
+    if args.workload in DENSE_SHAPES:
+        v, sample, per_step = time_oracle_dense(args.workload, args.seed, budget, args.steps, args.rmsnorm)
+        T, D, F = DENSE_SHAPES[args.workload]
+        return {
+            "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded PCG64 x and bf16 weights N(0, 0.02); no dataset)",
+            "config": {"workload": "%s: dense SwiGLU FFN layer, T=%d, d_model=%d, d_ff=%d" % (args.workload, T, D, F),
+                       "parallelism": "CPU oracle on the host cores"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
     if args.workload == "quantize":
         v, sample, per_step = time_oracle_quantize(args.seed, budget, args.steps, args.warmup, args.group_size)
         return {
@@ -683,7 +810,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scout_decode",
                     choices=["tiny", "scout_decode", "scout_prefill", "skewed", "maverick_fp8", "maverick_fp8_e16",
-                             "quantize"])
+                             "quantize", "dense_decode", "dense_prefill"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rmsnorm", action="store_true",
@@ -712,7 +839,13 @@ def main(argv=None):
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    if args.workload == "quantize":
+    if args.workload in DENSE_SHAPES:
+        result = run_dense(args, rank, world, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, sample, _ = time_oracle_dense(args.workload, args.seed, 10.0, 1, args.rmsnorm)
+            result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
+                                      "sample": sample}
+    elif args.workload == "quantize":
         result = run_quantize(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             v, sample, _ = time_oracle_quantize(args.seed, budget_s=5.0, n_steps=2, n_warm=0, group=args.group_size)

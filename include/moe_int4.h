@@ -13,6 +13,8 @@
  *        activation quantization, or int4 group-128 weights with zero points
  *        equal to zero; activations stay bf16; a smaller group_size named as
  *        the int4 path's likely next step).
+ *   [P4] "Llama" (illegalscreed.cn): introduction (dense and MoE layers
+ *        alternate; 16 routed experts, 128 routed + 1 shared).
  *   [P5] "Llama 开源模型系列" (docs.ifdog.com): "MoE 架构详解" (router =
  *        linear layer, top-1 of 16 / top-8 of 128), "SwiGLU：门控激活的数学"
  *        and "RMSNorm：为什么去掉减均值也能工作" (the block's normalization).
@@ -267,6 +269,45 @@ MOE_API int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, con
  */
 MOE_API moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
                                            void* stream);
+
+/*
+ * Description of a dense SwiGLU FFN layer, the FFN of the dense layers that
+ * alternate with the MoE layers ([P4] introduction; [P5] "SwiGLU：门控激活的
+ * 数学").  All pointers are device pointers.
+ *   w_gate, w_up bf16 [F, D]; w_down bf16 [D, F].
+ *   path: a moe_path; AUTO streams the weights (DECODE) for T <= 64 and
+ *         uses the tensor-core tiles (PREFILL) above.
+ *   rms_weight / rms_eps: as in moe_layer_desc (an RMSNorm of x first; NULL: none).
+ */
+typedef struct moe_dense_desc {
+    int32_t D, F;
+    int32_t path;              /* moe_path */
+    const void* w_gate;        /* bf16 [F, D] */
+    const void* w_up;          /* bf16 [F, D] */
+    const void* w_down;        /* bf16 [D, F] */
+    const void* rms_weight;    /* bf16 [D], or NULL */
+    float rms_eps;
+} moe_dense_desc;
+
+/*
+ * Bytes of device workspace moe_dense_ffn_forward needs for up to T_max
+ * tokens (0 if the description is invalid); with AUTO, the larger of the
+ * two paths' needs.
+ */
+MOE_API size_t moe_dense_ffn_workspace_size(const moe_dense_desc* layer, int32_t T_max);
+
+/*
+ * moe_dense_ffn_forward -- out = bf16( (silu(x Wg^T) * (x Wu^T)) Wd^T ) with
+ * bf16 weights, fp32 accumulation and the hidden activation rounded to bf16:
+ * the MoE layer's shared expert on its own ([P5] "SwiGLU：门控激活的数学").
+ *   x    device, bf16 [T, D];  out  device, bf16 [T, D] (may not alias x)
+ *   workspace  device, >= moe_dense_ffn_workspace_size(layer, T) bytes,
+ *              256-byte aligned; scratch between calls.
+ * Requires 1 <= T <= 1048576; D and F multiples of 128 in [128, 16384].
+ * No host synchronization.
+ */
+MOE_API moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const void* x, int32_t T, void* out,
+                                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * moe_ffn_device_status -- SYNCHRONIZES `stream`, then reads the device

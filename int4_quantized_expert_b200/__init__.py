@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "LIB_PATH", "lib", "MoEError", "Status", "LayerDesc", "quantize_int4", "quantize_fp8_rows", "rmsnorm",
-    "route", "MoELayer", "FMT_INT4", "FMT_FP8", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
+    "route", "MoELayer", "DenseDesc", "DenseLayer", "FMT_INT4", "FMT_FP8", "PATH_AUTO", "PATH_DECODE",
+    "PATH_PREFILL",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmoe_int4.so")
@@ -50,6 +51,15 @@ class LayerDesc(ctypes.Structure):
         ("w_down", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
         ("act_scale_ub", ctypes.c_float),
         ("ws_gate", ctypes.c_void_p), ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p),
+        ("rms_weight", ctypes.c_void_p), ("rms_eps", ctypes.c_float),
+    ]
+
+
+class DenseDesc(ctypes.Structure):
+    """Mirror of ``moe_dense_desc``."""
+    _fields_ = [
+        ("D", ctypes.c_int32), ("F", ctypes.c_int32), ("path", ctypes.c_int32),
+        ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
         ("rms_weight", ctypes.c_void_p), ("rms_eps", ctypes.c_float),
     ]
 
@@ -89,6 +99,10 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_launch_names.restype = i32
         L.moe_ffn_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp]
         L.moe_ffn_forward_noalloc.restype = ctypes.c_int
+        L.moe_dense_ffn_workspace_size.argtypes = [ctypes.POINTER(DenseDesc), i32]
+        L.moe_dense_ffn_workspace_size.restype = ctypes.c_size_t
+        L.moe_dense_ffn_forward.argtypes = [ctypes.POINTER(DenseDesc), vp, i32, vp, vp, ctypes.c_size_t, vp]
+        L.moe_dense_ffn_forward.restype = ctypes.c_int
         L.moe_rmsnorm.argtypes = [vp, i32, i32, vp, f32, vp, vp]
         L.moe_rmsnorm.restype = ctypes.c_int
         L.moe_ffn_device_status.argtypes = [vp, vp]
@@ -278,6 +292,63 @@ class MoELayer:
         _check("moe_ffn_forward_timed", lib().moe_ffn_forward_timed(
             ctypes.byref(self.desc), _ptr(x), T, _ptr(out), _ptr(self.workspace), self.workspace.numel(),
             _stream(stream), handles, len(events)))
+
+    def device_status(self, stream=None) -> int:
+        """Synchronizes the stream; the device status of the last forward."""
+        return lib().moe_ffn_device_status(_ptr(self.workspace), _stream(stream))
+
+
+class DenseLayer:
+    """A dense SwiGLU FFN layer (``moe_dense_ffn_forward``): bf16 weights
+    w_gate, w_up [F, D] and w_down [D, F], an optional RMSNorm of x first,
+    and a workspace for up to ``T_max`` tokens."""
+
+    def __init__(self, *, D: int, F: int, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                 path: int = PATH_AUTO, T_max: int = 16, rms_weight: Optional[torch.Tensor] = None,
+                 rms_eps: float = 1e-5):
+        self.tensors = [w_gate, w_up, w_down, rms_weight]   # keep alive
+        d = DenseDesc()
+        d.D, d.F, d.path = D, F, path
+        d.w_gate, d.w_up, d.w_down = _ptr(w_gate), _ptr(w_up), _ptr(w_down)
+        d.rms_weight, d.rms_eps = _ptr(rms_weight), rms_eps
+        self.desc = d
+        self.D = D
+        self.device = w_gate.device
+        self.workspace = None
+        self.T_max = 0
+        self.reserve(T_max)
+
+    def workspace_bytes(self, T: int) -> int:
+        n = lib().moe_dense_ffn_workspace_size(ctypes.byref(self.desc), T)
+        if n == 0:
+            raise MoEError("moe_dense_ffn_workspace_size", Status.UNSUPPORTED_SHAPE)
+        return n
+
+    def reserve(self, T_max: int) -> None:
+        if T_max <= self.T_max:
+            return
+        n = self.workspace_bytes(T_max)
+        if self.workspace is None or self.workspace.numel() < n:
+            self.workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
+        self.T_max = T_max
+
+    def set_path(self, path: int) -> None:
+        if path != self.desc.path:
+            self.desc.path = path
+            T_max, self.T_max = self.T_max, 0
+            self.reserve(T_max)
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        self.reserve(T)
+        if out is None:
+            out = torch.empty(T, self.D, dtype=torch.bfloat16, device=x.device)
+        _check("moe_dense_ffn_forward", lib().moe_dense_ffn_forward(
+            ctypes.byref(self.desc), _ptr(x), T, _ptr(out), _ptr(self.workspace), self.workspace.numel(),
+            _stream(stream)))
+        return out
+
+    __call__ = forward
 
     def device_status(self, stream=None) -> int:
         """Synchronizes the stream; the device status of the last forward."""

@@ -727,3 +727,236 @@ extern "C" moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const
     if (s != MOE_OK) return s;
     return ffn_forward_impl(layer, x, T, out, scratch, kNoAllocScratchBytes, as_stream(stream));
 }
+
+// ---------------------------------------------------------------------------
+// Dense SwiGLU FFN layer: the FFN of the dense layers that alternate with the
+// MoE layers ("Llama" (illegalscreed.cn), introduction: dense and MoE layers
+// alternate; "Llama 开源模型系列" (docs.ifdog.com), "SwiGLU：门控激活的数学"):
+//   out = bf16( (silu(x Wg^T) * (x Wu^T)) Wd^T ), bf16 weights, the hidden
+// activation rounded to bf16 -- the MoE layer's shared expert without the
+// routed experts.  It runs the shared-expert kernels of either path:
+//   weight streaming: [rmsnorm,] dense_prep, decode gate/up, decode down, combine
+//   tensor cores:     [rmsnorm,] dense_prep, copy to whole tiles, gate/up, down, combine
+// dense_prep writes the token chunk list the kernels take their tasks from.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int32_t kDenseDecodeMaxT = 64;   // AUTO streams the weights up to this many tokens
+
+struct DenseWs {
+    size_t status, counters, zeros_end, chunks, nchunks, xn;
+    size_t h, y;          // hidden [T(_pad), F] bf16, fp32 result [T, D]
+    size_t x_pad;         // tensor-core path: x in whole 256-row tiles
+    size_t total;
+};
+
+int dense_path(const moe_dense_desc& L, int64_t T) {
+    if (L.path == MOE_PATH_DECODE) return PATH_SEL_DECODE;
+    if (L.path == MOE_PATH_PREFILL) return PATH_SEL_PREFILL;
+    return T <= kDenseDecodeMaxT ? PATH_SEL_DECODE : PATH_SEL_PREFILL;
+}
+
+DenseWs dense_layout(const moe_dense_desc& L, int64_t T, int path) {
+    DenseWs w;
+    memset(&w, 0, sizeof(w));
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    const int64_t T_pad = ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
+    const int64_t rows = path == PATH_SEL_DECODE ? T : T_pad;
+    w.status = take(64);
+    w.counters = take(64);
+    w.zeros_end = off;
+    w.chunks = take(size_t(ceil_div(T, 16)) * sizeof(ChunkEntry));
+    w.nchunks = take(16);
+    w.xn = take(L.rms_weight ? size_t(T) * L.D * 2 : 0);
+    w.h = take(size_t(rows) * L.F * 2);
+    w.y = take(size_t(T) * L.D * 4);
+    w.x_pad = take(path == PATH_SEL_DECODE ? 0 : size_t(T_pad) * L.D * 2);
+    w.total = off;
+    return w;
+}
+
+moe_status check_dense(const moe_dense_desc* L) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    if (!valid_dim(L->D) || !valid_dim(L->F)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {L->w_gate, L->w_up, L->w_down};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (L->rms_weight && (!aligned16(L->rms_weight) || !(L->rms_eps >= 0.0f) || L->rms_eps > 1.0f))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// The chunk list of the shared-expert tasks: chunks of `ct` tokens; both
+// counts of the list header = the number of chunks (no routed chunks).
+__global__ void dense_prep_kernel(ChunkEntry* chunks, int32_t* n_chunks, int T, int ct) {
+    const int n = (T + ct - 1) / ct;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        ChunkEntry ce;
+        ce.expert = -1;
+        ce.start = i * ct;
+        ce.count = min(ct, T - i * ct);
+        ce.pad = 0;
+        chunks[i] = ce;
+    }
+    if (threadIdx.x == 0) { n_chunks[0] = n; n_chunks[1] = n; }
+}
+
+struct DenseKey {
+    moe_dense_desc L;
+    const void* ws;
+    const void* x;
+    int64_t T;
+    int path;
+    bool valid;
+};
+
+DenseKey dense_key(const moe_dense_desc& L, const void* ws, const void* x, int64_t T, int path) {
+    DenseKey k;
+    memset(&k, 0, sizeof(k));
+    memcpy(&k.L, &L, sizeof(L));
+    k.ws = ws;
+    k.x = x;
+    k.T = T;
+    k.path = path;
+    k.valid = true;
+    return k;
+}
+
+bool same_dense_key(const DenseKey& a, const DenseKey& b) {
+    return a.valid && b.valid && memcmp(&a.L, &b.L, sizeof(a.L)) == 0 && a.ws == b.ws && a.x == b.x &&
+           a.T == b.T && a.path == b.path;
+}
+
+moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_t T, void* out, void* ws,
+                              size_t ws_bytes, cudaStream_t st) {
+    moe_status s = check_dense(layer);
+    if (s != MOE_OK) return s;
+    const moe_dense_desc& L = *layer;
+    if (T < 1 || T > kMaxT) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !out || !ws || !aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return MOE_ERR_INVALID_ARG;
+    const int path = dense_path(L, T);
+    const DenseWs W = dense_layout(L, T, path);
+    if (ws_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (cudaMemsetAsync(at<int32_t>(ws, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const bf16* xin = static_cast<const bf16*>(x);
+    if (L.rms_weight) {
+        s = launch_rmsnorm(xin, T, L.D, static_cast<const bf16*>(L.rms_weight), L.rms_eps, at<bf16>(ws, W.xn), st);
+        if (s != MOE_OK) return s;
+        xin = at<bf16>(ws, W.xn);
+    }
+    ChunkEntry* chunks = at<ChunkEntry>(ws, W.chunks);
+    int32_t* nch = at<int32_t>(ws, W.nchunks);
+    int32_t* status = at<int32_t>(ws, W.status);
+    bf16* h = at<bf16>(ws, W.h);
+    float* y = at<float>(ws, W.y);
+    dense_prep_kernel<<<1, 256, 0, st>>>(chunks, nch, T, path == PATH_SEL_DECODE ? 16 : TC_BLOCK_TOKENS);
+    s = launch_status();
+    if (s != MOE_OK) return s;
+
+    if (path == PATH_SEL_DECODE) {
+        static thread_local DenseKey key_d;
+        static thread_local DecodeMaps m1, m2;
+        const DenseKey key = dense_key(L, ws, xin, T, path);
+        if (!same_dense_key(key, key_d)) {
+            key_d.valid = false;
+            const uint32_t rows = uint32_t(decode_task_rows());
+            bool ok = make_tmap_2d(&m1.s0, L.w_gate, 2, L.D, L.F, 64, rows, true) &&
+                      make_tmap_2d(&m1.s1, L.w_up, 2, L.D, L.F, 64, rows, true) &&
+                      make_tmap_rows_3d(&m1.bs, xin, L.D, T, 16, 1) &&
+                      make_tmap_2d(&m2.s0, L.w_down, 2, L.F, L.D, 64, rows, true) &&
+                      make_tmap_rows_3d(&m2.bs, h, L.F, T, 16, 2);
+            if (!ok) return MOE_ERR_CUDA;
+            // no routed tasks: the routed maps are never used; valid copies fill them
+            m1.r0 = m1.r1 = m1.g0 = m1.g1 = m1.s0;
+            m1.br = m1.cr = m1.bs;
+            m2.s1 = m2.r0 = m2.r1 = m2.g0 = m2.g1 = m2.s0;
+            m2.br = m2.cr = m2.bs;
+            key_d = key;
+        }
+        DecodeParams p;
+        memset(&p, 0, sizeof(p));
+        p.T = T;
+        p.n_rows_r = decode_task_rows();   // routed rows: unused (no routed chunks)
+        p.n_rows_s = L.F;
+        p.K_r = L.D;
+        p.K_s = L.D;
+        p.k_top = 1;
+        p.scale_buf_floats = 0;
+        p.f16_magic_lo = kF16MagicLo;
+        p.f16_magic_hi = kF16MagicHi;
+        p.chunks = chunks;
+        p.n_chunks = nch;
+        p.h_s = h;
+        p.task_counter = at<int32_t>(ws, W.counters);
+        p.status = status;
+        s = launch_decode_ffn(0, m1, p, st);
+        if (s != MOE_OK) return s;
+        p.n_rows_s = L.D;
+        p.K_r = L.F;
+        p.K_s = L.F;
+        p.y_s = y;
+        p.task_counter = at<int32_t>(ws, W.counters) + 1;
+        s = launch_decode_ffn(1, m2, p, st);
+        if (s != MOE_OK) return s;
+        return launch_combine(y, nullptr, nullptr, T, L.D, 0, static_cast<bf16*>(out), st);
+    }
+
+    const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
+    bf16* x_pad = at<bf16>(ws, W.x_pad);
+    static thread_local DenseKey key_p;
+    static thread_local TcMaps mg, md;
+    const DenseKey key = dense_key(L, ws, xin, T, path);
+    if (!same_dense_key(key, key_p)) {
+        key_p.valid = false;
+        bool ok = make_tmap_2d(&mg.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                  make_tmap_2d(&mg.a0, L.w_gate, 2, L.D, L.F, 64, 16, true) &&
+                  make_tmap_2d(&mg.a1, L.w_up, 2, L.D, L.F, 64, 16, true) &&
+                  make_tmap_2d(&md.b, h, 2, L.F, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                  make_tmap_2d(&md.a0, L.w_down, 2, L.F, L.D, 64, 16, true);
+        if (!ok) return MOE_ERR_CUDA;
+        md.a1 = md.a0;
+        key_p = key;
+    }
+    if (cudaMemcpyAsync(x_pad, xin, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.chunks = chunks;
+    p.n_chunks = nch;
+    p.k_top = 1;
+    p.group_shift = 7;
+    p.bf16_magic = kBf16Magic;
+    p.status = status;
+    p.K = L.D; p.n_rows = L.F; p.n_fblocks = L.F / 64; p.routed = 0;
+    p.h_out = h;
+    s = launch_tc_gemm(TC_GATEUP_BF16, mg, p, st);
+    if (s != MOE_OK) return s;
+    p.K = L.F; p.n_rows = L.D; p.n_fblocks = L.D / 128;
+    p.h_out = nullptr; p.y_out = y;
+    s = launch_tc_gemm(TC_DOWN_BF16, md, p, st);
+    if (s != MOE_OK) return s;
+    return launch_combine_slots(y, nullptr, T, L.D, 0, static_cast<bf16*>(out), st);
+}
+
+}  // namespace
+
+extern "C" size_t moe_dense_ffn_workspace_size(const moe_dense_desc* layer, int32_t T_max) {
+    if (check_dense(layer) != MOE_OK || T_max < 1 || T_max > kMaxT) return 0;
+    if (layer->path != MOE_PATH_AUTO) return dense_layout(*layer, T_max, dense_path(*layer, T_max)).total;
+    const size_t a = dense_layout(*layer, T_max, PATH_SEL_DECODE).total;
+    const size_t b = dense_layout(*layer, T_max, PATH_SEL_PREFILL).total;
+    return a > b ? a : b;
+}
+
+extern "C" moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const void* x, int32_t T, void* out,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+    return dense_forward_impl(layer, x, T, out, workspace, workspace_bytes, as_stream(stream));
+}

@@ -98,6 +98,18 @@ class Layer:
         return swiglu(x_rows, wg, wu, wd)
 
 
+def dense_forward(x, w_gate, w_up, w_down, rms_weight=None, rms_eps: float = 1e-5) -> np.ndarray:
+    """A dense SwiGLU FFN layer, the FFN of the dense layers that alternate
+    with the MoE layers ([P4] introduction; [P5] "SwiGLU：门控激活的数学"):
+    out = bf16(swiglu(x)) with bf16 weights -- the shared expert on its own.
+    With ``rms_weight``, x is first replaced by its RMSNorm (norm.rmsnorm).
+    Returns fp64 values of the bf16 outputs."""
+    if rms_weight is not None:
+        from .norm import rmsnorm
+        x = rmsnorm(x, rms_weight, rms_eps)
+    return bf16_round(swiglu(_f64(x), _f64(w_gate), _f64(w_up), _f64(w_down)))
+
+
 def moe_forward(layer: Layer, x, tokens: Optional[Sequence[int]] = None) -> dict:
     """The layer for all tokens, or for the listed ``tokens`` only.
 

@@ -26,7 +26,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 13
+    assert len(names) == 15
     for n in names:
         assert hasattr(lib, n), n
 
@@ -149,6 +149,26 @@ def test_rmsnorm_checks_and_layer_prologue(lib):
     assert names[0] == b"rmsnorm" and names[1] == b"router"
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f, rms_eps=-1.0)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f + 4, rms_eps=1e-5)), 16) == 0
+
+
+def test_dense_layer_checks(lib):
+    S = moe.Status
+    f = 1 << 20
+    d = moe.DenseDesc()
+    d.D, d.F, d.path = 256, 512, moe.PATH_AUTO
+    d.w_gate = d.w_up = d.w_down = f
+    d.rms_weight, d.rms_eps = None, 1e-5
+    n16 = lib.moe_dense_ffn_workspace_size(ctypes.byref(d), 16)
+    n512 = lib.moe_dense_ffn_workspace_size(ctypes.byref(d), 512)
+    assert 0 < n16 < n512 and n16 % 256 == 0
+    assert lib.moe_dense_ffn_forward(ctypes.byref(d), f, 16, f, f, 4096, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_dense_ffn_forward(ctypes.byref(d), f, 0, f, f, n16, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_dense_ffn_forward(ctypes.byref(d), None, 16, f, f, n16, None) == S.INVALID_ARG
+    assert lib.moe_dense_ffn_forward(None, f, 16, f, f, n16, None) == S.INVALID_ARG
+    d.F = 200
+    assert lib.moe_dense_ffn_workspace_size(ctypes.byref(d), 16) == 0
+    d.F, d.w_up = 512, None
+    assert lib.moe_dense_ffn_workspace_size(ctypes.byref(d), 16) == 0
 
 
 def test_launch_names(lib):
