@@ -311,8 +311,8 @@ MOE_API moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const void
 
 /*
  * moe_ffn_device_status -- SYNCHRONIZES `stream`, then reads the device
- * status word that the kernels of the last moe_ffn_forward on this workspace
- * set.  Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait gave up; the
+ * status word that the kernels of the last moe_ffn_forward (or
+ * moe_dense_ffn_forward) on this workspace set.  Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait gave up; the
  * outputs of that call are invalid) or MOE_ERR_CUDA.  The word is cleared at
  * the start of every moe_ffn_forward.
  */

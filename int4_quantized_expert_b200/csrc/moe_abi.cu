@@ -401,12 +401,7 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     float* y_pos = at<float>(ws, W.y_pos);
 
     RoutePrep prep;
-    memset(&prep, 0, sizeof(prep));
-    if (W.rt_cnt != W.zeros_end) {   // K-split router (few token tiles)
-        prep.router_part = at<float>(ws, W.rt_part);
-        prep.router_tile_cnt = at<int32_t>(ws, W.rt_cnt);
-    }
-    memset(&prep, 0, sizeof(prep));
+    memset(&prep, 0, sizeof(prep));   // unsplit router: the tensor-core path has many token tiles
     prep.chunks = chunks;
     prep.n_chunks = nch;
     prep.chunk_tokens = TC_BLOCK_TOKENS;
