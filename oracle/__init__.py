@@ -19,8 +19,8 @@ Sources (web pages; cited by title and section):
        linear layer + softmax, top-1 / top-8), "SwiGLU：门控激活的数学" and
        "RMSNorm：为什么去掉减均值也能工作".
 
-Where the pages are silent or ambiguous the oracle takes the readings listed in
-the design doc; every function states the reading it uses.
+Where the pages are silent or ambiguous the oracle takes a stated reading;
+every function states the reading it uses.
 
 Parity status: every function here is pinned by CPU tests against worked
 examples, brute force, closed forms, library special cases or invariants
