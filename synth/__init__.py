@@ -159,13 +159,16 @@ def expert_weights(seed: int, e: int, D: int, F: int):
 
 def iter_expert_weights(seed: int, experts: Sequence[int], D: int, F: int,
                         workers: Optional[int] = None,
-                        ahead: int = 2) -> Iterator[tuple]:
-    """Yield (e, W_gate, W_up, W_down) for each e, generated by a thread pool.
+                        ahead: Optional[int] = None) -> Iterator[tuple]:
+    """Yield (e, W_gate, W_up, W_down) for each e, generated by a thread pool
+    (numpy's generators release the GIL while they fill an array).
 
     At most ``ahead`` experts beyond the one being consumed are held in host
-    memory, so a 128-expert layer never needs all of its fp32 weights at once.
+    memory (by default enough to keep every worker busy), so a 128-expert
+    layer never needs all of its fp32 weights at once.
     """
-    workers = workers or min(8, os.cpu_count() or 1)
+    workers = workers or min(32, os.cpu_count() or 1)
+    ahead = ahead if ahead is not None else max(2, (workers + 2) // 3)
     experts = list(experts)
 
     def job(e, w):
