@@ -31,6 +31,32 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_header_compiles_and_links_as_plain_c(lib, tmp_path):
+    """The boundary is a C ABI: a strict C99 program includes the header,
+    links the library and calls it, with no Python or C++ involved."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "moe_int4.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        "    moe_layer_desc d; moe_dense_desc dd; (void)d; (void)dd;\n"
+        '    printf("%d %s\\n", moe_abi_version(), moe_status_string(MOE_ERR_TIMEOUT));\n'
+        "    return moe_quantize_int4(0, 0, 128, 128, 0, 0, 0) == MOE_OK ? 0 : 1;\n"
+        "}\n")
+    libdir = os.path.dirname(moe.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER), str(src),
+                        "-o", str(exe), "-L", libdir, "-lmoe_int4", "-Wl,-rpath," + libdir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "2 device wait timed out", (r.stdout, r.stderr)
+
+
 def test_version_and_status_strings(lib):
     assert lib.moe_abi_version() == 2
     assert lib.moe_status_string(0) == b"ok"
