@@ -3,8 +3,9 @@
 // The layer ("1 卡跑通 Llama 4" (discosf.com), "混合专家路由"; "Llama 开源模型
 // 系列" (docs.ifdog.com), "SwiGLU：门控激活的数学"): each expert runs
 // (silu(x Wg^T) * (x Wu^T)) Wd^T on its tokens; routed weights are int4 with
-// one fp32 scale per 128 K and zero point 0 ("Meta Llama Models Llama 4 单卡
-// 量化推理与选型指南" (lshu.cn), "量化环节做了什么"); the shared expert is bf16.
+// one fp32 scale per group of 128 K (or the smaller 64 / 32) and zero point 0
+// ("Meta Llama Models Llama 4 单卡量化推理与选型指南" (lshu.cn), "量化环节做了
+// 什么"), or e4m3 rows; the shared expert is bf16.
 //
 // One persistent CTA per SM, tiles of 128 output features x 256 tokens:
 //   A = weights (M = 128 rows), B = tokens (N = 256 rows), both K-major in
