@@ -1,6 +1,5 @@
 """Compile-time resources of the hot kernels (CPU only: nvcc cross-compiles
-for sm_100a): none of them may spill registers to local memory, and the
-weight-streaming and tensor-core kernels must fit one CTA per SM."""
+for sm_100a): none of them may spill registers to local memory."""
 import os
 import re
 import shutil
