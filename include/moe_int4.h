@@ -262,13 +262,27 @@ MOE_API int32_t moe_ffn_launch_names(const moe_layer_desc* layer, int32_t T, con
  * No cudaMalloc, cudaFree or other allocation is made.
  * The first call on each device looks up the array's device address with
  * that device current; make that first call before any stream capture.
+ * The address is kept for the life of the process: after cudaDeviceReset
+ * on a device, do not call this function on that device again (the array
+ * may have moved).
  * All calls on a device share the one array: calls that may overlap on the
  * GPU (different streams, or different host threads) race and corrupt each
  * other's results -- serialize them.  Leftover contents from an earlier call
  * are harmless; what must start at zero is cleared by every call.
+ * Argument errors (null or misaligned x / out, unsupported shapes) return
+ * before the CUDA runtime is touched.
  */
 MOE_API moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const void* x, int32_t T, void* out,
                                            void* stream);
+
+/*
+ * moe_ffn_noalloc_device_status -- moe_ffn_device_status for the calls of
+ * moe_ffn_forward_noalloc on the current device, whose status word lives in
+ * the library's own scratch array: SYNCHRONIZES `stream`, then returns MOE_OK,
+ * MOE_ERR_TIMEOUT (a bounded device wait of the last no-alloc call gave up;
+ * its output is invalid) or MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_ffn_noalloc_device_status(void* stream);
 
 /*
  * Description of a dense SwiGLU FFN layer, the FFN of the dense layers that
@@ -317,6 +331,19 @@ MOE_API moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const void
  * the start of every moe_ffn_forward.
  */
 MOE_API moe_status moe_ffn_device_status(const void* workspace, void* stream);
+
+/*
+ * moe_set_wait_limit -- the limit, in SM clock cycles, of every bounded
+ * device wait that reports to a status word (the kernels' waits on their
+ * pipeline barriers), for the current device.  cycles <= 0 restores the
+ * default of 2e9 cycles (about one second).  A lowered limit makes waits give
+ * up as soon as they miss their first try, so the next layer call ends with
+ * MOE_ERR_TIMEOUT in its status word: it exists to test that path.  Waits
+ * that let a kernel's own copies in flight land before it exits keep the
+ * default.  Synchronous; call it while no kernel of this library is running.
+ * The pages have no counterpart.
+ */
+MOE_API moe_status moe_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

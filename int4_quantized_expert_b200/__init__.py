@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LIB_PATH", "lib", "MoEError", "Status", "LayerDesc", "quantize_int4", "quantize_fp8_rows", "rmsnorm",
     "route", "MoELayer", "DenseDesc", "DenseLayer", "FMT_INT4", "FMT_FP8", "PATH_AUTO", "PATH_DECODE",
-    "PATH_PREFILL",
+    "PATH_PREFILL", "noalloc_device_status", "set_wait_limit",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmoe_int4.so")
@@ -99,6 +99,10 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_launch_names.restype = i32
         L.moe_ffn_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp]
         L.moe_ffn_forward_noalloc.restype = ctypes.c_int
+        L.moe_ffn_noalloc_device_status.argtypes = [vp]
+        L.moe_ffn_noalloc_device_status.restype = ctypes.c_int
+        L.moe_set_wait_limit.argtypes = [i64]
+        L.moe_set_wait_limit.restype = ctypes.c_int
         L.moe_dense_ffn_workspace_size.argtypes = [ctypes.POINTER(DenseDesc), i32]
         L.moe_dense_ffn_workspace_size.restype = ctypes.c_size_t
         L.moe_dense_ffn_forward.argtypes = [ctypes.POINTER(DenseDesc), vp, i32, vp, vp, ctypes.c_size_t, vp]
@@ -296,6 +300,26 @@ class MoELayer:
     def device_status(self, stream=None) -> int:
         """Synchronizes the stream; the device status of the last forward."""
         return lib().moe_ffn_device_status(_ptr(self.workspace), _stream(stream))
+
+    def forward_noalloc(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """forward() without the workspace: the library's own fixed scratch
+        (``moe_ffn_forward_noalloc``; decode-sized batches only)."""
+        if out is None:
+            out = torch.empty(x.shape[0], self.D, dtype=torch.bfloat16, device=x.device)
+        _check("moe_ffn_forward_noalloc", lib().moe_ffn_forward_noalloc(
+            ctypes.byref(self.desc), _ptr(x), x.shape[0], _ptr(out), _stream(stream)))
+        return out
+
+
+def noalloc_device_status(stream=None) -> int:
+    """Synchronizes the stream; the device status of the last no-alloc forward."""
+    return lib().moe_ffn_noalloc_device_status(_stream(stream))
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Limit of the kernels' bounded waits in SM cycles (<= 0: the default);
+    lowering it makes the next forward time out, to test that path."""
+    _check("moe_set_wait_limit", lib().moe_set_wait_limit(int(cycles)))
 
 
 class DenseLayer:

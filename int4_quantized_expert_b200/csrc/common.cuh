@@ -213,7 +213,14 @@ __device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f 
 // ---------------------------------------------------------------------------
 namespace moe {
 
-constexpr long long kWaitCycles = 2000000000LL;   // about one second at 1.9 GHz
+constexpr uint32_t kWaitCycles = 2000000000u;   // about one second at 1.9 GHz
+
+// The limit of the waits that report to a status word, in SM cycles.  It is
+// kWaitCycles unless a test lowers it (moe_set_wait_limit) to make waits run
+// out on purpose; waits that drain a CTA's own copies in flight (no status
+// word) always keep kWaitCycles.  Each translation unit that waits on
+// mbarriers has its own copy, set by set_wait_limit_<unit>().
+static __constant__ uint32_t c_wait_limit = kWaitCycles;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -262,18 +269,39 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
+// Non-blocking test of a phase (try_wait may suspend the thread for a while).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  The
 // device status word (another wait of this launch timed out) and the clock
-// are checked only every 64 sleeps, so a wait that misses its first try
-// costs no global-memory round trip.
+// are checked only every 64 sleeps, so a wait that misses its first try costs
+// no global-memory round trip.  With a lowered limit (tests) the waiter only
+// polls, without ever suspending, so the limit decides when it gives up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    if (status != nullptr && c_wait_limit != kWaitCycles) {
+        const uint32_t t0 = uint32_t(clock64());
+        for (;;) {
+            if (mbar_test_wait(bar, parity)) return true;
+            if (uint32_t(clock64()) - t0 > c_wait_limit) {
+                atomicExch(status, DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
     if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
+    const uint32_t t0 = uint32_t(clock64());   // 32-bit differences: the limit is below 2^32 cycles
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_sleep(bar, parity, 10000u)) return true;
         if ((i & 63u) == 0) {
             if (status && ld_volatile(status) != DEV_OK) return false;
-            if (clock64() - t0 > kWaitCycles) {
+            if (uint32_t(clock64()) - t0 > kWaitCycles) {
                 if (status) atomicExch(status, DEV_TIMEOUT);
                 return false;
             }

@@ -503,7 +503,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         }
         if (!ok) break;
 
-        // ---- sum the K phases (phases 1..2 hand their partial sums to phase 0) ----
+        // ---- sum the K phases (phases 1.. hand their partial sums to phase 0) ----
         if (q > 0) {
             if (!mbar_wait(&sm->red_empty, (tn & 1) ^ 1, p.status)) break;
             float* my = red + ((q - 1) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
@@ -515,14 +515,29 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             if (lane == 0) mbar_arrive(&sm->red_full);
         } else {
             if (!mbar_wait(&sm->red_full, tn & 1, p.status)) break;
+            // Phase qq holds the task's stages s with s % DC_KPH == (qq - it_base) % DC_KPH,
+            // which depends on the tasks this CTA ran before.  The partials are summed
+            // in the order of that residue, so every output has the same rounding
+            // whichever CTA computed it.
+            float t0[DC_NT][4], t1[DC_NT][4];
 #pragma unroll
-            for (int qq = 1; qq < DC_KPH; ++qq) {
-                const float* o = red + ((qq - 1) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
+            for (int rr = 0; rr < DC_KPH; ++rr) {
+                const int qq = int((uint32_t(rr) + it_base) % DC_KPH);   // the phase holding residue rr
+                const float* o = red + ((qq > 0 ? qq - 1 : 0) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
 #pragma unroll
                 for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) { acc0[nt][r] += o[nt * 8 + r]; acc1[nt][r] += o[nt * 8 + 4 + r]; }
+                    for (int r = 0; r < 4; ++r) {
+                        const float v0 = qq == 0 ? acc0[nt][r] : o[nt * 8 + r];
+                        const float v1 = qq == 0 ? acc1[nt][r] : o[nt * 8 + 4 + r];
+                        t0[nt][r] = rr == 0 ? v0 : t0[nt][r] + v0;
+                        t1[nt][r] = rr == 0 ? v1 : t1[nt][r] + v1;
+                    }
             }
+#pragma unroll
+            for (int nt = 0; nt < DC_NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) { acc0[nt][r] = t0[nt][r]; acc1[nt][r] = t1[nt][r]; }
             // ---- epilogue: C rows (row_a, row_b) x columns (2c, 2c + 1) of each n-tile,
             // column n of n-tile nt being token nt * 8 + sigma8(n) of the chunk ----
             // routed results are rescaled by their token row's power of two;
@@ -582,6 +597,11 @@ __global__ void combine_kernel(const float* __restrict__ y_s, const float* __res
         o.y = pack_bf16x2(a.z, a.w);
         *reinterpret_cast<uint2*>(out + t * D + d) = o;
     }
+}
+
+// This file's copy of the wait limit (see c_wait_limit).
+moe_status set_wait_limit_decode(uint32_t cycles) {
+    return cuda_status(cudaMemcpyToSymbol(c_wait_limit, &cycles, sizeof(cycles)));
 }
 
 // shared-expert chunks of 16 tokens, routed ones of 8 (at most one partial chunk per expert)

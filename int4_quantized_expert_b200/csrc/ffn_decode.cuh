@@ -92,4 +92,6 @@ moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* s
 moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
                           bf16* out, cudaStream_t stream);
 
+moe_status set_wait_limit_decode(uint32_t cycles);
+
 }  // namespace moe

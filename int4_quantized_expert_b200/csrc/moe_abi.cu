@@ -47,7 +47,7 @@ struct WsLayout {
     // weight-streaming path
     size_t x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
     // tensor-core path (row counts padded to whole 256-token tiles)
-    size_t x_sorted, h_sorted, x_pad, h_s_pad, y_pos, y_shared;
+    size_t x_sorted, h_sorted, h_s_pad, y_pos, y_shared;
     size_t xq, xq_scale, hq, hq_scale;   // e4m3 activations of FP8_ROW layers
     // host staging of moe_ffn_forward_host
     size_t x_in, out;
@@ -107,7 +107,6 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
             w.x_sorted = take(S_pad * L.D * 2);
         }
         w.h_sorted = take(S_pad * L.F * 2);
-        w.x_pad = take(T_pad * L.D * 2);
         w.h_s_pad = take(T_pad * L.F_shared * 2);
         w.y_pos = take(S * L.D * 4);
         w.y_shared = take(T * L.D * 4);
@@ -396,7 +395,6 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
     bf16* x_sorted = at<bf16>(ws, W.x_sorted);
     bf16* h_sorted = at<bf16>(ws, W.h_sorted);
-    bf16* x_pad = at<bf16>(ws, W.x_pad);
     bf16* h_s = at<bf16>(ws, W.h_s_pad);
     float* y_pos = at<float>(ws, W.y_pos);
 
@@ -421,9 +419,6 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     else
         s = launch_gather_rows(x, perm, S, L.k, L.D, x_sorted, st);
     if (s != MOE_OK) return s;
-    // the shared expert reads x through a 256-row tile map: copy it into whole tiles
-    if (cudaMemcpyAsync(x_pad, x, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
 
     static thread_local MapCacheKey pkey;
     static thread_local TcMaps pm[4];
@@ -445,7 +440,9 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
                  make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D / 2, E * L.F, 32, 64, false) &&
                  make_tmap_2d(&m_dn.b, h_sorted, 2, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
                  make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
-        ok = ok && make_tmap_2d(&m_sgu.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+        // the shared expert's token tiles come straight from x: a 256-row box that
+        // runs past row T - 1 reads zeros there
+        ok = ok && make_tmap_2d(&m_sgu.b, x, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
                   make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
@@ -683,7 +680,8 @@ moe_status moe_ffn_device_status(const void* workspace, void* stream) {
 // device asks the runtime for the real address, with that device current,
 // and remembers it.  Calls share the array and it keeps whatever the previous
 // call left; the layer path already clears what must start at zero (the
-// device status word and the task counters) on every call.
+// device status word and the task counters) on every call.  The status word
+// sits at the array's start, where moe_ffn_noalloc_device_status reads it.
 // ---------------------------------------------------------------------------
 namespace {
 
@@ -716,11 +714,28 @@ extern "C" moe_status moe_ffn_forward_noalloc(const moe_layer_desc* layer, const
     if (s != MOE_OK) return s;
     s = check_route_shape(T, layer->D, layer->E, layer->k);
     if (s != MOE_OK) return s;
+    // argument errors first: nothing below touches the CUDA runtime until they pass
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     if (ws_layout(*layer, T, choose_path(*layer, T)).total > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
     void* scratch = nullptr;
     s = noalloc_scratch_address(&scratch);
     if (s != MOE_OK) return s;
     return ffn_forward_impl(layer, x, T, out, scratch, kNoAllocScratchBytes, as_stream(stream));
+}
+
+extern "C" moe_status moe_ffn_noalloc_device_status(void* stream) {
+    void* scratch = nullptr;
+    moe_status s = noalloc_scratch_address(&scratch);
+    if (s != MOE_OK) return s;
+    return moe_ffn_device_status(scratch, stream);
+}
+
+extern "C" moe_status moe_set_wait_limit(int64_t cycles) {
+    // the default, or the caller's limit (at most the default)
+    const uint32_t c = cycles > 0 && cycles < int64_t(kWaitCycles) ? uint32_t(cycles) : kWaitCycles;
+    moe_status s = set_wait_limit_decode(c);
+    if (s != MOE_OK) return s;
+    return set_wait_limit_tc(c);
 }
 
 // ---------------------------------------------------------------------------
@@ -741,7 +756,6 @@ constexpr int32_t kDenseDecodeMaxT = 64;   // AUTO streams the weights up to thi
 struct DenseWs {
     size_t status, counters, zeros_end, chunks, nchunks, xn;
     size_t h, y;          // hidden [T(_pad), F] bf16, fp32 result [T, D]
-    size_t x_pad;         // tensor-core path: x in whole 256-row tiles
     size_t total;
 };
 
@@ -770,7 +784,6 @@ DenseWs dense_layout(const moe_dense_desc& L, int64_t T, int path) {
     w.xn = take(L.rms_weight ? size_t(T) * L.D * 2 : 0);
     w.h = take(size_t(rows) * L.F * 2);
     w.y = take(size_t(T) * L.D * 4);
-    w.x_pad = take(path == PATH_SEL_DECODE ? 0 : size_t(T_pad) * L.D * 2);
     w.total = off;
     return w;
 }
@@ -905,13 +918,12 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
     }
 
     const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
-    bf16* x_pad = at<bf16>(ws, W.x_pad);
     static thread_local DenseKey key_p;
     static thread_local TcMaps mg, md;
     const DenseKey key = dense_key(L, ws, xin, T, path);
     if (!same_dense_key(key, key_p)) {
         key_p.valid = false;
-        bool ok = make_tmap_2d(&mg.b, x_pad, 2, L.D, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+        bool ok = make_tmap_2d(&mg.b, xin, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
                   make_tmap_2d(&mg.a0, L.w_gate, 2, L.D, L.F, 64, 16, true) &&
                   make_tmap_2d(&mg.a1, L.w_up, 2, L.D, L.F, 64, 16, true) &&
                   make_tmap_2d(&md.b, h, 2, L.F, T_pad, 64, TC_BLOCK_TOKENS, true) &&
@@ -920,8 +932,6 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         md.a1 = md.a0;
         key_p = key;
     }
-    if (cudaMemcpyAsync(x_pad, xin, size_t(T) * L.D * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
     TcParams p;
     memset(&p, 0, sizeof(p));
     p.chunks = chunks;

@@ -527,6 +527,11 @@ moe_status launch_combine_slots(const float* y_s, const float* y, int64_t T, int
     return launch_status();
 }
 
+// This file's copy of the wait limit (see c_wait_limit).
+moe_status set_wait_limit_tc(uint32_t cycles) {
+    return cuda_status(cudaMemcpyToSymbol(c_wait_limit, &cycles, sizeof(cycles)));
+}
+
 size_t tc_smem_bytes() {
     return 1024 + size_t(TC_STAGES) * TC_STAGE_BYTES + size_t(TC_CSTAGES) * TC_C_BYTES + sizeof(TcSmem);
 }

@@ -59,4 +59,6 @@ moe_status launch_combine_slots(const float* y_s, const float* y, int64_t T, int
 moe_status launch_gather_rows(const bf16* x, const int32_t* perm, int64_t n, int k, int D, bf16* out,
                               cudaStream_t stream);
 
+moe_status set_wait_limit_tc(uint32_t cycles);
+
 }  // namespace moe

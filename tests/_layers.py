@@ -72,6 +72,19 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
         fmt=fmt, T_max=shape.T, path=path, group_size=group_size,
         rms_weight=None if gamma is None else gamma.to(dev), rms_eps=rms_eps)
 
+    olayer = oracle_layer(shape, seed, group_size, gamma, rms_eps)
+    return Built(shape, x, layer, olayer, wr, bias)
+
+
+def oracle_layer(shape: synth.LayerShape, seed: int = 0, group_size: int = 128, gamma=None,
+                 rms_eps: float = 1e-5) -> offn.Layer:
+    """The oracle's view of the layer ``build`` makes: the same seeded
+    router, shared and routed weights, the routed ones quantized by the oracle."""
+    E, k, D, F, Fs = shape.E, shape.k, shape.D, shape.F, shape.F_shared
+    wr = synth.router_weight(seed, E, D)
+    bias = synth.router_bias(shape)
+    shared = synth.shared_weights(seed, D, Fs)
+
     @functools.lru_cache(maxsize=4)
     def expert(e):
         ws = synth.expert_weights(seed, e, D, F)
@@ -79,9 +92,57 @@ def build(shape: synth.LayerShape, seed: int = 0, margin: bool = True, path: int
             return tuple(oq.int4_row_quantize(w, group_size=group_size) for w in ws)
         return tuple(oq.fp8_row_quantize(w) for w in ws)
 
-    olayer = offn.Layer(shape.fmt, k, wr, bias, expert, (sg, su, sd), group_size=group_size,
-                        rms_weight=gamma, rms_eps=rms_eps)
-    return Built(shape, x, layer, olayer, wr, bias)
+    return offn.Layer(shape.fmt, k, wr, bias, expert, shared, group_size=group_size,
+                      rms_weight=gamma, rms_eps=rms_eps)
+
+
+def covering_tokens(ids: np.ndarray, E: int, n_extra: int, seed: int) -> np.ndarray:
+    """Tokens to check at full size: for every expert that some token chose,
+    one (seeded, random) token that chose it -- taken greedily, so a token
+    covers all of its k experts -- plus ``n_extra`` more random tokens."""
+    rng = np.random.default_rng(seed)
+    T = ids.shape[0]
+    chosen, covered = [], set()
+    for e in rng.permutation(E):
+        if e in covered:
+            continue
+        cand = np.nonzero((ids == e).any(axis=1))[0]
+        if cand.size == 0:
+            continue
+        t = int(rng.choice(cand))
+        chosen.append(t)
+        covered.update(int(v) for v in ids[t])
+    rest = np.setdiff1d(np.arange(T), chosen)
+    extra = rng.choice(rest, min(n_extra, rest.size), replace=False)
+    return np.sort(np.concatenate([np.asarray(chosen, dtype=np.int64), extra.astype(np.int64)]))
+
+
+def _oracle_part(args):
+    shape, seed, group_size, x, tokens = args
+    layer = oracle_layer(shape, seed, group_size)
+    return offn.moe_forward(layer, x, tokens=tokens)["out"]
+
+
+def oracle_outputs(shape: synth.LayerShape, x, tokens: np.ndarray, ids: np.ndarray, seed: int = 0,
+                   group_size: int = 128, workers: int = 0) -> np.ndarray:
+    """oracle moe_forward rows of ``tokens``, computed by ``workers`` spawned
+    processes (the cost is one weight preparation per distinct expert, so the
+    tokens are split into parts with few experts each).  Same values as one
+    call: every token's row depends on its own experts only."""
+    import multiprocessing as mp
+    import os
+    from concurrent.futures import ProcessPoolExecutor
+    workers = workers or min(16, os.cpu_count() or 1)
+    # order the tokens by their first expert so each part touches few experts
+    order = np.argsort(ids[tokens, 0], kind="stable")
+    parts = [p for p in np.array_split(tokens[order], workers) if p.size]
+    with ProcessPoolExecutor(len(parts), mp_context=mp.get_context("spawn")) as ex:
+        outs = list(ex.map(_oracle_part, [(shape, seed, group_size, x, p) for p in parts]))
+    rows = {}
+    for p, o in zip(parts, outs):
+        for i, t in enumerate(p):
+            rows[int(t)] = o[i]
+    return np.stack([rows[int(t)] for t in tokens])
 
 
 def rel_err(gpu_out: np.ndarray, ref: np.ndarray) -> float:

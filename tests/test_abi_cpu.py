@@ -26,7 +26,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 15
+    assert len(names) == 17
     for n in names:
         assert hasattr(lib, n), n
 
@@ -212,3 +212,40 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         moe.quantize_int4(torch.zeros(2, 128))
+
+
+def _scout_decode_desc(**kw):
+    """The Scout-shaped decode layer (D=5120, F=8192, 16 experts, top-1), fake
+    pointers: only for calls that return before touching the device."""
+    return _desc(E=16, k=1, D=5120, F=8192, F_shared=8192, **kw)
+
+
+def test_noalloc_checks_arguments_before_the_cuda_runtime(lib):
+    """Argument errors of moe_ffn_forward_noalloc come back as such, before
+    the library looks up its scratch array (which needs a device)."""
+    S = moe.Status
+    f = 1 << 20
+    d = _scout_decode_desc()
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(d), None, 16, f, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(d), f, 16, None, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(d), f, 16, f + 8, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(d), f + 4, 16, f, None) == S.INVALID_ARG
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(d), f, 0, f, None) == S.UNSUPPORTED_SHAPE
+    assert lib.moe_ffn_forward_noalloc(None, f, 16, f, None) == S.INVALID_ARG
+
+
+def test_noalloc_scratch_covers_scout_decode_batches(lib):
+    """The no-alloc entry point's 8 MiB scratch holds every batch of the
+    Scout-shaped decode layer that takes the weight-streaming path (T * k <=
+    4 E, i.e. T <= 64); the first batch past it (T = 65, tensor-core path)
+    is refused with WORKSPACE_TOO_SMALL before anything is launched."""
+    S = moe.Status
+    f = 1 << 20
+    scratch = 8 << 20
+    dec = _scout_decode_desc(path=moe.PATH_DECODE)
+    assert lib.moe_ffn_workspace_size(ctypes.byref(dec), 64) <= scratch
+    pre = _scout_decode_desc(path=moe.PATH_PREFILL)
+    assert lib.moe_ffn_workspace_size(ctypes.byref(pre), 65) > scratch
+    auto = _scout_decode_desc()
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(auto), f, 65, f, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_ffn_forward_noalloc(ctypes.byref(auto), f, 4096, f, None) == S.WORKSPACE_TOO_SMALL

@@ -7,7 +7,8 @@ import torch
 import int4_quantized_expert_b200 as moe
 import synth
 from oracle import ffn as offn
-from tests._layers import build, rel_err
+from oracle import route as oroute
+from tests._layers import build, covering_tokens, oracle_outputs, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -88,27 +89,37 @@ def test_scout_decode_full_size():
     assert rel_err(got, ref) <= TOL
 
 
-def _sampled(name, n_tokens, seed=0):
+def _sampled(name, n_extra, seed=0):
+    """The workload at full size through AUTO; checked on a covering sample:
+    one token for every expert that some token chose, plus ``n_extra`` random
+    tokens, against the oracle (evaluated by spawned processes)."""
     shape = synth.SHAPES[name]
     b = build(shape)
-    rng = np.random.default_rng(seed)
-    tokens = np.sort(rng.choice(shape.T, n_tokens, replace=False))
-    got, ref = _run(b, moe.PATH_AUTO, tokens=tokens)
+    ids = oroute.route(b.x, b.w_router, b.bias, shape.k)["ids"]
+    tokens = covering_tokens(ids, shape.E, n_extra, seed)
+    chosen = set(ids.reshape(-1).tolist())
+    assert chosen == set(ids[tokens].reshape(-1).tolist())      # every used expert is checked
+    b.gpu.set_path(moe.PATH_AUTO)
+    out = b.gpu(b.x.cuda())
+    assert b.gpu.device_status() == moe.Status.OK
+    got = out.float().cpu().numpy().astype(np.float64)[tokens]
+    ref = oracle_outputs(shape, b.x, tokens, ids, seed=0)
     return got, ref
 
 
 @pytest.mark.slow
 def test_scout_prefill_full_size_sampled():
     """The prefill workload at full size (T=8192) through the tensor-core
-    path, 24 sampled tokens checked against the oracle."""
-    got, ref = _sampled("scout_prefill", 24)
+    path: a token of every expert plus 16 random ones."""
+    got, ref = _sampled("scout_prefill", 16)
     assert rel_err(got, ref) <= TOL
 
 
 @pytest.mark.slow
 def test_skewed_full_size_sampled():
-    """The Zipf-routed workload at full size (T=32768), 24 sampled tokens."""
-    got, ref = _sampled("skewed", 24, seed=1)
+    """The Zipf-routed workload at full size (T=32768): a token of every
+    expert, the 0.2 %-load tail included, plus 16 random ones."""
+    got, ref = _sampled("skewed", 16, seed=1)
     assert rel_err(got, ref) <= TOL
 
 
@@ -144,7 +155,47 @@ def test_fp8_layers(shape):
 
 @pytest.mark.slow
 def test_maverick_fp8_full_size_sampled():
-    """The Maverick-shaped FP8 layer at full size (T=4096, 128 experts, top-8),
-    8 sampled tokens (up to 64 experts) checked against the oracle."""
-    got, ref = _sampled("maverick_fp8", 8, seed=2)
+    """The Maverick-shaped FP8 layer at full size (T=4096, 128 experts,
+    top-8): a covering sample that checks a token of each of the 128 experts."""
+    got, ref = _sampled("maverick_fp8", 0, seed=2)
     assert rel_err(got, ref) <= TOL
+
+
+def _wide_range_tokens(shape, w_router, bias, seed):
+    """bf16 token rows whose elements span 30 binades (magnitudes 2^U(-20, 10),
+    random signs), each row also scaled by 2^0, 2^-8 or 2^-16, so some rows --
+    and every hidden activation h they produce -- are tiny.  Rows whose top-
+    (k+1) logits are closer than 1e-4 of the row's largest logit are redrawn."""
+    rng = np.random.default_rng(seed)
+    x = np.empty((shape.T, shape.D), dtype=np.float64)
+    todo = np.arange(shape.T)
+    while todo.size:
+        n = todo.size
+        mag = np.exp2(rng.uniform(-20.0, 10.0, (n, shape.D)))
+        sign = np.where(rng.random((n, shape.D)) < 0.5, -1.0, 1.0)
+        row = np.exp2(-8.0 * rng.integers(0, 3, (n, 1)))
+        x[todo] = torch.from_numpy(sign * mag * row).to(torch.bfloat16).double().numpy()
+        lg = oroute.router_logits(x[todo], w_router, bias)
+        m = min(shape.k + 1, shape.E)
+        top = -np.sort(-lg, axis=1)[:, :m]
+        ok = (np.diff(-top, axis=1) > 1e-4 * np.abs(lg).max(axis=1, keepdims=True)).all(axis=1)
+        todo = todo[~ok]
+    return torch.from_numpy(x).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("path", [moe.PATH_DECODE, moe.PATH_PREFILL])
+@pytest.mark.parametrize("T,D,F,Fs,E,k", [(48, 256, 512, 512, 4, 1), (37, 384, 640, 384, 5, 2)])
+def test_wide_dynamic_range_rows(T, D, F, Fs, E, k, path):
+    """Token rows spanning 30 binades, and rows 2^-16 smaller than others,
+    through the weight-streaming path's scaled fp16 re-encoding of x and h
+    (and the tensor-core path): every row within 1e-2 of its own largest
+    oracle value."""
+    b = build(synth.LayerShape("wide", T, D, F, E, k, Fs), margin=False)
+    b.x = _wide_range_tokens(b.shape, b.w_router, b.bias, seed=5)
+    b.gpu.set_path(path)
+    out = b.gpu(b.x.cuda())
+    assert b.gpu.device_status() == moe.Status.OK
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = offn.moe_forward(b.oracle, b.x)["out"]
+    row_err = np.abs(got - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert row_err.max() <= TOL, row_err.max()

@@ -1,6 +1,6 @@
 """GPU routing vs the oracle: ids, counts, offsets and the permutation are
 bit-exact on inputs whose top-(k+1) logits are more than 1e-3 apart; gates
-agree to within the fp32 evaluation error."""
+agree to within the error of fp32 logits (relative bound below)."""
 import numpy as np
 import pytest
 import torch
@@ -12,8 +12,16 @@ from tests._layers import margin_tokens
 
 pytestmark = pytest.mark.gpu
 
-# gates: fp32 logits (error ~1e-6 of the logit scale ~1.4) through expf
-GATE_ATOL = 2e-5
+# Gates: the GPU sums each logit in fp32, the oracle in fp64.  A gate's
+# relative error is at most its logits' absolute error for the sigmoid
+# (d ln sigma = (1 - sigma) dl) and twice it for a softmax (d ln g_j = dl_j -
+# sum_i g_i dl_i), plus a few ulps of expf.  The fp32 running sum of a logit
+# takes about D / 16 roundings (16 products per MMA step), each at most half
+# an ulp of a value below ~10 (4.8e-7); as independent errors they come to
+# about sqrt(D / 16) * 4.8e-7, ~9e-6 for D = 5120 at worst, typically a few
+# times less.  Measured on a B200 at the workloads' full sizes: at most
+# 2.4e-6 relative (Maverick, top-8 softmax), 8.3e-7 absolute.
+GATE_RTOL = 1e-5
 
 
 def _check(shape, seed=0):
@@ -28,7 +36,7 @@ def _check(shape, seed=0):
     assert np.array_equal(r["offsets"].cpu().numpy(), ref["offsets"])
     assert np.array_equal(r["perm"].cpu().numpy(), ref["perm"])
     g = r["gates"].cpu().numpy().astype(np.float64)
-    assert np.abs(g - ref["gates"]).max() <= GATE_ATOL
+    assert (np.abs(g - ref["gates"]) / ref["gates"]).max() <= GATE_RTOL
     if shape.k > 1:
         assert np.allclose(g.sum(axis=1), 1.0, atol=1e-5)
     return ref
