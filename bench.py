@@ -291,12 +291,13 @@ def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> di
         "router": ("flops", 2 * T * D * E),
         "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
         "act16_x": ("bytes", T * D * 2 * 2),
+        # weights once; x read; h written as bf16 (routed and shared) and as the
+        # down pass's fp16 operands (routed)
         "decode_gate_up": ("bytes", n_touched * (codes_gu + scales_gu) + 2 * Fs * D * 2 + T * D * 2
-                           + (S * F + T * Fs) * 2),
-        "act16_h": ("bytes", S * F * 2 * 2),
+                           + (S * F + T * Fs) * 2 + S * F * 2),
+        # weights once; h read; y written (routed and shared); out written
         "decode_down": ("bytes", n_touched * (codes_d + scales_d) + D * Fs * 2 + (S * F + T * Fs) * 2
-                        + (S + T) * D * 4),
-        "combine": ("bytes", (S + T) * D * 4 + T * D * 2),
+                        + (S + T) * D * 4 + T * D * 2),
         "gather": ("bytes", S * D * 2 * 2),
         "tc_gate_up": ("flops", 2 * S * D * 2 * F),
         "tc_down": ("flops", 2 * S * F * D),

@@ -14,19 +14,23 @@
 //     whole K) from a global counter, shared expert first, and streams each
 //     task through a ring of 6 stages.  A stage holds 16 KB of weights (2-D
 //     TMA, 64 rows x 128 bytes, 128-byte swizzle), the chunk's token rows for
-//     the stage's K range (one 3-D TMA box) and, for int4, the rows' group
-//     offsets (one 2-D box).  The benchmark's fp32 scales arrive first, one padded
-//     2-D box per matrix.
+//     the stage's K range (one 3-D TMA box) and, for int4, the rows' per-group
+//     (offset, scale) pairs (one 2-D box).  The benchmark's fp32 weight scales
+//     arrive first, one padded 2-D box per matrix.
 //   * 12 consumer warps: 4 row blocks of 16 rows x 3 K phases (a stage goes to
 //     phase (global stage index) % 3), three per SM sub-partition to hide each
 //     one's MMA and load latencies.  Each converts int4 codes to exact fp16
 //     integers in registers (no scale multiply per element), runs m16n8k16
 //     tensor-core MMAs against the tokens (fp32 accumulate), and applies the
-//     group's scale to the 128-K partial sum.  The 3 K phases are summed
-//     through shared memory, then the epilogue applies SwiGLU (gate/up pass)
-//     or the gate (down pass).
+//     group's weight scale (times the token group's power of two) to the
+//     128-K partial sum.  At the end of a task every consumer warp hands its
+//     partial sums over through shared memory and goes on with the next task.
+//   * 3 epilogue warps (the rest of the producer's warpgroup) sum the K
+//     phases in a fixed order and apply SwiGLU (gate/up pass) or the gate
+//     (down pass), off the consumers' path.
 //   * Tokens are the MMA's N operand (8 per n-tile), written by act16_kernel as
-//     fp16 rows in the order the int4 unpacking yields.
+//     fp16 rows in the order the int4 unpacking yields, each group of 128
+//     scaled by its own power of two.
 //   * Every wait is bounded; a timeout sets the status word and the CTA
 //     drains its copies in flight and returns.
 //   * Launches chain by programmatic dependent launch: each kernel's setup
@@ -53,7 +57,7 @@ static_assert(128 * DC_PRODUCER_REGS + 32 * DC_CONSUMERS * DC_CONSUMER_REGS <= D
 constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 64 rows x 128 B
 constexpr int DC_STAGE = 2 * DC_CHUNK;      // weights of a stage: 16 KB
 constexpr int DC_B_OFF = DC_STAGE;          // then the chunk's token rows for the stage's K range
-// then the rows' int4 group offsets (8 rows x 4 groups) in a 1 KB unit; the
+// then the rows' per-group (offset, scale) pairs (8 rows x 4 groups) in a 1 KB unit; the
 // token rows take 4 KB (gate/up: 256 K of 8 routed or 64 K of 16 shared rows)
 // or 8 KB (down: 512 K routed, 128 K shared)
 __host__ __device__ constexpr int dc_c_off(int mode) { return DC_B_OFF + (mode == 0 ? 4096 : 8192); }
@@ -67,7 +71,9 @@ __host__ __device__ constexpr int dc_nstages(int mode) { return mode == 0 ? 6 : 
 constexpr int DC_MAX_STAGES = 6;
 static_assert(dc_nstages(0) % DC_KPH == 0 && dc_nstages(1) % DC_KPH == 0, "ring depth vs K phases");
 constexpr int DC_NT = 2;                    // n-tiles of 8 tokens per task
-constexpr int DC_RED_FLOATS = (DC_KPH - 1) * DC_RB * 32 * DC_NT * 8;   // partial sums of K phases 1..2
+constexpr int DC_HELPERS = 3;              // epilogue warps: warps 1..3 (the producer warpgroup)
+constexpr int DC_RED_PITCH = DC_NT * 8 + 1; // floats per consumer lane in red[] (odd: no bank conflicts)
+constexpr int DC_RED_FLOATS = DC_KPH * DC_RB * 32 * DC_RED_PITCH;   // every consumer warp's partial sums
 
 struct TaskInfo {
     int32_t kind;       // 0 = shared (bf16), 1 = routed (int4), -1 = done
@@ -85,16 +91,12 @@ struct DecodeSmem {
     uint64_t empty[DC_MAX_STAGES];
     uint64_t sfull[2];
     uint64_t sempty[2];
-    uint64_t red_full;    // K phases 1..2 -> phase 0: partial sums written
-    uint64_t red_empty;   // phase 0 -> phases 1..2: partial sums consumed
+    uint64_t red_full;    // consumers -> epilogue warps: a task's partial sums written
+    uint64_t red_empty;   // epilogue warps -> consumers: partial sums consumed
     TaskInfo task[2];
 };
 
 __device__ __forceinline__ int sigma8(int g) { return ((g & 1) << 2) | (g >> 1); }
-
-__device__ __forceinline__ uint4 lds128(const unsigned char* p) {
-    return *reinterpret_cast<const uint4*>(p);
-}
 
 // The first stage of a task (its stages are it_base, it_base + 1, ...) that
 // belongs to K phase q: phases take stages by their global index.
@@ -124,12 +126,13 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 // Codes enter fp16 MMAs as exact integers: per 32-bit word of 8 codes, one
 // shift and four LOP3s give (k0,k4) and (k2,k6) as 1032 + q and (k1,k5),
 // (k3,k7) as 1152 + 16 q (f16_lo_nibbles / f16_hi_nibbles, the magic numbers
-// held in registers klo, khi).  The token rows (fp16, scaled per row by a
-// power of two) store odd positions divided by 16 and every 8-block in the
-// order x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x plus a
-// per-group offset (negc) that is added to the group's partial sum.  The
-// stage holds the chunk's 8 token rows for its K range and their group
-// offsets next to the codes; MMA column g is token row sigma8(g).
+// held in registers klo, khi).  The token rows (fp16, each group of 128
+// scaled by a power of two) store odd positions divided by 16 and every
+// 8-block in the order x0 x4 x2 x6 x1 x5 x3 x7, so one accumulator sums q * x
+// plus a per-group offset that is added to the group's partial sum.  The
+// stage holds the chunk's 8 token rows for its K range and their groups'
+// (offset, scale) pairs next to the codes; MMA column g is token row
+// sigma8(g).
 template <int MODE>
 __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
                                              const float* sc, uint32_t it_base, int q, int lane, int row_a,
@@ -171,12 +174,14 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
         const int gi = gl & 1;
         uint4 xc[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xc[i] = lds128(bt + gl * 2048 + offx[i]);
-        const float cc0 = ct[tc0 * 4 + cg0 + gl], cc1 = ct[tc1 * 4 + cg0 + gl];
-        const uint4 wa = lds128(tile + off_a[gi]);
-        const uint4 wb = lds128(tile + off_b[gi]);
+        for (int i = 0; i < 4; ++i) xc[i] = ld_shared_v4(bt + gl * 2048 + offx[i]);
+        const float2 m0 = ld_shared_f32x2(ct + tc0 * 8 + 2 * (cg0 + gl));   // (offset, 2^e) of token row tc0
+        const float2 m1 = ld_shared_f32x2(ct + tc1 * 8 + 2 * (cg0 + gl));
+        const float cc0 = m0.x, cc1 = m1.x;
+        const uint4 wa = ld_shared_v4(tile + off_a[gi]);
+        const uint4 wb = ld_shared_v4(tile + off_b[gi]);
         uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-        if (MODE == 0) { va = lds128(st + DC_CHUNK + off_a[gi]); vb = lds128(st + DC_CHUNK + off_b[gi]); }
+        if (MODE == 0) { va = ld_shared_v4(st + DC_CHUNK + off_a[gi]); vb = ld_shared_v4(st + DC_CHUNK + off_b[gi]); }
         const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
         const uint32_t VA[4] = {va.x, va.y, va.z, va.w}, VB[4] = {vb.x, vb.y, vb.z, vb.w};
         // one accumulation chain per matrix over the group's 8 MMAs, started
@@ -210,14 +215,17 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
                               f16_hi_nibbles(va8, khi), f16_hi_nibbles(vb8, khi), xc[jj].z, xc[jj].w);
             }
         }
-        // C columns 2c and 2c + 1 (r & 1) are token rows tc0 and tc1
-        const float sga = sga_p[G], sgb = sgb_p[G];
+        // C columns 2c and 2c + 1 (r & 1) are token rows tc0 and tc1; the group's
+        // weight scale times the token group's power of two (an exact product)
+        const float sga = ld_shared_f32(sga_p + G), sgb = ld_shared_f32(sgb_p + G);
+        const float wg[4] = {sga * m0.y, sga * m1.y, sgb * m0.y, sgb * m1.y};
 #pragma unroll
-        for (int r = 0; r < 4; ++r) acc0[r] = fmaf(pg[r] + ((r & 1) ? cc1 : cc0), r < 2 ? sga : sgb, acc0[r]);
+        for (int r = 0; r < 4; ++r) acc0[r] = fmaf(pg[r] + ((r & 1) ? cc1 : cc0), wg[r], acc0[r]);
         if (MODE == 0) {
-            const float sua = sua_p[G], sub = sub_p[G];
+            const float sua = ld_shared_f32(sua_p + G), sub = ld_shared_f32(sub_p + G);
+            const float wu[4] = {sua * m0.y, sua * m1.y, sub * m0.y, sub * m1.y};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc1[r] = fmaf(pu[r] + ((r & 1) ? cc1 : cc0), r < 2 ? sua : sub, acc1[r]);
+            for (int r = 0; r < 4; ++r) acc1[r] = fmaf(pu[r] + ((r & 1) ? cc1 : cc0), wu[r], acc1[r]);
         }
     };
 
@@ -247,6 +255,189 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
     return ok;
 }
 
+// One 8-block of a row's fp16 operands (the format act16_kernel describes):
+// 16 consecutive lanes hold one group of 128 values; every lane of the warp
+// takes part (its shuffles span each aligned half-warp), only `valid` lanes
+// store.
+__device__ __forceinline__ void act16_block(const uint4 v, bool valid, __half* out16_row, float* meta_row, int b) {
+    const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));   // the group's 16 lanes
+    int e = 0;
+    if (m > 0.0f) {
+        e = int((__float_as_uint(m) >> 23) & 0xFF) - 127 - 14;
+        e = max(-100, min(e, 113));
+    }
+    const float down = __uint_as_float(uint32_t(127 - e) << 23);
+    const int order[8] = {0, 4, 2, 6, 1, 5, 3, 7};
+    __half h[8];
+    float ev = 0.0f, od = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = __float2half_rn(x[order[i]] * down * (i < 4 ? 1.0f : 0.0625f));
+        if (i < 4) ev += __half2float(h[i]); else od += __half2float(h[i]);
+    }
+    float cs = 1032.0f * ev + 1152.0f * od;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    if (valid) {
+        const int lc = b & 15, ci = lc >> 2, ii = lc & 3;
+        const int sb = (b & ~15) + 8 * (ii >> 1) + ci + 4 * (ii & 1);
+        *reinterpret_cast<uint4*>(out16_row + 8 * sb) = *reinterpret_cast<const uint4*>(h);
+        if (lc == 0) *reinterpret_cast<float2*>(meta_row + 2 * (b / 16)) = make_float2(-cs, __uint_as_float(uint32_t(127 + e) << 23));
+    }
+}
+
+// The epilogue warps (warps 1..3; `hw` = 0..2): for each task, once the
+// consumer warps have handed over their partial sums, sum the K phases and
+// finish the task's outputs -- SwiGLU into h (gate/up pass) or the gate-scaled
+// y (down pass) -- while the consumers go on with the next task's stages.
+// Warp hw takes the task's columns hw, hw + 3, ...: all 64 rows of each, two
+// per lane, so consecutive lanes store consecutive rows.
+//
+// Consumer warp (q, rb) lane (g, c) holds C rows 16 rb + sigma8(g) (r < 2)
+// and + 8 (r >= 2) of the task's 64, columns nt * 8 + sigma8(2 c + (r & 1)).
+//
+// Then, with no wait on another CTA, the last writer finishes what needs
+// several tasks' results (an atomic counter says who is last):
+//   gate/up pass: a group of 128 rows of h is written by two tasks; the second
+//     to finish a token column converts the group into the down pass's fp16
+//     operands (act16_block), so no separate conversion pass is needed;
+//   down pass: out[t] rows of one 64-row block get one contribution from the
+//     shared expert and one per routed slot; the last of them writes
+//     out = bf16(y_s + sum_j y_r[slot j]), summed in that fixed order.
+template <int MODE>
+__device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSmem* sm, const float* red, int hw,
+                                                int lane) {
+    uint32_t it_base = 0;
+    bool waited = false;
+    for (uint32_t tn = 0;; ++tn) {
+        const int b = tn & 1;
+        if (!mbar_wait(&sm->sfull[b], (tn >> 1) & 1, p.status)) return;
+        const TaskInfo ti = sm->task[b];
+        if (ti.kind < 0) return;
+        if (!waited && (MODE == 1 || ti.kind == 1)) {   // per-slot data comes from the kernels before
+            griddep_wait();
+            waited = true;
+        }
+        // column values, lane l holding column l: in the down pass the token the
+        // column belongs to and, for a routed column, its slot's gate
+        float colgate = 1.0f;
+        int coltok = 0;
+        if (MODE == 1 && lane < ti.count) {
+            if (ti.kind == 1) {
+                const int slot = p.perm[ti.start + lane];
+                coltok = slot / p.k_top;
+                colgate = p.gates[slot];
+            } else {
+                coltok = ti.start + lane;
+            }
+        }
+        if (!mbar_wait(&sm->red_full, tn & 1, p.status)) return;
+        for (int col = hw; col < ti.count; col += DC_HELPERS) {
+            const float gt = __shfl_sync(0xffffffffu, colgate, col);
+            const int nt = col >> 3, cn = col & 7;
+            const int jc = ((cn & 3) << 1) | (cn >> 2);             // sigma8(jc) == cn
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int i = half * 32 + lane;                      // row of the task's 64
+                const int i16 = i & 15, ih = i16 & 7;
+                const int g = ((ih & 3) << 1) | (ih >> 2);          // sigma8(g) == ih
+                const int r = (i16 >= 8 ? 2 : 0) + (jc & 1);
+                const int ln = g * 4 + (jc >> 1);
+                // Phase qq holds the task's stages s with s % DC_KPH == (qq - it_base) % DC_KPH,
+                // which depends on the tasks this CTA ran before: the partials are
+                // summed in the order of that residue, so every output has the same
+                // rounding whichever CTA computed it.
+                float v0 = 0.0f, v1 = 0.0f;
+#pragma unroll
+                for (int rr = 0; rr < DC_KPH; ++rr) {
+                    const int qq = int((uint32_t(rr) + it_base) % DC_KPH);
+                    const float* o = red + (qq * DC_RB + (i >> 4)) * 32 * DC_RED_PITCH + ln * DC_RED_PITCH + nt * 8;
+                    const float a0 = ld_shared_f32(o + r);
+                    v0 = rr == 0 ? a0 : v0 + a0;
+                    if (MODE == 0) {
+                        const float a1 = ld_shared_f32(o + 4 + r);
+                        v1 = rr == 0 ? a1 : v1 + a1;
+                    }
+                }
+                const int n = ti.row0 + i;
+                if (MODE == 0) {
+                    const bf16 hv = __float2bfloat16_rn(silu_f32(v0) * v1);
+                    if (ti.kind == 1) p.h_r[int64_t(ti.start + col) * p.n_rows_r + n] = hv;
+                    else p.h_s[int64_t(ti.start + col) * p.n_rows_s + n] = hv;
+                } else {
+                    if (ti.kind == 1) p.y_r[int64_t(ti.start + col) * p.n_rows_r + n] = v0 * gt;
+                    else p.y_s[int64_t(ti.start + col) * p.n_rows_s + n] = v0;
+                }
+            }
+        }
+        // red[] and the task slot are free again (ti is a copy)
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&sm->red_empty);
+            mbar_arrive(&sm->sempty[b]);
+        }
+        it_base += ti.n_stages;
+
+        // ---- last writers: this warp's stores are made visible first ----
+        const int n_mine = ti.count > hw ? (ti.count - hw + DC_HELPERS - 1) / DC_HELPERS : 0;
+        const int mycol = hw + DC_HELPERS * lane;                    // lane j < n_mine: this warp's j-th column
+        if (MODE == 0 && ti.kind == 1) {
+            const int F = p.n_rows_r, grp = ti.row0 >> 7;
+            __threadfence();
+            __syncwarp();
+            bool last = false;
+            if (lane < n_mine) last = atomicAdd(&p.hcnt[int64_t(ti.start + mycol) * (F >> 7) + grp], 1) == 1;
+            uint32_t todo = __ballot_sync(0xffffffffu, last);
+            if (todo) __threadfence();
+            while (todo) {   // two columns per pass: lanes 0..15 and 16..31, one 8-block each
+                const int j0 = __ffs(todo) - 1;
+                todo &= todo - 1;
+                int j1 = -1;
+                if (todo) {
+                    j1 = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                }
+                const int j = lane < 16 ? j0 : j1;
+                const bool valid = j >= 0;
+                const int64_t pos = ti.start + hw + DC_HELPERS * (valid ? j : j0);
+                const int bb = grp * 16 + (lane & 15);                  // 8-block of the row
+                const uint4 v = valid ? __ldcg(reinterpret_cast<const uint4*>(p.h_r + pos * F + 8 * bb))
+                                      : make_uint4(0, 0, 0, 0);
+                act16_block(v, valid, p.h16 + pos * F, p.h_meta + pos * act16_meta_pitch(F), bb);
+            }
+        }
+        if (MODE == 1 && p.out != nullptr) {
+            const int D = p.n_rows_s, blk = ti.row0 >> 6;
+            const int tok = __shfl_sync(0xffffffffu, coltok, mycol & 31);
+            __threadfence();
+            __syncwarp();
+            bool last = false;
+            if (lane < n_mine) last = atomicAdd(&p.ocnt[int64_t(tok) * (D >> 6) + blk], 1) == p.k_top;
+            uint32_t todo = __ballot_sync(0xffffffffu, last);
+            if (todo) __threadfence();
+            while (todo) {
+                const int j = __ffs(todo) - 1;
+                todo &= todo - 1;
+                const int64_t t = __shfl_sync(0xffffffffu, tok, j);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int n = ti.row0 + half * 32 + lane;
+                    float a = __ldcg(p.y_s + t * D + n);
+                    for (int js = 0; js < p.k_top; ++js)
+                        a += __ldcg(p.y_r + int64_t(__ldcg(p.inv_perm + t * p.k_top + js)) * D + n);
+                    p.out[t * D + n] = __float2bfloat16_rn(a);
+                }
+            }
+        }
+    }
+}
+
 template <int MODE>   // 0 = gate/up with SwiGLU, 1 = down
 __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const __grid_constant__ CUtensorMap tm_r0, const __grid_constant__ CUtensorMap tm_r1,
@@ -267,9 +458,12 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) { mbar_init(&sm->full[i], 1); mbar_init(&sm->empty[i], DC_RB); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&sm->sfull[i], 1); mbar_init(&sm->sempty[i], DC_CONSUMERS); }
-        mbar_init(&sm->red_full, (DC_KPH - 1) * DC_RB);
-        mbar_init(&sm->red_empty, DC_RB);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm->sfull[i], 1);
+            mbar_init(&sm->sempty[i], DC_CONSUMERS + DC_HELPERS);
+        }
+        mbar_init(&sm->red_full, DC_CONSUMERS);
+        mbar_init(&sm->red_empty, DC_HELPERS);
         fence_barrier_init();
     }
     griddep_launch_dependents();
@@ -357,11 +551,11 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 }
                 const int kbytes = ti.kind ? 128 : 64;   // tile x extent in elements (uint8 codes / bf16)
                 // token rows of the chunk (8 routed, 16 shared) for the stage's K range,
-                // in boxes of 64 K; routed stages also carry the rows' group offsets
+                // in boxes of 64 K; routed stages also carry the rows' group (offset, scale) pairs
                 const int kstage = (MODE == 0 ? 1 : 2) * kchunk;   // K values per stage
                 const int nbox = kstage / 64;
                 const uint32_t box_bytes = ti.kind ? 1024u : 2048u;
-                const uint32_t b_bytes = uint32_t(nbox) * box_bytes + (ti.kind ? 128u : 0u);
+                const uint32_t b_bytes = uint32_t(nbox) * box_bytes + (ti.kind ? 256u : 0u);
                 const CUtensorMap* mb = ti.kind ? &tm_br : &tm_bs;
                 for (int s = 0; s < ti.n_stages; ++s, ++it) {
                     const uint32_t slot = it % NST;
@@ -380,8 +574,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     }
                     // one 3-D box: nbox 64-K chunks x the chunk's rows (chunks beyond K read zeros)
                     tma_load_3d(st + DC_B_OFF, mb, &sm->full[slot], 0, ti.start, s * kstage / 64);
-                    if (ti.kind)   // group offsets: 4 groups from the stage's first, rounded down to a multiple of 4
-                        tma_load_2d(st + C_OFF, &tm_cr, &sm->full[slot], (s * kstage / kGroup) & ~3, ti.start);
+                    if (ti.kind)   // group (offset, scale) pairs: 4 groups from the stage's first, rounded down to a multiple of 4
+                        tma_load_2d(st + C_OFF, &tm_cr, &sm->full[slot], 2 * ((s * kstage / kGroup) & ~3), ti.start);
                 }
             }
             // this grid completes only after the kernels before it
@@ -391,6 +585,8 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const uint32_t j = it - 1 - i;
                 mbar_wait(&sm->full[j % NST], (j / NST) & 1, nullptr);
             }
+        } else if (warp >= 1 && warp <= DC_HELPERS) {
+            decode_epilogue<MODE>(p, sm, red, warp - 1, lane);
         }
         return;
     }
@@ -416,17 +612,6 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         }
         const float* sc = sbuf + b * p.scale_buf_floats;
 
-        // MMA column g of n-tile nt is token row nt * 8 + sigma8(g) of the chunk;
-        // routed results are rescaled per token by their row's power of two
-        // (C columns 2c and 2c + 1 of this thread)
-        float cscale[2] = {1.0f, 1.0f};
-        if (ti.kind == 1) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int tok = sigma8(2 * c + h);
-                if (tok < ti.count) cscale[h] = p.rscale_r[ti.start + tok];
-            }
-        }
         const int nt_used = ti.count > 8 ? 2 : 1;
 
         float acc0[DC_NT][4], acc1[DC_NT][4];
@@ -462,14 +647,14 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
 #pragma unroll
                     for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) xc[nt][h2] = lds128(swz(tb, nt * 8 + trow, c + 4 * h2));
+                        for (int h2 = 0; h2 < 2; ++h2) xc[nt][h2] = ld_shared_v4(swz(tb, nt * 8 + trow, c + 4 * h2));
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int j = c + 4 * h2;
-                        const uint4 wa = lds128(swz(ta, row_a, j));
-                        const uint4 wb = lds128(swz(ta, row_b, j));
+                        const uint4 wa = ld_shared_v4(swz(ta, row_a, j));
+                        const uint4 wb = ld_shared_v4(swz(ta, row_b, j));
                         uint4 va = make_uint4(0, 0, 0, 0), vb = va;
-                        if (MODE == 0) { va = lds128(swz(st + DC_CHUNK, row_a, j)); vb = lds128(swz(st + DC_CHUNK, row_b, j)); }
+                        if (MODE == 0) { va = ld_shared_v4(swz(st + DC_CHUNK, row_a, j)); vb = ld_shared_v4(swz(st + DC_CHUNK, row_b, j)); }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             // MMA h takes K values 8 j + 4 h .. + 3 of the rows (natural order):
@@ -503,99 +688,19 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         }
         if (!ok) break;
 
-        // ---- sum the K phases (phases 1.. hand their partial sums to phase 0) ----
-        if (q > 0) {
-            if (!mbar_wait(&sm->red_empty, (tn & 1) ^ 1, p.status)) break;
-            float* my = red + ((q - 1) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
+        // ---- hand the partial sums to the epilogue warps ----
+        if (!mbar_wait(&sm->red_empty, (tn & 1) ^ 1, p.status)) break;
+        float* my = red + (q * DC_RB + rb) * 32 * DC_RED_PITCH + lane * DC_RED_PITCH;
 #pragma unroll
-            for (int nt = 0; nt < DC_NT; ++nt)
+        for (int nt = 0; nt < DC_NT; ++nt)
 #pragma unroll
-                for (int r = 0; r < 4; ++r) { my[nt * 8 + r] = acc0[nt][r]; my[nt * 8 + 4 + r] = acc1[nt][r]; }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->red_full);
-        } else {
-            if (!mbar_wait(&sm->red_full, tn & 1, p.status)) break;
-            // Phase qq holds the task's stages s with s % DC_KPH == (qq - it_base) % DC_KPH,
-            // which depends on the tasks this CTA ran before.  The partials are summed
-            // in the order of that residue, so every output has the same rounding
-            // whichever CTA computed it.
-            float t0[DC_NT][4], t1[DC_NT][4];
-#pragma unroll
-            for (int rr = 0; rr < DC_KPH; ++rr) {
-                const int qq = int((uint32_t(rr) + it_base) % DC_KPH);   // the phase holding residue rr
-                const float* o = red + ((qq > 0 ? qq - 1 : 0) * DC_RB + rb) * 32 * DC_NT * 8 + lane * DC_NT * 8;
-#pragma unroll
-                for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const float v0 = qq == 0 ? acc0[nt][r] : o[nt * 8 + r];
-                        const float v1 = qq == 0 ? acc1[nt][r] : o[nt * 8 + 4 + r];
-                        t0[nt][r] = rr == 0 ? v0 : t0[nt][r] + v0;
-                        t1[nt][r] = rr == 0 ? v1 : t1[nt][r] + v1;
-                    }
-            }
-#pragma unroll
-            for (int nt = 0; nt < DC_NT; ++nt)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) { acc0[nt][r] = t0[nt][r]; acc1[nt][r] = t1[nt][r]; }
-            // ---- epilogue: C rows (row_a, row_b) x columns (2c, 2c + 1) of each n-tile,
-            // column n of n-tile nt being token nt * 8 + sigma8(n) of the chunk ----
-            // routed results are rescaled by their token row's power of two;
-            // h is stored in natural order (the routed rows' fp16 copy is made next)
-#pragma unroll
-            for (int nt = 0; nt < DC_NT; ++nt) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int col = nt * 8 + sigma8(2 * c + (r & 1));
-                    if (col >= ti.count) continue;
-                    const int n = ti.row0 + (r < 2 ? row_a : row_b);
-                    const float cs = cscale[r & 1];   // 1 for the shared expert (one n-tile for routed chunks)
-                    if (MODE == 0) {
-                        if (ti.kind == 1) {
-                            const float hv = silu_f32(acc0[nt][r] * cs) * (acc1[nt][r] * cs);
-                            p.h_r[int64_t(ti.start + col) * p.n_rows_r + n] = __float2bfloat16_rn(hv);
-                        } else {
-                            const float hv = silu_f32(acc0[nt][r]) * acc1[nt][r];
-                            p.h_s[int64_t(ti.start + col) * p.n_rows_s + n] = __float2bfloat16_rn(hv);
-                        }
-                    } else {
-                        if (ti.kind == 1) {
-                            const int pp = ti.start + col;
-                            p.y_r[int64_t(pp) * p.n_rows_r + n] = acc0[nt][r] * cs * p.gates[p.perm[pp]];
-                        } else {
-                            p.y_s[int64_t(ti.start + col) * p.n_rows_s + n] = acc0[nt][r];
-                        }
-                    }
-                }
-            }
-        }
+            for (int r = 0; r < 4; ++r) { my[nt * 8 + r] = acc0[nt][r]; my[nt * 8 + 4 + r] = acc1[nt][r]; }
         __syncwarp();
-        if (q == 0 && lane == 0) mbar_arrive(&sm->red_empty);   // red[] is free again
-        if (lane == 0) mbar_arrive(&sm->sempty[b]);
-        it_base += ti.n_stages;
-    }
-}
-
-// out[t] = bf16(y_s[t] + sum_j y_r[inv_perm[t k + j]])
-__global__ void combine_kernel(const float* __restrict__ y_s, const float* __restrict__ y_r,
-                               const int32_t* __restrict__ inv_perm, int T, int D, int k,
-                               bf16* __restrict__ out) {
-    griddep_launch_dependents();
-    griddep_wait();
-    const int64_t n4 = int64_t(T) * D / 4;
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t t = i / (D / 4);
-        const int d = int(i % (D / 4)) * 4;
-        float4 a = *reinterpret_cast<const float4*>(y_s + t * D + d);
-        for (int j = 0; j < k; ++j) {
-            const int64_t pp = inv_perm[t * k + j];
-            const float4 b = *reinterpret_cast<const float4*>(y_r + pp * D + d);
-            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        if (lane == 0) {
+            mbar_arrive(&sm->red_full);
+            mbar_arrive(&sm->sempty[b]);
         }
-        uint2 o;
-        o.x = pack_bf16x2(a.x, a.y);
-        o.y = pack_bf16x2(a.z, a.w);
-        *reinterpret_cast<uint2*>(out + t * D + d) = o;
+        it_base += ti.n_stages;
     }
 }
 
@@ -689,13 +794,6 @@ moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParam
                       maps.cr, maps.bs, maps.g0, maps.g1, prm);
 }
 
-moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
-                          bf16* out, cudaStream_t stream) {
-    const int64_t n4 = int64_t(T) * D / 4;
-    int64_t blocks = ceil_div(n4, 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    return launch_pdl(combine_kernel, dim3(unsigned(blocks)), dim3(256), 0, stream, y_s, y_r, inv_perm, T, D, k, out);
-}
 
 }  // namespace moe
 
@@ -706,84 +804,43 @@ namespace moe {
 //
 // One CTA per output row of a bf16 matrix (the tokens x gathered into
 // expert-sorted position order, or the routed experts' hidden h, already by
-// position):
-//   scale = 2^-e with e chosen from the row's largest magnitude so that the
-//           scaled row stays below 2^15 (fp16 keeps every bf16 value exactly
-//           in that range); rscale[r] = 2^e undoes it on the MMA results;
+// position).  Each group of 128 values (16 threads, one 8-block each) gets
+// its own power of two:
+//   scale = 2^-e with e chosen from the group's largest magnitude so that the
+//           scaled values stay below 2^15 (fp16 keeps every bf16 value exactly
+//           in that range, down to 2^-24 of its largest);
 //   out16  every 8-block stored as x0 x4 x2 x6 x1/16 x5/16 x3/16 x7/16 (scaled)
 //          -- the K order and the 1/16 factors the int4 unpacking expects --
 //          and, inside each group of 128, 8-block 4 c + i (c, i = 0..3) stored
 //          at 8-block 8 (i >> 1) + c + 4 (i & 1), so that the four threads c
 //          of an MMA fragment read distinct shared-memory banks;
-//   negc   per group of 128: -(1032 * sum of the even-position stored values
-//          + 1152 * sum of the odd-position stored values), the offset the
-//          unpacked codes (1032 + q and 1152 + 16 q) add to a dot product;
-//          rows of act16_negc_pitch(cols) floats.
+//   meta   per group of 128, the pair (offset, 2^e): offset = -(1032 * sum of
+//          the even-position stored values + 1152 * sum of the odd-position
+//          stored values), what the unpacked codes (1032 + q and 1152 + 16 q)
+//          add to a dot product, and 2^e, which undoes the scaling on the
+//          group's partial sum; rows of act16_meta_pitch(cols) floats.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in, int cols,
                                                     const int32_t* __restrict__ src_perm, int k,
-                                                    __half* __restrict__ out16, float* __restrict__ negc,
-                                                    float* __restrict__ rscale) {
-    __shared__ float red[8];
+                                                    __half* __restrict__ out16, float* __restrict__ meta) {
     griddep_launch_dependents();
     griddep_wait();   // the rows (h) or the permutation come from the kernels before
     const int64_t r = blockIdx.x;
     // out row r: input row src_perm[r] / k (tokens into expert-sorted positions), else row r
     const bf16* row = in + (src_perm ? int64_t(src_perm[r] / k) : r) * cols;
-    const int nblk = cols / 8;
-    float m = 0.0f;
-    for (int b = threadIdx.x; b < nblk; b += 256) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * b);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    m = red[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
-    int e = 0;
-    if (m > 0.0f) {
-        e = int((__float_as_uint(m) >> 23) & 0xFF) - 127 - 14;
-        e = max(-100, min(e, 113));
-    }
-    const float down = __uint_as_float(uint32_t(127 - e) << 23);
-    if (threadIdx.x == 0) rscale[r] = __uint_as_float(uint32_t(127 + e) << 23);
-    // 256 threads take consecutive 8-blocks; 16 consecutive threads hold one group
+    const int nblk = cols / 8;   // a multiple of 16: a group's 16 threads are all valid or all not
     for (int b0 = 0; b0 < nblk; b0 += 256) {
         const int b = b0 + threadIdx.x;
-        float ev = 0.0f, od = 0.0f;
-        if (b < nblk) {
-            const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * b);
-            const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-            const int order[8] = {0, 4, 2, 6, 1, 5, 3, 7};
-            __half h[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float s = x[order[i]] * down * (i < 4 ? 1.0f : 0.0625f);
-                h[i] = __float2half_rn(s);
-                if (i < 4) ev += __half2float(h[i]); else od += __half2float(h[i]);
-            }
-            const int lc = b & 15, ci = lc >> 2, ii = lc & 3;
-            const int sb = (b & ~15) + 8 * (ii >> 1) + ci + 4 * (ii & 1);
-            *reinterpret_cast<uint4*>(out16 + r * cols + 8 * sb) = *reinterpret_cast<const uint4*>(h);
-        }
-        float cs = 1032.0f * ev + 1152.0f * od;
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
-        if (b < nblk && (threadIdx.x & 15) == 0) negc[r * act16_negc_pitch(cols) + b / 16] = -cs;
+        const bool valid = b < nblk;
+        const uint4 v = valid ? *reinterpret_cast<const uint4*>(row + 8 * b) : make_uint4(0, 0, 0, 0);
+        act16_block(v, valid, out16 + r * cols, meta + r * act16_meta_pitch(cols), b);
     }
 }
 
 moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
-                        float* negc, float* rscale, cudaStream_t stream) {
+                        float* meta, cudaStream_t stream) {
     if (rows == 0) return MOE_OK;
-    return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, src_perm, k, out16, negc,
-                      rscale);
+    return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, src_perm, k, out16, meta);
 }
 
 }  // namespace moe

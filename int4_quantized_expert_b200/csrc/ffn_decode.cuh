@@ -32,11 +32,16 @@ struct DecodeParams {
     const float* gates;     // per slot
     const float* sc0;       // routed scales: gate/up: gate; down: down   ([E * rows, K / 128])
     const float* sc1;       // routed scales: gate/up: up
-    const float* rscale_r;  // routed token rows (by position): power-of-two scale of each row
     bf16* h_r;              // gate/up outputs: routed [T*k, F] by position, shared [T, F_shared]
     bf16* h_s;
     float* y_r;             // down outputs: routed gate * y [T*k, D] by position, shared [T, D]
     float* y_s;
+    __half* h16;            // gate/up pass: the down pass's fp16 operands of h [T*k, F] (act16 format)
+    float* h_meta;          //   and their per-group (offset, scale) pairs [T*k, act16_meta_pitch(F)]
+    int32_t* hcnt;          //   token columns written per (position, group of 128 rows) [T*k, F / 128], zeroed
+    bf16* out;              // down pass: the layer output [T, D] (null: none)
+    const int32_t* inv_perm;  // slot -> position
+    int32_t* ocnt;          //   contributions written per (token, block of 64 rows) [T, D / 64], zeroed
     int32_t* task_counter;  // cleared with the status word
     int32_t* status;        // device status word
 };
@@ -60,7 +65,7 @@ struct RoutePrep {
 //   s0, s1  shared bf16 weights, box 64 x 64, 128-B swizzle
 //   br      routed token rows, fp16 [T * k, K] by position (act16 layout), 3-D box of 8 rows x the
 //           stage's 64-K chunks (make_tmap_rows_3d)
-//   cr      their group offsets, fp32 [T * k, act16_negc_pitch(K)], box 4 x 8
+//   cr      their per-group (offset, scale) pairs, fp32 [T * k, act16_meta_pitch(K)], box 8 x 8
 //   bs      shared-expert token rows, bf16 [T, K] (x, or the shared h), 3-D box of 16 rows x chunks
 //   g0, g1  routed int4 scales fp32 [E * rows, K / 128] (gate, up; or down), box
 //           scale_row_floats(K / 128) x 64 (when K / 128 is a multiple of 4)
@@ -68,9 +73,9 @@ struct DecodeMaps {
     CUtensorMap r0, r1, s0, s1, br, cr, bs, g0, g1;
 };
 
-// Row pitch (floats) of act16's group offsets: K / 128 rounded up to 4, so
-// every row starts on 16 bytes.
-__host__ __device__ inline int act16_negc_pitch(int cols) { return int(ceil_div(cols / kGroup, 4) * 4); }
+// Row pitch (floats) of act16's per-group (offset, scale) pairs: K / 128
+// groups rounded up to 4, two floats each, so every row starts on 32 bytes.
+__host__ __device__ inline int act16_meta_pitch(int cols) { return int(ceil_div(cols / kGroup, 4) * 8); }
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);
@@ -88,9 +93,7 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between);
 moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
-                        float* negc, float* rscale, cudaStream_t stream);
-moe_status launch_combine(const float* y_s, const float* y_r, const int32_t* inv_perm, int T, int D, int k,
-                          bf16* out, cudaStream_t stream);
+                        float* meta, cudaStream_t stream);
 
 moe_status set_wait_limit_decode(uint32_t cycles);
 

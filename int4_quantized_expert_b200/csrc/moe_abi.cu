@@ -41,11 +41,11 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
 // are shared by both paths; the rest is laid out per path from there, and a
 // workspace must be large enough for either.
 struct WsLayout {
-    size_t status, rt_cnt, zeros_end, counters, rt_part, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t status, rt_cnt, dec_cnt, zeros_end, counters, rt_part, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
     size_t xn;   // RMSNorm of x (layers with rms_weight)
     size_t common_end;
     // weight-streaming path
-    size_t x16, x_negc, x_scale, h_r, h16, h_negc, h_scale, h_s, y_r, y_s;
+    size_t x16, x_meta, h_r, h16, h_meta, h_s, y_r, y_s;
     // tensor-core path (row counts padded to whole 256-token tiles)
     size_t x_sorted, h_sorted, h_s_pad, y_pos, y_shared;
     size_t xq, xq_scale, hq, hq_scale;   // e4m3 activations of FP8_ROW layers
@@ -74,6 +74,9 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.counters = take(64);   // task counters of the weight-streaming kernels
     const bool rt_split = router_ksplit(int(T), L.D) > 1;
     w.rt_cnt = take(rt_split ? size_t(ceil_div(T, 16)) * 4 : 0);   // router tile counters
+    // weight-streaming path: the epilogues' last-writer counters, per (position,
+    // group of 128 rows of h) and per (token, block of 64 output rows)
+    w.dec_cnt = take(path == PATH_SEL_DECODE ? size_t(S * (L.F / 128) + T * (L.D / 64)) * 4 : 0);
     w.zeros_end = off;   // [status, zeros_end) is cleared at the start of every call
     w.rt_part = take(router_partial_floats(int(T), L.D, L.E) * 4);
     w.ids = take(S * 4);
@@ -88,12 +91,10 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
         w.x16 = take(S * L.D * 2);                 // tokens by expert-sorted position
-        w.x_negc = take(S * act16_negc_pitch(L.D) * 4);
-        w.x_scale = take(S * 4);
+        w.x_meta = take(S * act16_meta_pitch(L.D) * 4);
         w.h_r = take(S * L.F * 2);
         w.h16 = take(S * L.F * 2);
-        w.h_negc = take(S * act16_negc_pitch(L.F) * 4);
-        w.h_scale = take(S * 4);
+        w.h_meta = take(S * act16_meta_pitch(L.F) * 4);
         w.h_s = take(T * L.F_shared * 2);
         w.y_r = take(S * L.D * 4);
         w.y_s = take(T * L.D * 4);
@@ -176,9 +177,8 @@ struct Marks {
     }
 };
 
-const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up",
-                                       "act16_h", "decode_down", "combine"};
-constexpr int32_t kDecodeLaunchCount = 7;
+const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up", "decode_down"};
+constexpr int32_t kDecodeLaunchCount = 5;
 
 template <typename T>
 T* at(void* base, size_t off) {
@@ -252,8 +252,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     ++mk.i;
     if (s != MOE_OK) return s;
     mk.mark(st);
-    s = launch_act16(x, S, L.D, perm, L.k, at<__half>(ws, W.x16), at<float>(ws, W.x_negc), at<float>(ws, W.x_scale),
-                     st);
+    s = launch_act16(x, S, L.D, perm, L.k, at<__half>(ws, W.x16), at<float>(ws, W.x_meta), st);
     if (s != MOE_OK) return s;
 
     // tensor maps: built once per (layer, workspace, input, T) and thread
@@ -271,12 +270,12 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
                   make_tmap_2d(&m1.s0, L.ws_gate, 2, L.D, L.F_shared, 64, rows, true) &&
                   make_tmap_2d(&m1.s1, L.ws_up, 2, L.D, L.F_shared, 64, rows, true) &&
                   make_tmap_rows_3d(&m1.br, at<__half>(ws, W.x16), L.D, S, 8, 4) &&
-                  make_tmap_2d(&m1.cr, at<float>(ws, W.x_negc), 4, act16_negc_pitch(L.D), S, 4, 8, false) &&
+                  make_tmap_2d(&m1.cr, at<float>(ws, W.x_meta), 4, act16_meta_pitch(L.D), S, 8, 8, false) &&
                   make_tmap_rows_3d(&m1.bs, x, L.D, T, 16, 1) &&
                   make_tmap_2d(&m2.r0, L.w_down, 1, L.F / 2, E * L.D, 128, rows, true) &&
                   make_tmap_2d(&m2.s0, L.ws_down, 2, L.F_shared, L.D, 64, rows, true) &&
                   make_tmap_rows_3d(&m2.br, at<__half>(ws, W.h16), L.F, S, 8, 8) &&
-                  make_tmap_2d(&m2.cr, at<float>(ws, W.h_negc), 4, act16_negc_pitch(L.F), S, 4, 8, false) &&
+                  make_tmap_2d(&m2.cr, at<float>(ws, W.h_meta), 4, act16_meta_pitch(L.F), S, 8, 8, false) &&
                   make_tmap_rows_3d(&m2.bs, h_s, L.F_shared, T, 16, 2);
         // the task scales: one box per matrix when their rows are whole 16-byte units
         const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
@@ -314,18 +313,15 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.gates = gates;
     p.sc0 = L.s_gate;
     p.sc1 = L.s_up;
-    p.rscale_r = at<float>(ws, W.x_scale);
     p.h_r = h_r;
     p.h_s = h_s;
+    p.h16 = at<__half>(ws, W.h16);      // the gate/up epilogue also writes h's fp16 operands
+    p.h_meta = at<float>(ws, W.h_meta);
+    p.hcnt = at<int32_t>(ws, W.dec_cnt);
     p.task_counter = counters;
     p.status = status;
     mk.mark(st);
     s = launch_decode_ffn(0, m1, p, st);
-    if (s != MOE_OK) return s;
-
-    mk.mark(st);
-    s = launch_act16(h_r, S, L.F, nullptr, 1, at<__half>(ws, W.h16), at<float>(ws, W.h_negc),
-                     at<float>(ws, W.h_scale), st);
     if (s != MOE_OK) return s;
 
     p.n_rows_r = L.D;
@@ -335,15 +331,14 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.scale_buf_floats = decode_scale_floats(1, L.F);
     p.sc0 = L.s_down;
     p.sc1 = nullptr;
-    p.rscale_r = at<float>(ws, W.h_scale);
     p.y_r = y_r;
     p.y_s = y_s;
+    p.out = out;                        // the down epilogue finishes each token
+    p.inv_perm = inv;
+    p.ocnt = at<int32_t>(ws, W.dec_cnt) + S * (L.F / 128);
     p.task_counter = counters + 1;
     mk.mark(st);
     s = launch_decode_ffn(1, m2, p, st);
-    if (s != MOE_OK) return s;
-    mk.mark(st);
-    s = launch_combine(y_s, y_r, inv, T, L.D, L.k, out, st);
     mk.mark(st);
     return s;
 }
@@ -745,7 +740,7 @@ extern "C" moe_status moe_set_wait_limit(int64_t cycles) {
 //   out = bf16( (silu(x Wg^T) * (x Wu^T)) Wd^T ), bf16 weights, the hidden
 // activation rounded to bf16 -- the MoE layer's shared expert without the
 // routed experts.  It runs the shared-expert kernels of either path:
-//   weight streaming: [rmsnorm,] dense_prep, decode gate/up, decode down, combine
+//   weight streaming: [rmsnorm,] dense_prep, decode gate/up, decode down (its epilogue writes out)
 //   tensor cores:     [rmsnorm,] dense_prep, copy to whole tiles, gate/up, down, combine
 // dense_prep writes the token chunk list the kernels take their tasks from.
 // ---------------------------------------------------------------------------
@@ -754,7 +749,7 @@ namespace {
 constexpr int32_t kDenseDecodeMaxT = 64;   // AUTO streams the weights up to this many tokens
 
 struct DenseWs {
-    size_t status, counters, zeros_end, chunks, nchunks, xn;
+    size_t status, counters, ocnt, zeros_end, chunks, nchunks, xn;
     size_t h, y;          // hidden [T(_pad), F] bf16, fp32 result [T, D]
     size_t total;
 };
@@ -778,6 +773,7 @@ DenseWs dense_layout(const moe_dense_desc& L, int64_t T, int path) {
     const int64_t rows = path == PATH_SEL_DECODE ? T : T_pad;
     w.status = take(64);
     w.counters = take(64);
+    w.ocnt = take(path == PATH_SEL_DECODE ? size_t(T) * (L.D / 64) * 4 : 0);   // contributions per output block
     w.zeros_end = off;
     w.chunks = take(size_t(ceil_div(T, 16)) * sizeof(ChunkEntry));
     w.nchunks = take(16);
@@ -896,7 +892,7 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         p.n_rows_s = L.F;
         p.K_r = L.D;
         p.K_s = L.D;
-        p.k_top = 1;
+        p.k_top = 0;   // no routed slots: the shared expert's contribution is each output's only one
         p.scale_buf_floats = 0;
         p.f16_magic_lo = kF16MagicLo;
         p.f16_magic_hi = kF16MagicHi;
@@ -911,10 +907,10 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         p.K_r = L.F;
         p.K_s = L.F;
         p.y_s = y;
+        p.out = static_cast<bf16*>(out);
+        p.ocnt = at<int32_t>(ws, W.ocnt);
         p.task_counter = at<int32_t>(ws, W.counters) + 1;
-        s = launch_decode_ffn(1, m2, p, st);
-        if (s != MOE_OK) return s;
-        return launch_combine(y, nullptr, nullptr, T, L.D, 0, static_cast<bf16*>(out), st);
+        return launch_decode_ffn(1, m2, p, st);
     }
 
     const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);

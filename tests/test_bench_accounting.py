@@ -17,14 +17,15 @@ def test_decode_bytes_per_touched_expert():
     assert gate_up + down == 66_846_720                      # codes 62.9 MB + scales 3.93 MB
     assert gate_up == 2 * (8192 * 5120 // 2 + 8192 * 40 * 4)
     # the whole gate/up launch at 12 touched experts: routed + shared + activations
-    assert w12["decode_gate_up"][1] == 703_234_048
+    # (x read; h written as bf16 and, for the routed rows, as fp16 operands)
+    assert w12["decode_gate_up"][1] == 703_234_048 + 16 * 8192 * 2
 
 
 def test_decode_shared_expert_bytes():
     s = synth.SHAPES["scout_decode"]
     w0 = bench.kernel_work(s, 0)
-    act_gu = 16 * 5120 * 2 + (16 * 8192 + 16 * 8192) * 2
-    act_dn = (16 * 8192 + 16 * 8192) * 2 + (16 + 16) * 5120 * 4
+    act_gu = 16 * 5120 * 2 + (16 * 8192 + 16 * 8192) * 2 + 16 * 8192 * 2
+    act_dn = (16 * 8192 + 16 * 8192) * 2 + (16 + 16) * 5120 * 4 + 16 * 5120 * 2
     assert (w0["decode_gate_up"][1] - act_gu) + (w0["decode_down"][1] - act_dn) == 251_658_240
 
 

@@ -12,7 +12,7 @@ CSRC = os.path.join(ROOT, "int4_quantized_expert_b200", "csrc")
 
 # kernels (mangled-name fragments) that must not spill
 HOT = {
-    "ffn_decode.cu": ["decode_ffn_kernel", "act16_kernel", "combine_kernel"],
+    "ffn_decode.cu": ["decode_ffn_kernel", "act16_kernel"],
     "tc_gemm.cu": ["tc_gemm_kernel", "gather_rows_kernel", "combine_slots_kernel"],
     "quantize.cu": ["quantize_int4_kernel"],
     "norm.cu": ["rmsnorm_kernel"],
