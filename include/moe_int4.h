@@ -324,11 +324,57 @@ MOE_API moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const void
                                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Expert parallelism ([P1], the closing section on dependencies: fairscale
+ * model-parallel splitting; [P4] introduction: Maverick FP8 on one 8-GPU
+ * node).  With the experts spread over P GPUs, a layer is: moe_route on each
+ * GPU's own tokens; an all-to-all that sends every slot's row to the GPU
+ * holding its expert; moe_expert_ffn_forward there; an all-to-all back; and
+ * moe_shared_ffn_combine, which adds the shared expert and sums each token's
+ * slots.  The two calls below are those compute steps; the exchanges are the
+ * caller's (the Python package's expert-parallel layer uses NCCL).  Rows
+ * that arrive from another GPU are in this GPU's memory before either call
+ * reads them.
+ *
+ * moe_expert_ffn_forward -- the routed experts alone, on rows whose expert
+ * and gate are given:
+ *   y[r] = gates[r] * expert_{expert_ids[r]}(x[r])   (fp32, as in the layer)
+ * with `layer`'s routed weights (its router, shared expert and k are not
+ * used; expert_ids index its E experts).
+ *   x  device, bf16 [n, D] (already normalized if the layer has an RMSNorm)
+ *   expert_ids  device, int32 [n], 0 <= id < E;  gates  device, fp32 [n]
+ *   y  device, fp32 [n, D] (output)
+ *   workspace  device, >= moe_expert_ffn_workspace_size(layer, n) bytes,
+ *              256-byte aligned.
+ * An id out of range is counted as expert 0 and reported by
+ * moe_ffn_device_status(workspace) as MOE_ERR_INVALID_ARG.
+ */
+MOE_API size_t moe_expert_ffn_workspace_size(const moe_layer_desc* layer, int32_t n_max);
+MOE_API moe_status moe_expert_ffn_forward(const moe_layer_desc* layer, const void* x, int32_t n,
+                                          const int32_t* expert_ids, const float* gates, float* y,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_shared_ffn_combine -- the rest of the layer for T tokens whose k slots'
+ * routed outputs are given:
+ *   out[t] = bf16( shared(x[t]) + sum_{j < k} y_slots[t, j] )
+ * summed in that order, as moe_ffn_forward does (with layer->rms_weight set,
+ * x is first replaced by moe_rmsnorm(x)).
+ *   x  device, bf16 [T, D];  y_slots  device, fp32 [T, k, D];  out  device, bf16 [T, D]
+ *   workspace  device, >= moe_shared_ffn_workspace_size(layer, T) bytes, 256-byte aligned.
+ */
+MOE_API size_t moe_shared_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max);
+MOE_API moe_status moe_shared_ffn_combine(const moe_layer_desc* layer, const void* x, int32_t T,
+                                          const float* y_slots, void* out, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+/*
  * moe_ffn_device_status -- SYNCHRONIZES `stream`, then reads the device
- * status word that the kernels of the last moe_ffn_forward (or
- * moe_dense_ffn_forward) on this workspace set.  Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait gave up; the
- * outputs of that call are invalid) or MOE_ERR_CUDA.  The word is cleared at
- * the start of every moe_ffn_forward.
+ * status word that the kernels of the last call on this workspace
+ * (moe_ffn_forward, moe_dense_ffn_forward, moe_expert_ffn_forward,
+ * moe_shared_ffn_combine) set.  Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded
+ * device wait gave up; the outputs of that call are invalid),
+ * MOE_ERR_INVALID_ARG (moe_expert_ffn_forward was given an expert id out of
+ * range) or MOE_ERR_CUDA.  The word is cleared at the start of every call.
  */
 MOE_API moe_status moe_ffn_device_status(const void* workspace, void* stream);
 

@@ -101,6 +101,14 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_forward_noalloc.restype = ctypes.c_int
         L.moe_ffn_noalloc_device_status.argtypes = [vp]
         L.moe_ffn_noalloc_device_status.restype = ctypes.c_int
+        L.moe_expert_ffn_workspace_size.argtypes = [ctypes.POINTER(LayerDesc), i32]
+        L.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
+        L.moe_expert_ffn_forward.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.moe_expert_ffn_forward.restype = ctypes.c_int
+        L.moe_shared_ffn_workspace_size.argtypes = [ctypes.POINTER(LayerDesc), i32]
+        L.moe_shared_ffn_workspace_size.restype = ctypes.c_size_t
+        L.moe_shared_ffn_combine.argtypes = [ctypes.POINTER(LayerDesc), vp, i32, vp, vp, vp, ctypes.c_size_t, vp]
+        L.moe_shared_ffn_combine.restype = ctypes.c_int
         L.moe_set_wait_limit.argtypes = [i64]
         L.moe_set_wait_limit.restype = ctypes.c_int
         L.moe_dense_ffn_workspace_size.argtypes = [ctypes.POINTER(DenseDesc), i32]
@@ -309,6 +317,51 @@ class MoELayer:
         _check("moe_ffn_forward_noalloc", lib().moe_ffn_forward_noalloc(
             ctypes.byref(self.desc), _ptr(x), x.shape[0], _ptr(out), _stream(stream)))
         return out
+
+
+    # ---- the compute steps of an expert-parallel layer (see moe_expert_ffn_forward) ----
+    def _scratch(self, attr: str, n: int) -> torch.Tensor:
+        ws = getattr(self, attr, None)
+        if ws is None or ws.numel() < n:
+            ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+            setattr(self, attr, ws)
+        return ws
+
+    def expert_forward(self, x: torch.Tensor, expert_ids: torch.Tensor, gates: torch.Tensor,
+                       stream=None) -> torch.Tensor:
+        """y[r] = gates[r] * expert_{ids[r]}(x[r]), fp32 [n, D]."""
+        n = x.shape[0]
+        y = torch.empty(n, self.D, dtype=torch.float32, device=x.device)
+        if n == 0:
+            return y
+        need = lib().moe_expert_ffn_workspace_size(ctypes.byref(self.desc), n)
+        if need == 0:
+            raise MoEError("moe_expert_ffn_workspace_size", Status.UNSUPPORTED_SHAPE)
+        ws = self._scratch("_expert_ws", need)
+        _check("moe_expert_ffn_forward", lib().moe_expert_ffn_forward(
+            ctypes.byref(self.desc), _ptr(x), n, _ptr(expert_ids), _ptr(gates), _ptr(y), _ptr(ws), ws.numel(),
+            _stream(stream)))
+        self._last_ws = ws
+        return y
+
+    def shared_combine(self, x: torch.Tensor, y_slots: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+        """out[t] = bf16(shared(x[t]) + sum_j y_slots[t, j]), y_slots fp32 [T, k, D]."""
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, self.D, dtype=torch.bfloat16, device=x.device)
+        need = lib().moe_shared_ffn_workspace_size(ctypes.byref(self.desc), T)
+        if need == 0:
+            raise MoEError("moe_shared_ffn_workspace_size", Status.UNSUPPORTED_SHAPE)
+        ws = self._scratch("_shared_ws", need)
+        _check("moe_shared_ffn_combine", lib().moe_shared_ffn_combine(
+            ctypes.byref(self.desc), _ptr(x), T, _ptr(y_slots), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+        self._last_ws = ws
+        return out
+
+    def last_call_status(self, stream=None) -> int:
+        """Synchronizes; the device status of the last expert_forward / shared_combine."""
+        return lib().moe_ffn_device_status(_ptr(self._last_ws), _stream(stream))
 
 
 def noalloc_device_status(stream=None) -> int:

@@ -17,7 +17,7 @@ namespace moe {
 typedef __nv_bfloat16 bf16;
 
 // Device status word values (written into the workspace's first int32).
-enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 1 };
+enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_EXPERT = 2 };
 
 constexpr int kGroup = 128;   // int4 group size along K
 
@@ -236,6 +236,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void* p) {
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
     return v;
 }
+__device__ __forceinline__ uint32_t ld_shared_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+    return v;
+}
 __device__ __forceinline__ float ld_shared_f32(const float* p) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
@@ -292,6 +297,41 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
     return ok != 0;
+}
+
+// Thread-block cluster barrier (every thread of every CTA of the cluster).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A float in the shared memory of CTA `rank` of this cluster, at the address
+// `p` has in this CTA.
+__device__ __forceinline__ float ld_dsmem_f32(const float* p, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// Bounded wait until a global counter written by other CTAs (atomicAdd after
+// a __threadfence) reaches `target`; acquire semantics.  Followed by a proxy
+// fence, so TMA (async-proxy) reads issued after it see what the counted
+// writers stored.
+__device__ __forceinline__ bool wait_counter(const int32_t* cnt, int32_t target, int32_t* status) {
+    const uint32_t t0 = uint32_t(clock64());
+    for (;;) {
+        int32_t v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v >= target) break;
+        if (uint32_t(clock64()) - t0 > c_wait_limit) {
+            atomicExch(status, DEV_TIMEOUT);
+            return false;
+        }
+        __nanosleep(256);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
 }
 
 // Non-blocking test of a phase (try_wait may suspend the thread for a while).

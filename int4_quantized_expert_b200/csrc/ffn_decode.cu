@@ -57,11 +57,18 @@ static_assert(128 * DC_PRODUCER_REGS + 32 * DC_CONSUMERS * DC_CONSUMER_REGS <= D
 constexpr int DC_CHUNK = DC_ROWS * 128;     // one matrix tile of a stage: 64 rows x 128 B
 constexpr int DC_STAGE = 2 * DC_CHUNK;      // weights of a stage: 16 KB
 constexpr int DC_B_OFF = DC_STAGE;          // then the chunk's token rows for the stage's K range
-// then the rows' per-group (offset, scale) pairs (8 rows x 4 groups) in a 1 KB unit; the
-// token rows take 4 KB (gate/up: 256 K of 8 routed or 64 K of 16 shared rows)
-// or 8 KB (down: 512 K routed, 128 K shared)
+// then the rows' per-group (offset, scale) pairs (8 rows x the stage's groups,
+// at most 16) in a 1 KB unit; the token rows take 4 KB (gate/up: 256 K of 8
+// routed or 64 K of 16 shared rows) or 8 KB (down: 512 K routed, 128 K
+// shared).  With groups of 64 or 32 the stage also carries its weight scales
+// (64 rows x the stage's groups, per matrix) in a 4 KB unit.
 __host__ __device__ constexpr int dc_c_off(int mode) { return DC_B_OFF + (mode == 0 ? 4096 : 8192); }
-__host__ __device__ constexpr int dc_slot(int mode) { return dc_c_off(mode) + 1024; }   // a multiple of 1024
+__host__ __device__ constexpr int dc_s_off(int mode) { return dc_c_off(mode) + 1024; }
+__host__ __device__ constexpr int dc_slot(int mode, int G) {   // a multiple of 1024
+    return G == kGroup ? dc_c_off(mode) + 1024 : dc_s_off(mode) + 4096;
+}
+// K values per stage and groups of G per stage
+__host__ __device__ constexpr int dc_kstage(int mode) { return mode == 0 ? 256 : 512; }
 // Ring depth: a multiple of the K-phase count.  A stage goes to K phase
 // (global stage index) % DC_KPH, so every slot is always consumed by the same
 // phase, in order, and no warp ever waits on a slot's next use while its
@@ -133,13 +140,13 @@ __device__ __forceinline__ const unsigned char* swz(const unsigned char* tile, i
 // stage holds the chunk's 8 token rows for its K range and their groups'
 // (offset, scale) pairs next to the codes; MMA column g is token row
 // sigma8(g).
-template <int MODE>
+template <int MODE, int G>
 __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
                                              const float* sc, uint32_t it_base, int q, int lane, int row_a,
                                              int row_b, uint32_t klo, uint32_t khi, float (&acc0)[4],
                                              float (&acc1)[4], int32_t* status) {
     constexpr int GPS = MODE == 0 ? 2 : 4;   // groups per stage
-    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
+    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE, G), C_OFF = dc_c_off(MODE);
     const int g = lane >> 2, c = lane & 3;
     const int ng = ti.K / kGroup;
     // byte offsets of this thread's 16-byte code chunks in a swizzled 64 x 128 B
@@ -255,18 +262,110 @@ __device__ __forceinline__ bool consume_int4(const TaskInfo& ti, DecodeSmem* sm,
     return ok;
 }
 
+// The int4 part of a decode task for groups of G = 64 or 32 K ("Meta Llama
+// Models Llama 4 单卡量化推理与选型指南", "量化环节做了什么": a smaller
+// group_size).  The layout of consume_int4 sums all four 32-K quarters of a
+// 128-K block in every MMA, so it cannot apply one scale per 64 or 32 K.
+// Here the MMAs go quarter by quarter: thread c takes word c (8 codes) of
+// each 32-K quarter of rows row_a and row_b (4-byte loads; the 128-byte
+// swizzle puts a warp's 32 words in 32 banks) and the matching token
+// 8-block, 8 c .. 8 c + 7 of the quarter (act16 keeps the 8-blocks of such
+// groups in their natural order).  A quarter is two MMAs per matrix (low and
+// high nibbles); a group chains its G / 32 quarters, adds the group's token
+// offset and multiplies by the group's weight scale times the token group's
+// power of two.  The stage carries its groups' weight scales and token
+// (offset, scale) pairs.
+template <int MODE, int G>
+__device__ __forceinline__ bool consume_int4_qm(const TaskInfo& ti, DecodeSmem* sm, const unsigned char* ring,
+                                                uint32_t it_base, int q, int lane, int row_a, int row_b, uint32_t klo,
+                                                uint32_t khi, float (&acc0)[4], float (&acc1)[4], int32_t* status) {
+    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE, G), C_OFF = dc_c_off(MODE), S_OFF = dc_s_off(MODE);
+    constexpr int GPS = dc_kstage(MODE) / G;   // groups per stage
+    constexpr int QPG = G / 32;                // quarters per group
+    const int g = lane >> 2, c = lane & 3;
+    const int trow = sigma8(g);
+    const int tc0 = sigma8(2 * c), tc1 = sigma8(2 * c + 1);   // token rows of C columns 2c, 2c + 1
+    const int ng = ti.K / G;
+    bool ok = true;
+    for (int s = first_stage(q, it_base); s < ti.n_stages; s += DC_KPH) {
+        const uint32_t it = it_base + s;
+        const uint32_t slot = it % NST;
+        if (!mbar_wait(&sm->full[slot], (it / NST) & 1, status)) { ok = false; break; }
+        const unsigned char* st = ring + slot * SLOT;
+        const unsigned char* bt = st + DC_B_OFF;
+        const float* meta = reinterpret_cast<const float*>(st + C_OFF);   // [8 token rows][GPS][2]
+        const float* scl = reinterpret_cast<const float*>(st + S_OFF);    // [matrix][64 rows][GPS]
+        const int G0 = s * GPS;
+#pragma unroll
+        for (int gl = 0; gl < GPS; ++gl) {
+            if (G0 + gl >= ng) break;   // the last stage of a task may be partial
+            float pg[4], pu[4];
+#pragma unroll
+            for (int qq = 0; qq < QPG; ++qq) {
+                const int Q = gl * QPG + qq;   // quarter of the stage
+                const unsigned char* tile = st + (MODE == 0 ? 0 : (Q >> 3) * DC_CHUNK);
+                const int ch = Q & 7;
+                const uint32_t wa = ld_shared_u32(tile + row_a * 128 + ((ch ^ (row_a & 7)) << 4) + 4 * c);
+                const uint32_t wb = ld_shared_u32(tile + row_b * 128 + ((ch ^ (row_b & 7)) << 4) + 4 * c);
+                const uint4 xc = ld_shared_v4(bt + (Q >> 1) * 1024 + trow * 128 + ((((Q & 1) * 4 + c) ^ (trow & 7)) << 4));
+                const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+                if (qq == 0)
+                    mma_f16_16816(pg, f16_lo_nibbles(wa, klo), f16_lo_nibbles(wb, klo), f16_lo_nibbles(wa8, klo),
+                                  f16_lo_nibbles(wb8, klo), xc.x, xc.y, 0.0f, 0.0f, 0.0f, 0.0f);
+                else
+                    mma_f16_16816(pg, f16_lo_nibbles(wa, klo), f16_lo_nibbles(wb, klo), f16_lo_nibbles(wa8, klo),
+                                  f16_lo_nibbles(wb8, klo), xc.x, xc.y);
+                mma_f16_16816(pg, f16_hi_nibbles(wa, khi), f16_hi_nibbles(wb, khi), f16_hi_nibbles(wa8, khi),
+                              f16_hi_nibbles(wb8, khi), xc.z, xc.w);
+                if (MODE == 0) {
+                    const unsigned char* up = st + DC_CHUNK;
+                    const uint32_t va = ld_shared_u32(up + row_a * 128 + ((ch ^ (row_a & 7)) << 4) + 4 * c);
+                    const uint32_t vb = ld_shared_u32(up + row_b * 128 + ((ch ^ (row_b & 7)) << 4) + 4 * c);
+                    const uint32_t va8 = va >> 8, vb8 = vb >> 8;
+                    if (qq == 0)
+                        mma_f16_16816(pu, f16_lo_nibbles(va, klo), f16_lo_nibbles(vb, klo), f16_lo_nibbles(va8, klo),
+                                      f16_lo_nibbles(vb8, klo), xc.x, xc.y, 0.0f, 0.0f, 0.0f, 0.0f);
+                    else
+                        mma_f16_16816(pu, f16_lo_nibbles(va, klo), f16_lo_nibbles(vb, klo), f16_lo_nibbles(va8, klo),
+                                      f16_lo_nibbles(vb8, klo), xc.x, xc.y);
+                    mma_f16_16816(pu, f16_hi_nibbles(va, khi), f16_hi_nibbles(vb, khi), f16_hi_nibbles(va8, khi),
+                                  f16_hi_nibbles(vb8, khi), xc.z, xc.w);
+                }
+            }
+            const float2 m0 = ld_shared_f32x2(meta + (tc0 * GPS + gl) * 2);
+            const float2 m1 = ld_shared_f32x2(meta + (tc1 * GPS + gl) * 2);
+            const float sga = ld_shared_f32(scl + row_a * GPS + gl), sgb = ld_shared_f32(scl + row_b * GPS + gl);
+            const float wg[4] = {sga * m0.y, sga * m1.y, sgb * m0.y, sgb * m1.y};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc0[r] = fmaf(pg[r] + ((r & 1) ? m1.x : m0.x), wg[r], acc0[r]);
+            if (MODE == 0) {
+                const float* su = scl + DC_ROWS * GPS;
+                const float sua = ld_shared_f32(su + row_a * GPS + gl), sub = ld_shared_f32(su + row_b * GPS + gl);
+                const float wu[4] = {sua * m0.y, sua * m1.y, sub * m0.y, sub * m1.y};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc1[r] = fmaf(pu[r] + ((r & 1) ? m1.x : m0.x), wu[r], acc1[r]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->empty[slot]);
+    }
+    return ok;
+}
+
 // One 8-block of a row's fp16 operands (the format act16_kernel describes):
-// 16 consecutive lanes hold one group of 128 values; every lane of the warp
-// takes part (its shuffles span each aligned half-warp), only `valid` lanes
-// store.
+// G / 8 consecutive lanes hold one group of G values; every lane of the warp
+// takes part (its shuffles stay inside aligned groups of G / 8 lanes), only
+// `valid` lanes store.  b is the 8-block's index in the row.
+template <int G>
 __device__ __forceinline__ void act16_block(const uint4 v, bool valid, __half* out16_row, float* meta_row, int b) {
+    constexpr int LPG = G / 8;   // lanes per group
     const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));   // the group's 16 lanes
+    for (int o = LPG / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     int e = 0;
     if (m > 0.0f) {
         e = int((__float_as_uint(m) >> 23) & 0xFF) - 127 - 14;
@@ -283,12 +382,16 @@ __device__ __forceinline__ void act16_block(const uint4 v, bool valid, __half* o
     }
     float cs = 1032.0f * ev + 1152.0f * od;
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    for (int o = LPG / 2; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
     if (valid) {
-        const int lc = b & 15, ci = lc >> 2, ii = lc & 3;
-        const int sb = (b & ~15) + 8 * (ii >> 1) + ci + 4 * (ii & 1);
+        const int lc = b % LPG;
+        int sb = b;   // groups of 64 / 32: 8-blocks in their natural order
+        if (G == kGroup) {   // groups of 128: 8-block 4 c + i stored at 8 (i >> 1) + c + 4 (i & 1)
+            const int ci = lc >> 2, ii = lc & 3;
+            sb = (b & ~15) + 8 * (ii >> 1) + ci + 4 * (ii & 1);
+        }
         *reinterpret_cast<uint4*>(out16_row + 8 * sb) = *reinterpret_cast<const uint4*>(h);
-        if (lc == 0) *reinterpret_cast<float2*>(meta_row + 2 * (b / 16)) = make_float2(-cs, __uint_as_float(uint32_t(127 + e) << 23));
+        if (lc == 0) *reinterpret_cast<float2*>(meta_row + 2 * (b / LPG)) = make_float2(-cs, __uint_as_float(uint32_t(127 + e) << 23));
     }
 }
 
@@ -309,8 +412,10 @@ __device__ __forceinline__ void act16_block(const uint4 v, bool valid, __half* o
 //     operands (act16_block), so no separate conversion pass is needed;
 //   down pass: out[t] rows of one 64-row block get one contribution from the
 //     shared expert and one per routed slot; the last of them writes
-//     out = bf16(y_s + sum_j y_r[slot j]), summed in that fixed order.
-template <int MODE>
+//     out = bf16(y_s + sum_j y_r[slot j]), summed in that fixed order (y_r
+//     may also come from the caller, by slot: then the shared expert's
+//     contribution is the only one).
+template <int MODE, int G>
 __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSmem* sm, const float* red, int hw,
                                                 int lane) {
     uint32_t it_base = 0;
@@ -327,12 +432,12 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
         // column values, lane l holding column l: in the down pass the token the
         // column belongs to and, for a routed column, its slot's gate
         float colgate = 1.0f;
-        int coltok = 0;
+        int coltok = 0, colslot = 0;
         if (MODE == 1 && lane < ti.count) {
             if (ti.kind == 1) {
-                const int slot = p.perm[ti.start + lane];
-                coltok = slot / p.k_top;
-                colgate = p.gates[slot];
+                colslot = p.perm[ti.start + lane];
+                coltok = colslot / p.k_top;
+                colgate = p.gates[colslot];
             } else {
                 coltok = ti.start + lane;
             }
@@ -340,6 +445,7 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
         if (!mbar_wait(&sm->red_full, tn & 1, p.status)) return;
         for (int col = hw; col < ti.count; col += DC_HELPERS) {
             const float gt = __shfl_sync(0xffffffffu, colgate, col);
+            const int yrow = p.y_by_slot ? __shfl_sync(0xffffffffu, colslot, col) : ti.start + col;
             const int nt = col >> 3, cn = col & 7;
             const int jc = ((cn & 3) << 1) | (cn >> 2);             // sigma8(jc) == cn
 #pragma unroll
@@ -371,7 +477,7 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
                     if (ti.kind == 1) p.h_r[int64_t(ti.start + col) * p.n_rows_r + n] = hv;
                     else p.h_s[int64_t(ti.start + col) * p.n_rows_s + n] = hv;
                 } else {
-                    if (ti.kind == 1) p.y_r[int64_t(ti.start + col) * p.n_rows_r + n] = v0 * gt;
+                    if (ti.kind == 1) p.y_r[int64_t(yrow) * p.n_rows_r + n] = v0 * gt;
                     else p.y_s[int64_t(ti.start + col) * p.n_rows_s + n] = v0;
                 }
             }
@@ -387,7 +493,23 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
         // ---- last writers: this warp's stores are made visible first ----
         const int n_mine = ti.count > hw ? (ti.count - hw + DC_HELPERS - 1) / DC_HELPERS : 0;
         const int mycol = hw + DC_HELPERS * lane;                    // lane j < n_mine: this warp's j-th column
-        if (MODE == 0 && ti.kind == 1) {
+        if (MODE == 0 && ti.kind == 1 && G != kGroup) {
+            // groups of 64 / 32: the task's 64 rows are whole groups -- convert this
+            // warp's columns at once, 4 per pass (8 lanes, the column's 8 8-blocks)
+            const int F = p.n_rows_r;
+            __threadfence();
+            __syncwarp();
+            for (int j0 = 0; j0 < n_mine; j0 += 4) {
+                const int j = j0 + (lane >> 3);
+                const bool valid = j < n_mine;
+                const int64_t pos = ti.start + hw + DC_HELPERS * (valid ? j : j0);
+                const int bb = (ti.row0 >> 3) + (lane & 7);                 // 8-block of the row
+                const uint4 v = valid ? __ldcg(reinterpret_cast<const uint4*>(p.h_r + pos * F + 8 * bb))
+                                      : make_uint4(0, 0, 0, 0);
+                act16_block<G>(v, valid, p.h16 + pos * F, p.h_meta + pos * act16_meta_pitch(F, G), bb);
+            }
+        }
+        if (MODE == 0 && ti.kind == 1 && G == kGroup) {
             const int F = p.n_rows_r, grp = ti.row0 >> 7;
             __threadfence();
             __syncwarp();
@@ -409,7 +531,7 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
                 const int bb = grp * 16 + (lane & 15);                  // 8-block of the row
                 const uint4 v = valid ? __ldcg(reinterpret_cast<const uint4*>(p.h_r + pos * F + 8 * bb))
                                       : make_uint4(0, 0, 0, 0);
-                act16_block(v, valid, p.h16 + pos * F, p.h_meta + pos * act16_meta_pitch(F), bb);
+                act16_block<G>(v, valid, p.h16 + pos * F, p.h_meta + pos * act16_meta_pitch(F, G), bb);
             }
         }
         if (MODE == 1 && p.out != nullptr) {
@@ -418,7 +540,7 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
             __threadfence();
             __syncwarp();
             bool last = false;
-            if (lane < n_mine) last = atomicAdd(&p.ocnt[int64_t(tok) * (D >> 6) + blk], 1) == p.k_top;
+            if (lane < n_mine) last = atomicAdd(&p.ocnt[int64_t(tok) * (D >> 6) + blk], 1) == p.n_contrib;
             uint32_t todo = __ballot_sync(0xffffffffu, last);
             if (todo) __threadfence();
             while (todo) {
@@ -429,8 +551,10 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
                 for (int half = 0; half < 2; ++half) {
                     const int n = ti.row0 + half * 32 + lane;
                     float a = __ldcg(p.y_s + t * D + n);
-                    for (int js = 0; js < p.k_top; ++js)
-                        a += __ldcg(p.y_r + int64_t(__ldcg(p.inv_perm + t * p.k_top + js)) * D + n);
+                    for (int js = 0; js < p.k_top; ++js) {
+                        const int64_t yr = p.inv_perm ? int64_t(__ldcg(p.inv_perm + t * p.k_top + js)) : t * p.k_top + js;
+                        a += __ldcg(p.y_r + yr * D + n);
+                    }
                     p.out[t * D + n] = __float2bfloat16_rn(a);
                 }
             }
@@ -438,14 +562,14 @@ __device__ __forceinline__ void decode_epilogue(const DecodeParams& p, DecodeSme
     }
 }
 
-template <int MODE>   // 0 = gate/up with SwiGLU, 1 = down
+template <int MODE, int G>   // MODE 0 = gate/up with SwiGLU, 1 = down; G = int4 group size (128, 64, 32)
 __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
     const __grid_constant__ CUtensorMap tm_r0, const __grid_constant__ CUtensorMap tm_r1,
     const __grid_constant__ CUtensorMap tm_s0, const __grid_constant__ CUtensorMap tm_s1,
     const __grid_constant__ CUtensorMap tm_br, const __grid_constant__ CUtensorMap tm_cr,
     const __grid_constant__ CUtensorMap tm_bs, const __grid_constant__ CUtensorMap tm_g0,
     const __grid_constant__ CUtensorMap tm_g1, DecodeParams p) {
-    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE), C_OFF = dc_c_off(MODE);
+    constexpr int NST = dc_nstages(MODE), SLOT = dc_slot(MODE, G), C_OFF = dc_c_off(MODE);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment of the ring is required by the 128-byte swizzle
     unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -485,6 +609,10 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
             uint32_t it = 0;
             bool ok = true, waited = false;
             int n_tasks = n_sh * nbs;   // grows by the routed tasks after the wait
+            // With an RMSNorm the shared-expert tasks' token rows are the router's
+            // xn: wait (bounded) until every router CTA has written its part.
+            if (MODE == 0 && p.xn_ready != nullptr && !wait_counter(p.xn_ready, p.xn_ready_target, p.status))
+                ok = false;
             for (uint32_t tn = 0; ok; ++tn) {
                 const int t = atomicAdd(p.task_counter, 1);
                 // Wait for the kernels before this one before the first load of
@@ -532,7 +660,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const CUtensorMap* m0 = ti.kind ? &tm_r0 : &tm_s0;
                 const CUtensorMap* m1 = ti.kind ? &tm_r1 : &tm_s1;
                 const int grow = ti.kind ? ti.expert * p.n_rows_r + ti.row0 : ti.row0;   // global tile row
-                if (ti.kind) {
+                if (ti.kind && G == kGroup) {
                     // one bulk copy per scale row, rows ldsc floats apart in
                     // shared memory so a warp's 8 rows fall in distinct banks
                     const int ng = ti.K / kGroup, ldsc = scale_row_floats(ng);
@@ -546,7 +674,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                         else                         // 64 rows at pitch ng: a multiple of 16 bytes
                             bulk_load(d, (m ? p.sc1 : p.sc0) + int64_t(grow) * ng, DC_ROWS * row_bytes, &sm->sfull[b]);
                     }
-                } else {
+                } else {   // shared expert, or groups of 64 / 32 (their scales come with the stages)
                     mbar_arrive(&sm->sfull[b]);
                 }
                 const int kbytes = ti.kind ? 128 : 64;   // tile x extent in elements (uint8 codes / bf16)
@@ -555,7 +683,13 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 const int kstage = (MODE == 0 ? 1 : 2) * kchunk;   // K values per stage
                 const int nbox = kstage / 64;
                 const uint32_t box_bytes = ti.kind ? 1024u : 2048u;
-                const uint32_t b_bytes = uint32_t(nbox) * box_bytes + (ti.kind ? 256u : 0u);
+                // routed stages: the token groups' (offset, scale) pairs (8 rows x 4
+                // groups of 128, or x the stage's groups of 64 / 32) and, for groups of
+                // 64 / 32, the weight scales of the stage's groups (64 rows per matrix)
+                constexpr int GPS = G == kGroup ? 4 : dc_kstage(MODE) / G;
+                const uint32_t meta_bytes = 8u * 2u * GPS * 4u;
+                const uint32_t scale_bytes = G == kGroup ? 0u : (MODE == 0 ? 2u : 1u) * DC_ROWS * GPS * 4u;
+                const uint32_t b_bytes = uint32_t(nbox) * box_bytes + (ti.kind ? meta_bytes + scale_bytes : 0u);
                 const CUtensorMap* mb = ti.kind ? &tm_br : &tm_bs;
                 for (int s = 0; s < ti.n_stages; ++s, ++it) {
                     const uint32_t slot = it % NST;
@@ -574,8 +708,14 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                     }
                     // one 3-D box: nbox 64-K chunks x the chunk's rows (chunks beyond K read zeros)
                     tma_load_3d(st + DC_B_OFF, mb, &sm->full[slot], 0, ti.start, s * kstage / 64);
-                    if (ti.kind)   // group (offset, scale) pairs: 4 groups from the stage's first, rounded down to a multiple of 4
+                    if (ti.kind && G == kGroup)   // 4 groups from the stage's first, rounded down to a multiple of 4
                         tma_load_2d(st + C_OFF, &tm_cr, &sm->full[slot], 2 * ((s * kstage / kGroup) & ~3), ti.start);
+                    if (ti.kind && G != kGroup) {   // exactly the stage's groups
+                        tma_load_2d(st + C_OFF, &tm_cr, &sm->full[slot], 2 * s * GPS, ti.start);
+                        unsigned char* sd = st + dc_s_off(MODE);
+                        tma_load_2d(sd, &tm_g0, &sm->full[slot], s * GPS, grow);
+                        if (MODE == 0) tma_load_2d(sd + DC_ROWS * GPS * 4, &tm_g1, &sm->full[slot], s * GPS, grow);
+                    }
                 }
             }
             // this grid completes only after the kernels before it
@@ -586,7 +726,7 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
                 mbar_wait(&sm->full[j % NST], (j / NST) & 1, nullptr);
             }
         } else if (warp >= 1 && warp <= DC_HELPERS) {
-            decode_epilogue<MODE>(p, sm, red, warp - 1, lane);
+            decode_epilogue<MODE, G>(p, sm, red, warp - 1, lane);
         }
         return;
     }
@@ -623,8 +763,12 @@ __global__ void __launch_bounds__(DC_THREADS, 1) decode_ffn_kernel(
         bool ok = true;
         if (ti.kind == 1) {
             // routed chunks hold at most 8 tokens: one n-tile
-            ok = consume_int4<MODE>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, p.f16_magic_lo, p.f16_magic_hi,
-                                   acc0[0], acc1[0], p.status);
+            if constexpr (G == kGroup)
+                ok = consume_int4<MODE, G>(ti, sm, ring, sc, it_base, q, lane, row_a, row_b, p.f16_magic_lo,
+                                           p.f16_magic_hi, acc0[0], acc1[0], p.status);
+            else
+                ok = consume_int4_qm<MODE, G>(ti, sm, ring, it_base, q, lane, row_a, row_b, p.f16_magic_lo,
+                                              p.f16_magic_hi, acc0[0], acc1[0], p.status);
         } else {
             // ---------------- bf16 weights (shared expert): 64 K per tile ----------------
             // thread c takes the 8-blocks c and c + 4 of each 64-K tile, of the
@@ -721,10 +865,14 @@ int decode_scale_pitch(int K) { return scale_rows_padded(K / kGroup) ? scale_row
 // rows, each row padded to scale_row_floats(K / 128)
 int decode_scale_floats(int mode, int K) { return (mode == 0 ? 2 : 1) * DC_ROWS * scale_row_floats(K / kGroup); }
 
-size_t decode_smem_bytes(int mode, int scale_buf_floats) {
-    return 1024 + size_t(dc_nstages(mode)) * dc_slot(mode) + 2 * size_t(scale_buf_floats) * 4 + DC_RED_FLOATS * 4 +
-           sizeof(DecodeSmem);
+size_t decode_smem_bytes(int mode, int scale_buf_floats, int G) {
+    return 1024 + size_t(dc_nstages(mode)) * dc_slot(mode, G) + 2 * size_t(scale_buf_floats) * 4 +
+           DC_RED_FLOATS * 4 + sizeof(DecodeSmem);
 }
+
+// groups of G per stage of a routed int4 task (4 for groups of 128: the
+// (offset, scale) box is 4 groups from the stage's first, rounded down)
+int decode_groups_per_stage(int mode, int G) { return G == kGroup ? 4 : dc_kstage(mode) / G; }
 
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launches
@@ -783,12 +931,14 @@ bool make_tmap_rows_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParams& prm, cudaStream_t stream) {
+moe_status launch_decode_ffn(int mode, int G, const DecodeMaps& maps, const DecodeParams& prm,
+                             cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = decode_smem_bytes(mode, prm.scale_buf_floats);
-    auto kern = mode == 0 ? decode_ffn_kernel<0> : decode_ffn_kernel<1>;
+    const size_t smem = decode_smem_bytes(mode, prm.scale_buf_floats, G);
+    auto kern = mode == 0 ? (G == 32 ? decode_ffn_kernel<0, 32> : G == 64 ? decode_ffn_kernel<0, 64> : decode_ffn_kernel<0, 128>)
+                          : (G == 32 ? decode_ffn_kernel<1, 32> : G == 64 ? decode_ffn_kernel<1, 64> : decode_ffn_kernel<1, 128>);
     if (allow_max_smem(kern) != MOE_OK) return MOE_ERR_CUDA;
     return launch_pdl(kern, dim3(sms), dim3(DC_THREADS), smem, stream, maps.r0, maps.r1, maps.s0, maps.s1, maps.br,
                       maps.cr, maps.bs, maps.g0, maps.g1, prm);
@@ -804,22 +954,25 @@ namespace moe {
 //
 // One CTA per output row of a bf16 matrix (the tokens x gathered into
 // expert-sorted position order, or the routed experts' hidden h, already by
-// position).  Each group of 128 values (16 threads, one 8-block each) gets
-// its own power of two:
+// position).  Each group of G values (the int4 group size: G / 8 threads, one
+// 8-block each) gets its own power of two:
 //   scale = 2^-e with e chosen from the group's largest magnitude so that the
 //           scaled values stay below 2^15 (fp16 keeps every bf16 value exactly
 //           in that range, down to 2^-24 of its largest);
 //   out16  every 8-block stored as x0 x4 x2 x6 x1/16 x5/16 x3/16 x7/16 (scaled)
 //          -- the K order and the 1/16 factors the int4 unpacking expects --
-//          and, inside each group of 128, 8-block 4 c + i (c, i = 0..3) stored
-//          at 8-block 8 (i >> 1) + c + 4 (i & 1), so that the four threads c
-//          of an MMA fragment read distinct shared-memory banks;
-//   meta   per group of 128, the pair (offset, 2^e): offset = -(1032 * sum of
+//          and, for groups of 128 only, inside each group 8-block 4 c + i
+//          (c, i = 0..3) stored at 8-block 8 (i >> 1) + c + 4 (i & 1), so that
+//          the four threads c of an MMA fragment read distinct shared-memory
+//          banks (the quarter-by-quarter MMAs of smaller groups read the
+//          8-blocks in their natural order without conflicts);
+//   meta   per group, the pair (offset, 2^e): offset = -(1032 * sum of
 //          the even-position stored values + 1152 * sum of the odd-position
 //          stored values), what the unpacked codes (1032 + q and 1152 + 16 q)
 //          add to a dot product, and 2^e, which undoes the scaling on the
-//          group's partial sum; rows of act16_meta_pitch(cols) floats.
+//          group's partial sum; rows of act16_meta_pitch(cols, G) floats.
 // ---------------------------------------------------------------------------
+template <int G>
 __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in, int cols,
                                                     const int32_t* __restrict__ src_perm, int k,
                                                     __half* __restrict__ out16, float* __restrict__ meta) {
@@ -828,19 +981,20 @@ __global__ void __launch_bounds__(256) act16_kernel(const bf16* __restrict__ in,
     const int64_t r = blockIdx.x;
     // out row r: input row src_perm[r] / k (tokens into expert-sorted positions), else row r
     const bf16* row = in + (src_perm ? int64_t(src_perm[r] / k) : r) * cols;
-    const int nblk = cols / 8;   // a multiple of 16: a group's 16 threads are all valid or all not
+    const int nblk = cols / 8;   // a multiple of 16: a group's threads are all valid or all not
     for (int b0 = 0; b0 < nblk; b0 += 256) {
         const int b = b0 + threadIdx.x;
         const bool valid = b < nblk;
         const uint4 v = valid ? *reinterpret_cast<const uint4*>(row + 8 * b) : make_uint4(0, 0, 0, 0);
-        act16_block(v, valid, out16 + r * cols, meta + r * act16_meta_pitch(cols), b);
+        act16_block<G>(v, valid, out16 + r * cols, meta + r * act16_meta_pitch(cols, G), b);
     }
 }
 
-moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
-                        float* meta, cudaStream_t stream) {
+moe_status launch_act16(const bf16* in, int64_t rows, int cols, int G, const int32_t* src_perm, int k,
+                        __half* out16, float* meta, cudaStream_t stream) {
     if (rows == 0) return MOE_OK;
-    return launch_pdl(act16_kernel, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, src_perm, k, out16, meta);
+    auto kern = G == 32 ? act16_kernel<32> : G == 64 ? act16_kernel<64> : act16_kernel<128>;
+    return launch_pdl(kern, dim3(unsigned(rows)), dim3(256), 0, stream, in, cols, src_perm, k, out16, meta);
 }
 
 }  // namespace moe

@@ -40,8 +40,12 @@ struct DecodeParams {
     float* h_meta;          //   and their per-group (offset, scale) pairs [T*k, act16_meta_pitch(F)]
     int32_t* hcnt;          //   token columns written per (position, group of 128 rows) [T*k, F / 128], zeroed
     bf16* out;              // down pass: the layer output [T, D] (null: none)
-    const int32_t* inv_perm;  // slot -> position
+    const int32_t* inv_perm;  // slot -> position of y_r's rows (null: y_r is stored by slot)
     int32_t* ocnt;          //   contributions written per (token, block of 64 rows) [T, D / 64], zeroed
+    int32_t n_contrib;      //   contributions before the last one (k, or 0 when y_r comes from the caller)
+    int32_t y_by_slot;      // down pass: routed y rows stored by slot (t * k + j) instead of by position
+    const int32_t* xn_ready;  // gate/up pass with an RMSNorm: the router CTAs that have written the
+    int32_t xn_ready_target;  //   normalized x the shared-expert tasks read (they start before the routing ends)
     int32_t* task_counter;  // cleared with the status word
     int32_t* status;        // device status word
 };
@@ -56,8 +60,13 @@ struct RoutePrep {
     int32_t* zero_words;  // zeroed by the bucketing kernel (or null)
     int32_t n_zero;
     bool router_after_kernel;   // the router may start while the kernel before it runs
-    float* router_part;         // router_partial_floats(T, D, E) floats for a K-split router (or null)
+    float* router_part;         // router_partial_floats(T, D, E, rms) floats for a K-split router (or null)
     int32_t* router_tile_cnt;   // ceil(T / 16) counters, zero on entry (with router_part)
+    const bf16* rms_weight;     // RMSNorm of x in the router (gamma [D]), or null
+    float rms_eps;
+    bf16* xn;                   // ... and where the router writes it, bf16 [T, D]
+    int32_t* xn_ready;          // ... counted by each router CTA once its part of xn is written (or null)
+    int32_t* status;            // device status word: out-of-range given expert ids are reported there
 };
 
 // TMA maps of one weight-streaming launch:
@@ -65,17 +74,20 @@ struct RoutePrep {
 //   s0, s1  shared bf16 weights, box 64 x 64, 128-B swizzle
 //   br      routed token rows, fp16 [T * k, K] by position (act16 layout), 3-D box of 8 rows x the
 //           stage's 64-K chunks (make_tmap_rows_3d)
-//   cr      their per-group (offset, scale) pairs, fp32 [T * k, act16_meta_pitch(K)], box 8 x 8
+//   cr      their per-group (offset, scale) pairs, fp32 [T * k, act16_meta_pitch(K, G)], box
+//           2 x decode_groups_per_stage floats x 8 rows
 //   bs      shared-expert token rows, bf16 [T, K] (x, or the shared h), 3-D box of 16 rows x chunks
-//   g0, g1  routed int4 scales fp32 [E * rows, K / 128] (gate, up; or down), box
-//           scale_row_floats(K / 128) x 64 (when K / 128 is a multiple of 4)
+//   g0, g1  routed int4 scales fp32 [E * rows, K / G] (gate, up; or down): groups of 128, box
+//           scale_row_floats(K / 128) x 64 (when K / 128 is a multiple of 4) for a task's rows;
+//           groups of 64 / 32, box (the stage's groups) x 64 rows, loaded with each stage
 struct DecodeMaps {
     CUtensorMap r0, r1, s0, s1, br, cr, bs, g0, g1;
 };
 
-// Row pitch (floats) of act16's per-group (offset, scale) pairs: K / 128
-// groups rounded up to 4, two floats each, so every row starts on 32 bytes.
-__host__ __device__ inline int act16_meta_pitch(int cols) { return int(ceil_div(cols / kGroup, 4) * 8); }
+// Row pitch (floats) of act16's per-group (offset, scale) pairs: K / G
+// groups (G = 128, 64 or 32) rounded up to 4, two floats each, so every row
+// starts on 32 bytes.
+__host__ __device__ inline int act16_meta_pitch(int cols, int G) { return int(ceil_div(cols / G, 4) * 8); }
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);
@@ -83,17 +95,23 @@ bool make_tmap_rows_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t ro
                        uint32_t nbox);
 int decode_scale_pitch(int K);
 int decode_max_chunks(int T, int k, int E);
-int router_ksplit(int T, int D);
-size_t router_partial_floats(int T, int D, int E);
-size_t decode_smem_bytes(int mode, int scale_buf_floats);
+int router_ksplit(int T, int D, bool rms);
+size_t router_partial_floats(int T, int D, int E, bool rms);
+size_t decode_smem_bytes(int mode, int scale_buf_floats, int G);
+int decode_groups_per_stage(int mode, int G);
 int decode_task_rows();
 int decode_scale_floats(int mode, int K);
-moe_status launch_decode_ffn(int mode, const DecodeMaps& maps, const DecodeParams& prm, cudaStream_t stream);
+moe_status launch_decode_ffn(int mode, int G, const DecodeMaps& maps, const DecodeParams& prm,
+                             cudaStream_t stream);
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between);
-moe_status launch_act16(const bf16* in, int64_t rows, int cols, const int32_t* src_perm, int k, __half* out16,
-                        float* meta, cudaStream_t stream);
+// The bucketing step alone, from given expert ids [T, k] (counts, offsets,
+// the stable permutation and, with `prep`, the FFN's chunk list).
+moe_status launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream);
+moe_status launch_act16(const bf16* in, int64_t rows, int cols, int G, const int32_t* src_perm, int k,
+                        __half* out16, float* meta, cudaStream_t stream);
 
 moe_status set_wait_limit_decode(uint32_t cycles);
 

@@ -72,13 +72,14 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     const int64_t T_pad = ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS;
     w.status = take(64);
     w.counters = take(64);   // task counters of the weight-streaming kernels
-    const bool rt_split = router_ksplit(int(T), L.D) > 1;
+    const bool rms = L.rms_weight != nullptr;
+    const bool rt_split = router_ksplit(int(T), L.D, rms) > 1;
     w.rt_cnt = take(rt_split ? size_t(ceil_div(T, 16)) * 4 : 0);   // router tile counters
     // weight-streaming path: the epilogues' last-writer counters, per (position,
     // group of 128 rows of h) and per (token, block of 64 output rows)
     w.dec_cnt = take(path == PATH_SEL_DECODE ? size_t(S * (L.F / 128) + T * (L.D / 64)) * 4 : 0);
     w.zeros_end = off;   // [status, zeros_end) is cleared at the start of every call
-    w.rt_part = take(router_partial_floats(int(T), L.D, L.E) * 4);
+    w.rt_part = take(router_partial_floats(int(T), L.D, L.E, rms) * 4);
     w.ids = take(S * 4);
     w.gates = take(S * 4);
     w.counts = take(size_t(L.E) * 4);
@@ -91,10 +92,10 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.common_end = off;
     if (path == PATH_SEL_DECODE) {
         w.x16 = take(S * L.D * 2);                 // tokens by expert-sorted position
-        w.x_meta = take(S * act16_meta_pitch(L.D) * 4);
+        w.x_meta = take(S * act16_meta_pitch(L.D, L.group_size) * 4);
         w.h_r = take(S * L.F * 2);
         w.h16 = take(S * L.F * 2);
-        w.h_meta = take(S * act16_meta_pitch(L.F) * 4);
+        w.h_meta = take(S * act16_meta_pitch(L.F, L.group_size) * 4);
         w.h_s = take(T * L.F_shared * 2);
         w.y_r = take(S * L.D * 4);
         w.y_s = take(T * L.D * 4);
@@ -131,13 +132,18 @@ size_t ws_bytes(const moe_layer_desc& L, int64_t T) {
     return a > b ? a : b;
 }
 
-// The weight-streaming kernels keep a task's int4 scales in shared memory,
-// and their MMAs sum whole groups of 128 K before scaling: smaller groups
-// run on the tensor-core tiles only.
+// Whether the weight-streaming kernels take this layer.  Groups of 128 keep
+// a task's scales in shared memory (it must fit); groups of 64 / 32 load
+// each stage's scales with it, as a TMA box of the stage's groups (at least
+// as many as a row has) whose rows (K / G scales) must be whole 16-byte units.
 bool decode_fits(const moe_layer_desc& L) {
-    if (L.format == MOE_WEIGHTS_INT4_G128 && L.group_size != 128) return false;
-    return decode_smem_bytes(0, decode_scale_floats(0, L.D)) <= kMaxDecodeSmem &&
-           decode_smem_bytes(1, decode_scale_floats(1, L.F)) <= kMaxDecodeSmem;
+    const int G = L.group_size;
+    if (L.format == MOE_WEIGHTS_INT4_G128 && G != 128)
+        return (L.D / G) % 4 == 0 && (L.F / G) % 4 == 0 && L.D / G >= decode_groups_per_stage(0, G) &&
+               L.F / G >= decode_groups_per_stage(1, G) && decode_smem_bytes(0, 0, G) <= kMaxDecodeSmem &&
+               decode_smem_bytes(1, 0, G) <= kMaxDecodeSmem;
+    return decode_smem_bytes(0, decode_scale_floats(0, L.D), 128) <= kMaxDecodeSmem &&
+           decode_smem_bytes(1, decode_scale_floats(1, L.F), 128) <= kMaxDecodeSmem;
 }
 
 int choose_path(const moe_layer_desc& L, int64_t T) {
@@ -213,8 +219,27 @@ bool same_key(const MapCacheKey& a, const MapCacheKey& b) {
            a.T == b.T && a.path == b.path;
 }
 
-moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
-                           const WsLayout& W, cudaStream_t st, Marks& mk) {
+// With an RMSNorm the router normalizes x itself and writes xn to the
+// workspace for the kernels after it; counters[2] counts its CTAs once done.
+void set_rms(RoutePrep& prep, const moe_layer_desc& L, void* ws, const WsLayout& W) {
+    if (!L.rms_weight) return;
+    prep.rms_weight = static_cast<const bf16*>(L.rms_weight);
+    prep.rms_eps = L.rms_eps;
+    prep.xn = at<bf16>(ws, W.xn);
+    prep.xn_ready = at<int32_t>(ws, W.counters) + 2;
+}
+
+// Rows whose expert and gate the caller gives (the routed experts alone: the
+// compute step of an expert-parallel layer).  The router and the shared
+// expert are skipped and each row's gate-scaled output goes to y by row.
+struct PreRouted {
+    const int32_t* ids;   // [T] expert of each row
+    const float* gates;   // [T]
+    float* y;             // [T, D] fp32
+};
+
+moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, const bf16* xin, int T, bf16* out, void* ws,
+                           const WsLayout& W, cudaStream_t st, Marks& mk, const PreRouted* pr = nullptr) {
     int32_t* status = at<int32_t>(ws, W.status);
     int32_t* counters = at<int32_t>(ws, W.counters);
     int32_t* perm = at<int32_t>(ws, W.perm);
@@ -233,7 +258,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     // (programmatic dependent launch) and waits before reading its outputs.
     RoutePrep prep;
     memset(&prep, 0, sizeof(prep));
-    if (W.rt_cnt != W.zeros_end) {   // K-split router (few token tiles)
+    if (router_ksplit(T, L.D, L.rms_weight != nullptr) > 1) {   // K-split router (few token tiles)
         prep.router_part = at<float>(ws, W.rt_part);
         prep.router_tile_cnt = at<int32_t>(ws, W.rt_cnt);
     }
@@ -245,14 +270,23 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     prep.chunk_tokens = 16;
     prep.routed_chunk_tokens = 8;   // one 8-column n-tile per routed chunk
     prep.router_after_kernel = false;
-    mk.mark(st);
-    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
-                     at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
-                     &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
-    ++mk.i;
+    set_rms(prep, L, ws, W);
+    moe_status s;
+    if (pr) {   // the rows' experts are given: bucketing only
+        prep.status = at<int32_t>(ws, W.status);
+        s = launch_bucket(pr->ids, T, 1, L.E, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
+                          &prep, st);
+        gates = const_cast<float*>(pr->gates);
+    } else {
+        mk.mark(st);
+        s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+                         at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm,
+                         inv, &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
+        ++mk.i;
+    }
     if (s != MOE_OK) return s;
     mk.mark(st);
-    s = launch_act16(x, S, L.D, perm, L.k, at<__half>(ws, W.x16), at<float>(ws, W.x_meta), st);
+    s = launch_act16(xin, S, L.D, L.group_size, perm, L.k, at<__half>(ws, W.x16), at<float>(ws, W.x_meta), st);
     if (s != MOE_OK) return s;
 
     // tensor maps: built once per (layer, workspace, input, T) and thread
@@ -264,26 +298,37 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
         auto build = [&](DecodeMaps& m1, DecodeMaps& m2) -> bool {
         const uint64_t E = uint64_t(L.E);
         const uint32_t rows = uint32_t(decode_task_rows());
+        const int G = L.group_size;
         // weights; token rows (8 per routed chunk, 16 per shared chunk) and group offsets
         bool ok = make_tmap_2d(&m1.r0, L.w_gate, 1, L.D / 2, E * L.F, 128, rows, true) &&
                   make_tmap_2d(&m1.r1, L.w_up, 1, L.D / 2, E * L.F, 128, rows, true) &&
                   make_tmap_2d(&m1.s0, L.ws_gate, 2, L.D, L.F_shared, 64, rows, true) &&
                   make_tmap_2d(&m1.s1, L.ws_up, 2, L.D, L.F_shared, 64, rows, true) &&
                   make_tmap_rows_3d(&m1.br, at<__half>(ws, W.x16), L.D, S, 8, 4) &&
-                  make_tmap_2d(&m1.cr, at<float>(ws, W.x_meta), 4, act16_meta_pitch(L.D), S, 8, 8, false) &&
-                  make_tmap_rows_3d(&m1.bs, x, L.D, T, 16, 1) &&
+                  make_tmap_2d(&m1.cr, at<float>(ws, W.x_meta), 4, act16_meta_pitch(L.D, G), S,
+                               2 * decode_groups_per_stage(0, G), 8, false) &&
+                  make_tmap_rows_3d(&m1.bs, xin, L.D, T, 16, 1) &&
                   make_tmap_2d(&m2.r0, L.w_down, 1, L.F / 2, E * L.D, 128, rows, true) &&
                   make_tmap_2d(&m2.s0, L.ws_down, 2, L.F_shared, L.D, 64, rows, true) &&
                   make_tmap_rows_3d(&m2.br, at<__half>(ws, W.h16), L.F, S, 8, 8) &&
-                  make_tmap_2d(&m2.cr, at<float>(ws, W.h_meta), 4, act16_meta_pitch(L.F), S, 8, 8, false) &&
+                  make_tmap_2d(&m2.cr, at<float>(ws, W.h_meta), 4, act16_meta_pitch(L.F, G), S,
+                               2 * decode_groups_per_stage(1, G), 8, false) &&
                   make_tmap_rows_3d(&m2.bs, h_s, L.F_shared, T, 16, 2);
-        // the task scales: one box per matrix when their rows are whole 16-byte units
-        const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
-        if (pd) ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / kGroup, E * L.F, pd, rows, false) &&
-                     make_tmap_2d(&m1.g1, L.s_up, 4, L.D / kGroup, E * L.F, pd, rows, false);
-        else m1.g0 = m1.g1 = m1.r0;   // unused: the scales come by bulk copy
-        if (pf) ok = ok && make_tmap_2d(&m2.g0, L.s_down, 4, L.F / kGroup, E * L.D, pf, rows, false);
-        else m2.g0 = m2.r0;
+        if (G == 128) {
+            // the task scales: one box per matrix when their rows are whole 16-byte units
+            const int pd = decode_scale_pitch(L.D), pf = decode_scale_pitch(L.F);
+            if (pd) ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / kGroup, E * L.F, pd, rows, false) &&
+                         make_tmap_2d(&m1.g1, L.s_up, 4, L.D / kGroup, E * L.F, pd, rows, false);
+            else m1.g0 = m1.g1 = m1.r0;   // unused: the scales come by bulk copy
+            if (pf) ok = ok && make_tmap_2d(&m2.g0, L.s_down, 4, L.F / kGroup, E * L.D, pf, rows, false);
+            else m2.g0 = m2.r0;
+        } else {
+            // groups of 64 / 32: each stage's scales, (the stage's groups) x 64 rows
+            const uint32_t g0 = uint32_t(decode_groups_per_stage(0, G)), g1 = uint32_t(decode_groups_per_stage(1, G));
+            ok = ok && make_tmap_2d(&m1.g0, L.s_gate, 4, L.D / G, E * L.F, g0, rows, false) &&
+                 make_tmap_2d(&m1.g1, L.s_up, 4, L.D / G, E * L.F, g0, rows, false) &&
+                 make_tmap_2d(&m2.g0, L.s_down, 4, L.F / G, E * L.D, g1, rows, false);
+        }
         if (!ok) return false;
         m2.r1 = m2.r0;
         m2.s1 = m2.s0;
@@ -304,7 +349,7 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.K_r = L.D;
     p.K_s = L.D;
     p.k_top = L.k;
-    p.scale_buf_floats = decode_scale_floats(0, L.D);
+    p.scale_buf_floats = L.group_size == 128 ? decode_scale_floats(0, L.D) : 0;
     p.f16_magic_lo = kF16MagicLo;
     p.f16_magic_hi = kF16MagicHi;
     p.chunks = chunks;
@@ -318,27 +363,39 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, int T, bf16* 
     p.h16 = at<__half>(ws, W.h16);      // the gate/up epilogue also writes h's fp16 operands
     p.h_meta = at<float>(ws, W.h_meta);
     p.hcnt = at<int32_t>(ws, W.dec_cnt);
+    if (L.rms_weight) {   // the shared-expert tasks read the router's xn: wait for all its CTAs
+        p.xn_ready = counters + 2;
+        p.xn_ready_target = int32_t(ceil_div(T, 16)) * router_ksplit(T, L.D, true);
+    }
     p.task_counter = counters;
     p.status = status;
+    if (pr) p.n_rows_s = 0;   // no shared-expert tasks
     mk.mark(st);
-    s = launch_decode_ffn(0, m1, p, st);
+    s = launch_decode_ffn(0, L.group_size, m1, p, st);
     if (s != MOE_OK) return s;
 
     p.n_rows_r = L.D;
     p.n_rows_s = L.D;
     p.K_r = L.F;
     p.K_s = L.F_shared;
-    p.scale_buf_floats = decode_scale_floats(1, L.F);
+    p.scale_buf_floats = L.group_size == 128 ? decode_scale_floats(1, L.F) : 0;
     p.sc0 = L.s_down;
     p.sc1 = nullptr;
     p.y_r = y_r;
     p.y_s = y_s;
     p.out = out;                        // the down epilogue finishes each token
     p.inv_perm = inv;
+    p.n_contrib = L.k;
     p.ocnt = at<int32_t>(ws, W.dec_cnt) + S * (L.F / 128);
     p.task_counter = counters + 1;
+    if (pr) {   // gate-scaled y of each row, by row; no shared expert, no combine
+        p.n_rows_s = 0;
+        p.y_r = pr->y;
+        p.y_by_slot = 1;
+        p.out = nullptr;
+    }
     mk.mark(st);
-    s = launch_decode_ffn(1, m2, p, st);
+    s = launch_decode_ffn(1, L.group_size, m2, p, st);
     mk.mark(st);
     return s;
 }
@@ -362,23 +419,15 @@ int prefill_launches(const moe_layer_desc& L, const char** names, int max_names)
     return n;
 }
 
-// The kernels one forward launches, in order: the RMSNorm (if the layer has
-// one), then the path's kernels.
+// The kernels one forward launches, in order (an RMSNorm runs inside the router).
 int32_t layer_launch_names(const moe_layer_desc& L, int64_t T, const char** names, int32_t max_names) {
-    int32_t n = 0;
-    if (L.rms_weight) {
-        if (names && max_names > 0) names[0] = "rmsnorm";
-        n = 1;
-    }
-    const char** rest = (names && max_names > n) ? names + n : nullptr;
-    const int32_t max_rest = max_names > n ? max_names - n : 0;
-    if (choose_path(L, T) != PATH_SEL_DECODE) return n + prefill_launches(L, rest, max_rest);
-    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_rest && rest; ++i) rest[i] = kDecodeLaunches[i];
-    return n + kDecodeLaunchCount;
+    if (choose_path(L, T) != PATH_SEL_DECODE) return prefill_launches(L, names, max_names);
+    for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
+    return kDecodeLaunchCount;
 }
 
-moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16* out, void* ws,
-                            const WsLayout& W, cudaStream_t st, Marks& mk) {
+moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, const bf16* xin, int T, bf16* out, void* ws,
+                            const WsLayout& W, cudaStream_t st, Marks& mk, const PreRouted* pr = nullptr) {
     int32_t* status = at<int32_t>(ws, W.status);
     int32_t* perm = at<int32_t>(ws, W.perm);
     int32_t* inv = at<int32_t>(ws, W.inv_perm);
@@ -399,20 +448,28 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     prep.n_chunks = nch;
     prep.chunk_tokens = TC_BLOCK_TOKENS;
     prep.routed_chunk_tokens = TC_BLOCK_TOKENS;
-    mk.mark(st);
-    moe_status s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
-                                at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts),
-                                at<int32_t>(ws, W.offsets), perm, inv, &prep, st,
-                                (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
-    ++mk.i;
+    set_rms(prep, L, ws, W);
+    moe_status s;
+    if (pr) {   // the rows' experts are given: bucketing only
+        prep.status = at<int32_t>(ws, W.status);
+        s = launch_bucket(pr->ids, T, 1, L.E, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm, inv,
+                          &prep, st);
+        gates = const_cast<float*>(pr->gates);
+    } else {
+        mk.mark(st);
+        s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
+                         at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm,
+                         inv, &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
+        ++mk.i;
+    }
     if (s != MOE_OK) return s;
     mk.mark(st);
     const bool fp8 = L.format == MOE_WEIGHTS_FP8_ROW;
     if (fp8)   // e4m3 rows of x, written to each token's slot positions
-        s = launch_quantize_fp8_scatter(x, T, L.D, L.act_scale_ub, inv, L.k, at<uint8_t>(ws, W.xq),
+        s = launch_quantize_fp8_scatter(xin, T, L.D, L.act_scale_ub, inv, L.k, at<uint8_t>(ws, W.xq),
                                         at<float>(ws, W.xq_scale), st);
     else
-        s = launch_gather_rows(x, perm, S, L.k, L.D, x_sorted, st);
+        s = launch_gather_rows(xin, perm, S, L.k, L.D, x_sorted, st);
     if (s != MOE_OK) return s;
 
     static thread_local MapCacheKey pkey;
@@ -437,7 +494,7 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
                  make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
         // the shared expert's token tiles come straight from x: a 256-row box that
         // runs past row T - 1 reads zeros there
-        ok = ok && make_tmap_2d(&m_sgu.b, x, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
+        ok = ok && make_tmap_2d(&m_sgu.b, xin, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
                   make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
@@ -468,18 +525,20 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.status = status;
     float* y_shared = at<float>(ws, W.y_shared);
 
-    // shared gate/up -> h_s (bf16, natural order, by token)
-    p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
-    p.h_out = h_s;
-    mk.mark(st);
-    s = launch_tc_gemm(TC_GATEUP_BF16, m_sgu, p, st);
-    if (s != MOE_OK) return s;
-    // shared down -> y_s (fp32, by token)
-    p.K = L.F_shared; p.n_rows = L.D; p.n_fblocks = L.D / 128;
-    p.h_out = nullptr; p.y_out = y_shared;
-    mk.mark(st);
-    s = launch_tc_gemm(TC_DOWN_BF16, m_sdn, p, st);
-    if (s != MOE_OK) return s;
+    if (!pr) {   // (rows with given experts: no shared expert)
+        // shared gate/up -> h_s (bf16, natural order, by token)
+        p.K = L.D; p.n_rows = L.F_shared; p.n_fblocks = L.F_shared / 64; p.routed = 0;
+        p.h_out = h_s;
+        mk.mark(st);
+        s = launch_tc_gemm(TC_GATEUP_BF16, m_sgu, p, st);
+        if (s != MOE_OK) return s;
+        // shared down -> y_s (fp32, by token)
+        p.K = L.F_shared; p.n_rows = L.D; p.n_fblocks = L.D / 128;
+        p.h_out = nullptr; p.y_out = y_shared;
+        mk.mark(st);
+        s = launch_tc_gemm(TC_DOWN_BF16, m_sdn, p, st);
+        if (s != MOE_OK) return s;
+    }
     // routed gate/up -> h (bf16 by slot position; int4: fragment order, e4m3: natural order)
     p.K = L.D; p.n_rows = L.F; p.n_fblocks = L.F / 64; p.routed = 1;
     p.s0 = L.s_gate; p.s1 = L.s_up; p.h_out = h_sorted; p.y_out = nullptr;
@@ -498,11 +557,13 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, int T, bf16*
     p.K = L.F; p.n_rows = L.D; p.n_fblocks = L.D / 128;
     p.s0 = L.s_down; p.s1 = nullptr; p.h_out = nullptr;
     p.tok_scale = fp8 ? at<float>(ws, W.hq_scale) : nullptr;
-    if (L.k == 1) { p.out = out; p.y_r = y_shared; p.y_out = nullptr; }
+    if (pr) { p.out = nullptr; p.y_r = nullptr; p.y_out = pr->y; }   // gate * y by row
+    else if (L.k == 1) { p.out = out; p.y_r = y_shared; p.y_out = nullptr; }
     else { p.out = nullptr; p.y_r = nullptr; p.y_out = y_pos; }
     mk.mark(st);
     s = launch_tc_gemm(fp8 ? TC_DOWN_FP8 : TC_DOWN_INT4, m_dn, p, st);
     if (s != MOE_OK) return s;
+    if (pr) return MOE_OK;
     if (L.k > 1) {
         mk.mark(st);
         s = launch_combine_slots(y_shared, y_pos, T, L.D, L.k, out, st);
@@ -527,17 +588,13 @@ moe_status ffn_forward_impl(const moe_layer_desc* layer, const void* x, int32_t 
     // the device status word and the zero rows read in place of missing tokens
     if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
         return MOE_ERR_CUDA;
-    const bf16* xin = static_cast<const bf16*>(x);
-    if (layer->rms_weight) {   // the block's RMSNorm first; the layer reads its result
-        mk.mark(st);
-        s = launch_rmsnorm(xin, T, layer->D, static_cast<const bf16*>(layer->rms_weight), layer->rms_eps,
-                           at<bf16>(workspace, W.xn), st);
-        if (s != MOE_OK) return s;
-        xin = at<bf16>(workspace, W.xn);
-    }
+    // With the block's RMSNorm the router normalizes x on the way and writes
+    // xn; every kernel after it reads xn.
+    const bf16* xr = static_cast<const bf16*>(x);
+    const bf16* xin = layer->rms_weight ? at<bf16>(workspace, W.xn) : xr;
     if (path == PATH_SEL_DECODE)
-        return ffn_decode_path(*layer, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
-    return ffn_prefill_path(*layer, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
+        return ffn_decode_path(*layer, xr, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
+    return ffn_prefill_path(*layer, xr, xin, T, static_cast<bf16*>(out), workspace, W, st, mk);
 }
 
 }  // namespace
@@ -659,7 +716,7 @@ moe_status moe_ffn_device_status(const void* workspace, void* stream) {
     cudaStream_t st = as_stream(stream);
     if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
-    return v == DEV_OK ? MOE_OK : MOE_ERR_TIMEOUT;
+    return v == DEV_OK ? MOE_OK : v == DEV_BAD_EXPERT ? MOE_ERR_INVALID_ARG : MOE_ERR_TIMEOUT;
 }
 
 }  // extern "C"
@@ -837,8 +894,11 @@ bool same_dense_key(const DenseKey& a, const DenseKey& b) {
            a.T == b.T && a.path == b.path;
 }
 
+// y_add (fp32 [T, k_add, D], or null): outputs of each token's k_add routed
+// slots, added in slot order (the shared-expert half of an expert-parallel
+// MoE layer): out = bf16(ffn(x) + sum_j y_add[t, j]).
 moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_t T, void* out, void* ws,
-                              size_t ws_bytes, cudaStream_t st) {
+                              size_t ws_bytes, cudaStream_t st, const float* y_add = nullptr, int k_add = 0) {
     moe_status s = check_dense(layer);
     if (s != MOE_OK) return s;
     const moe_dense_desc& L = *layer;
@@ -892,7 +952,9 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         p.n_rows_s = L.F;
         p.K_r = L.D;
         p.K_s = L.D;
-        p.k_top = 0;   // no routed slots: the shared expert's contribution is each output's only one
+        p.k_top = y_add ? k_add : 0;   // routed outputs by slot, if any, are given: the shared
+        p.n_contrib = 0;                 // expert's contribution is each output's only one
+        p.y_r = const_cast<float*>(y_add);
         p.scale_buf_floats = 0;
         p.f16_magic_lo = kF16MagicLo;
         p.f16_magic_hi = kF16MagicHi;
@@ -901,7 +963,7 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         p.h_s = h;
         p.task_counter = at<int32_t>(ws, W.counters);
         p.status = status;
-        s = launch_decode_ffn(0, m1, p, st);
+        s = launch_decode_ffn(0, 128, m1, p, st);
         if (s != MOE_OK) return s;
         p.n_rows_s = L.D;
         p.K_r = L.F;
@@ -910,7 +972,7 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
         p.out = static_cast<bf16*>(out);
         p.ocnt = at<int32_t>(ws, W.ocnt);
         p.task_counter = at<int32_t>(ws, W.counters) + 1;
-        return launch_decode_ffn(1, m2, p, st);
+        return launch_decode_ffn(1, 128, m2, p, st);
     }
 
     const uint64_t T_pad = uint64_t(ceil_div(T, TC_BLOCK_TOKENS) * TC_BLOCK_TOKENS);
@@ -944,7 +1006,7 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
     p.h_out = nullptr; p.y_out = y;
     s = launch_tc_gemm(TC_DOWN_BF16, md, p, st);
     if (s != MOE_OK) return s;
-    return launch_combine_slots(y, nullptr, T, L.D, 0, static_cast<bf16*>(out), st);
+    return launch_combine_slots(y, y_add, T, L.D, y_add ? k_add : 0, static_cast<bf16*>(out), st);
 }
 
 }  // namespace
@@ -961,3 +1023,76 @@ extern "C" moe_status moe_dense_ffn_forward(const moe_dense_desc* layer, const v
                                             void* workspace, size_t workspace_bytes, void* stream) {
     return dense_forward_impl(layer, x, T, out, workspace, workspace_bytes, as_stream(stream));
 }
+
+// ---- expert parallelism: the routed experts on given rows; the shared
+// expert plus the combine of given routed outputs ----
+namespace {
+moe_layer_desc one_slot_layer(const moe_layer_desc& L) {
+    moe_layer_desc L1 = L;   // rows with one expert each, no RMSNorm (the rows arrive normalized)
+    L1.k = 1;
+    L1.rms_weight = nullptr;
+    return L1;
+}
+
+moe_dense_desc shared_as_dense(const moe_layer_desc& L) {
+    moe_dense_desc d;
+    memset(&d, 0, sizeof(d));
+    d.D = L.D;
+    d.F = L.F_shared;
+    d.path = L.path;
+    d.w_gate = L.ws_gate;
+    d.w_up = L.ws_up;
+    d.w_down = L.ws_down;
+    d.rms_weight = L.rms_weight;
+    d.rms_eps = L.rms_eps;
+    return d;
+}
+}  // namespace
+
+extern "C" size_t moe_expert_ffn_workspace_size(const moe_layer_desc* layer, int32_t n_max) {
+    if (check_layer(layer) != MOE_OK || n_max < 1 || n_max > kMaxT) return 0;
+    return ws_bytes(one_slot_layer(*layer), n_max);
+}
+
+extern "C" moe_status moe_expert_ffn_forward(const moe_layer_desc* layer, const void* x, int32_t n,
+                                             const int32_t* expert_ids, const float* gates, float* y,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+    moe_status s = check_layer(layer);
+    if (s != MOE_OK) return s;
+    const moe_layer_desc L = one_slot_layer(*layer);
+    s = check_route_shape(n, L.D, L.E, 1);
+    if (s != MOE_OK) return s;
+    const void* ptrs[] = {x, expert_ids, gates, y, workspace};
+    for (const void* ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return MOE_ERR_INVALID_ARG;
+    const int path = choose_path(L, n);
+    const WsLayout W = ws_layout(L, n, path);
+    if (workspace_bytes < W.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (path == PATH_SEL_DECODE && !decode_fits(L)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemsetAsync(at<int32_t>(workspace, W.status), 0, W.zeros_end - W.status, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    PreRouted pr{expert_ids, gates, y};
+    Marks mk;
+    const bf16* xr = static_cast<const bf16*>(x);
+    if (path == PATH_SEL_DECODE) return ffn_decode_path(L, xr, xr, n, nullptr, workspace, W, st, mk, &pr);
+    return ffn_prefill_path(L, xr, xr, n, nullptr, workspace, W, st, mk, &pr);
+}
+
+extern "C" size_t moe_shared_ffn_workspace_size(const moe_layer_desc* layer, int32_t T_max) {
+    if (check_layer(layer) != MOE_OK) return 0;
+    const moe_dense_desc d = shared_as_dense(*layer);
+    return moe_dense_ffn_workspace_size(&d, T_max);
+}
+
+extern "C" moe_status moe_shared_ffn_combine(const moe_layer_desc* layer, const void* x, int32_t T,
+                                             const float* y_slots, void* out, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+    moe_status s = check_layer(layer);
+    if (s != MOE_OK) return s;
+    if (!y_slots || !aligned16(y_slots)) return MOE_ERR_INVALID_ARG;
+    const moe_dense_desc d = shared_as_dense(*layer);
+    return dense_forward_impl(&d, x, T, out, workspace, workspace_bytes, as_stream(stream), y_slots, layer->k);
+}
+

@@ -48,9 +48,11 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     const bf16* __restrict__ x, int T, int D, const bf16* __restrict__ wr,
     const float* __restrict__ bias, int E, int k, int32_t* __restrict__ ids,
     float* __restrict__ gates, bf16* __restrict__ x_frag, int ksplit, float* __restrict__ part_g,
-    int32_t* __restrict__ tile_cnt) {
+    int32_t* __restrict__ tile_cnt, const bf16* __restrict__ gamma, float rms_eps, bf16* __restrict__ xn,
+    int32_t* __restrict__ xn_ready) {
     extern __shared__ __align__(16) float part[];     // [nw][RT_TOK][E]
     __shared__ int s_last;
+    __shared__ float s_ss[RT_TOK], s_inv[RT_TOK];
     griddep_launch_dependents();
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -63,6 +65,68 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
     const bool row_a = t0 + g < T, row_b = t0 + g + 8 < T;
     const bf16* xa_row = x + int64_t(t0 + g) * D;
     const bf16* xb_row = x + int64_t(t0 + g + 8) * D;
+
+    if (gamma != nullptr) {
+        // RMSNorm of the tile's rows first ("Llama 开源模型系列", "RMSNorm：为什么
+        // 去掉减均值也能工作"): each CTA sums the squares over its own K range
+        // (a warp per row, lanes over 8-value chunks, a fixed shuffle tree), the
+        // tile's CTAs -- one thread-block cluster -- add the ksplit partial sums
+        // in rank (K range) order through distributed shared memory, so every
+        // CTA holds the same r = 1 / sqrt(sum / D + eps).  The GEMV below runs on
+        // xn = bf16((x * r) * gamma), which the CTA first writes out for the
+        // kernels after the router.
+        const int k0 = blockIdx.y * groups_per_cta * kGroup, nb = groups_per_cta * kGroup / 8;
+        for (int r = warp; r < RT_TOK; r += nw) {
+            float ss = 0.0f;
+            if (t0 + r < T) {
+                const bf16* row = x + int64_t(t0 + r) * D + k0;
+                for (int b = lane; b < nb; b += 32) {
+                    const uint4 v = ldg_cached(row + 8 * b);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float a = bf16_lo(w[i]), h = bf16_hi(w[i]);
+                        ss = fmaf(a, a, ss);
+                        ss = fmaf(h, h, ss);
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (lane == 0) s_ss[r] = ss;
+        }
+        cluster_sync();
+        if (threadIdx.x < RT_TOK) {
+            float tot = 0.0f;
+            for (int rk = 0; rk < ksplit; ++rk) tot += ld_dsmem_f32(&s_ss[threadIdx.x], rk);
+            s_inv[threadIdx.x] = t0 + int(threadIdx.x) < T ? 1.0f / sqrtf(tot / float(D) + rms_eps) : 0.0f;
+        }
+        cluster_sync();   // every CTA has read the others' sums; s_inv is visible
+    }
+    // x -> xn = bf16((x * r) * gamma) for 8 values of one row
+    auto rms_apply = [&](uint4 v, float r, uint4 gm) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w}, gw[4] = {gm.x, gm.y, gm.z, gm.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = pack_bf16x2((bf16_lo(w[i]) * r) * bf16_lo(gw[i]), (bf16_hi(w[i]) * r) * bf16_hi(gw[i]));
+        return make_uint4(o[0], o[1], o[2], o[3]);
+    };
+    if (gamma != nullptr) {
+        // this CTA's part of xn (the tile's rows over its K range) goes out
+        // first, and is counted, so kernels that need only xn can start before
+        // the GEMV below has finished
+        const int k0 = blockIdx.y * groups_per_cta * kGroup, nb = groups_per_cta * kGroup / 8;
+        for (int idx = threadIdx.x; idx < RT_TOK * nb; idx += blockDim.x) {
+            const int r = idx / nb, kk = k0 + 8 * (idx % nb);
+            if (t0 + r >= T) continue;
+            const uint4 v = ldg_cached(x + int64_t(t0 + r) * D + kk);
+            *reinterpret_cast<uint4*>(xn + int64_t(t0 + r) * D + kk) = rms_apply(v, s_inv[r], ldg_cached(gamma + kk));
+        }
+        __threadfence();
+        __syncthreads();
+        if (xn_ready != nullptr && threadIdx.x == 0) atomicAdd(xn_ready, 1);
+    }
 
     for (int e0 = 0; e0 < E; e0 += RT_EPASS) {
         float acc[8][4];
@@ -86,6 +150,11 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
         load(k_begin, xa, xb, wv);
         for (int kk = k_begin; kk < k_end; kk += 32) {
             if (kk + 32 < k_end) load(kk + 32, nxa, nxb, nwv);
+            if (gamma != nullptr) {   // the same xn values as written out above
+                const uint4 gm = ldg_cached(gamma + kk + 8 * c);
+                xa = rms_apply(xa, s_inv[g], gm);
+                xb = rms_apply(xb, s_inv[g + 8], gm);
+            }
             // thread (g, c) holds K values kk + 8c .. kk + 8c + 7 of rows g and g + 8;
             // the two MMAs below use them as K pairs (0,1)(2,3) and (4,5)(6,7)
             // of A, and the expert rows of W_r in the same order as B.
@@ -241,7 +310,7 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     const int32_t* __restrict__ ids, int n_slots, int T, int E, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
     ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks, int chunk_tokens, int routed_chunk_tokens,
-    int32_t* __restrict__ zero_words, int n_zero) {
+    int32_t* __restrict__ zero_words, int n_zero, int32_t* __restrict__ status) {
     __shared__ int s_count[BK_MAX_E];
     __shared__ int s_base[BK_MAX_E];
     __shared__ int s_warp[BK_WARPS][BK_MAX_E];   // per-warp counts, then exclusive prefix over warps
@@ -253,7 +322,15 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
         for (int i = tid; i < n_zero; i += BK_THREADS) zero_words[i] = 0;
     for (int e = tid; e < E; e += BK_THREADS) s_count[e] = 0;
     __syncthreads();
-    for (int s = tid; s < n_slots; s += BK_THREADS) atomicAdd(&s_count[ids[s]], 1);
+    // ids given by a caller may be out of range: such a slot is counted as
+    // expert 0 and the status word says so (the router's are always valid)
+    auto expert_of = [&](int s) {
+        const int e = ids[s];
+        if (unsigned(e) < unsigned(E)) return e;
+        if (status) atomicExch(status, DEV_BAD_EXPERT);
+        return 0;
+    };
+    for (int s = tid; s < n_slots; s += BK_THREADS) atomicAdd(&s_count[expert_of(s)], 1);
     __syncthreads();
     if (tid == 0) {
         int run = 0;
@@ -290,7 +367,7 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
         __syncthreads();
         const int s = s0 + tid;
         const bool valid = s < n_slots;
-        const int e = valid ? ids[s] : -1 - lane;    // distinct dummies never match real experts
+        const int e = valid ? expert_of(s) : -1 - lane;    // distinct dummies never match real experts
         const unsigned same = __match_any_sync(0xffffffffu, e);
         const int rank = __popc(same & ((1u << lane) - 1u));
         if (valid && rank == 0) s_warp[warp][e] = __popc(same);
@@ -322,16 +399,18 @@ size_t router_smem_bytes(int D, int E) { return size_t(router_warps(D, E)) * RT_
 // K ranges per token tile: with few tiles (a decode batch) the router would
 // run on a handful of SMs, so K is split over up to 32 CTAs per tile, each
 // with at least two groups of 128.
-int router_ksplit(int T, int D) {
+// With an RMSNorm the split CTAs of a tile form one thread-block cluster, so
+// at most 8 (the portable cluster size).
+int router_ksplit(int T, int D, bool rms) {
     const int tiles = int(ceil_div(T, RT_TOK)), groups = D / kGroup;
     if (tiles >= 37) return 1;
-    for (int ks = 32; ks > 1; --ks)
+    for (int ks = rms ? 8 : 32; ks > 1; --ks)
         if (groups % ks == 0 && groups / ks >= 2) return ks;
     return 1;
 }
 
-size_t router_partial_floats(int T, int D, int E) {
-    const int ks = router_ksplit(T, D);
+size_t router_partial_floats(int T, int D, int E, bool rms) {
+    const int ks = router_ksplit(T, D, rms);
     return ks > 1 ? size_t(ks) * ceil_div(T, RT_TOK) * RT_TOK * E : 0;
 }
 
@@ -339,7 +418,8 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between) {
     // K split only with scratch for the partial logits (the layer's workspace)
-    const int ks = (prep && prep->router_part) ? router_ksplit(T, D) : 1;
+    const bool rms = prep && prep->rms_weight;
+    const int ks = (prep && prep->router_part) ? router_ksplit(T, D, rms) : 1;
     const int nw = router_warps(D / ks, E);
     const size_t smem = router_smem_bytes(D / ks, E);
     if (allow_max_smem(router_kernel) != MOE_OK) return MOE_ERR_CUDA;
@@ -348,21 +428,49 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
     float* part_g = ks > 1 ? prep->router_part : nullptr;
     int32_t* tile_cnt = ks > 1 ? prep->router_tile_cnt : nullptr;
     const dim3 grid(unsigned(ceil_div(T, RT_TOK)), unsigned(ks));
-    if (prep && prep->router_after_kernel)   // may overlap the kernel before it (it reads only x and W_r)
-        st = launch_pdl(router_kernel, grid, dim3(nw * 32), smem, stream, x, T, D, wr, bias, E, k, ids, gates, x_frag,
-                        ks, part_g, tile_cnt);
-    else {
-        router_kernel<<<grid, nw * 32, smem, stream>>>(x, T, D, wr, bias, E, k, ids, gates, x_frag, ks, part_g,
-                                                       tile_cnt);
-        st = launch_status();
+    const bf16* gamma = rms ? prep->rms_weight : nullptr;
+    const float eps = rms ? prep->rms_eps : 0.0f;
+    bf16* xn = rms ? prep->xn : nullptr;
+    int32_t* xn_ready = rms ? prep->xn_ready : nullptr;
+    {
+        // with an RMSNorm, a tile's ks CTAs form one cluster; the router may
+        // overlap the kernel before it when asked (it reads only x, gamma and W_r)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(nw * 32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        if (rms) {
+            attr[na].id = cudaLaunchAttributeClusterDimension;
+            attr[na].val.clusterDim.x = 1;
+            attr[na].val.clusterDim.y = unsigned(ks);
+            attr[na].val.clusterDim.z = 1;
+            ++na;
+        }
+        if (prep && prep->router_after_kernel) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        st = cuda_status(cudaLaunchKernelEx(&cfg, router_kernel, x, T, D, wr, bias, E, k, ids, gates, x_frag, ks,
+                                            part_g, tile_cnt, gamma, eps, xn, xn_ready));
     }
     if (st != MOE_OK) return st;
     if (between) cudaEventRecord(between, stream);
-    return launch_pdl(bucket_kernel, dim3(1), dim3(BK_THREADS), 0, stream, (const int32_t*)ids, T * k, T, E, counts,
-                      offsets, perm, inv_perm, prep ? prep->chunks : (ChunkEntry*)nullptr,
-                      prep ? prep->n_chunks : (int32_t*)nullptr, prep ? prep->chunk_tokens : 16,
-                      prep ? prep->routed_chunk_tokens : 16, prep ? prep->zero_words : (int32_t*)nullptr,
-                      prep ? prep->n_zero : 0);
+    return launch_bucket(ids, T, k, E, counts, offsets, perm, inv_perm, prep, stream);
+}
+
+moe_status launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
+                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream) {
+    return launch_pdl(bucket_kernel, dim3(1), dim3(BK_THREADS), 0, stream, ids, T * k, T, E, counts, offsets, perm,
+                      inv_perm, prep ? prep->chunks : (ChunkEntry*)nullptr, prep ? prep->n_chunks : (int32_t*)nullptr,
+                      prep ? prep->chunk_tokens : 16, prep ? prep->routed_chunk_tokens : 16,
+                      prep ? prep->zero_words : (int32_t*)nullptr, prep ? prep->n_zero : 0,
+                      prep ? prep->status : (int32_t*)nullptr);
 }
 
 }  // namespace moe

@@ -26,7 +26,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 17
+    assert len(names) == 21
     for n in names:
         assert hasattr(lib, n), n
 
@@ -118,10 +118,10 @@ def test_workspace_size_and_layer_checks(lib):
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(D=200)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(k=5)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=16)), 16) == 0
-    # groups of 64 / 32 run on the tensor-core tiles only: AUTO sizes that
-    # path's workspace, and a forced weight-streaming path is refused
-    g64 = _desc(group_size=64)
-    pre = _desc(path=moe.PATH_PREFILL)
+    # groups of 64 / 32: with AUTO the workspace covers both paths when the
+    # weight-streaming kernels take the shape, the tensor-core path otherwise
+    g64 = _desc(group_size=64, D=384)
+    pre = _desc(group_size=64, D=384, path=moe.PATH_PREFILL)
     assert lib.moe_ffn_workspace_size(ctypes.byref(g64), 16) == lib.moe_ffn_workspace_size(ctypes.byref(pre), 16)
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(group_size=32)), 16) > 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(w_up=None)), 16) == 0
@@ -144,16 +144,22 @@ def test_forward_rejects_small_workspace_and_bad_pointers(lib):
     assert lib.moe_ffn_forward_timed(ctypes.byref(d), f, 16, f, f, need, None, ev, 2) == S.INVALID_ARG
 
 
-def test_small_groups_refuse_the_weight_streaming_path(lib):
+def test_small_groups_on_the_weight_streaming_path(lib):
+    """Groups of 64 / 32 run on the weight-streaming kernels when a stage's
+    scale box fits a row (K / G a multiple of 4 and at least a stage's
+    groups); other shapes are refused there and AUTO takes the tensor cores."""
     S = moe.Status
     f = 1 << 20
-    d = _desc(group_size=64, path=moe.PATH_DECODE)
-    need = lib.moe_ffn_workspace_size(ctypes.byref(d), 16)
-    assert need > 0
-    assert lib.moe_ffn_forward(ctypes.byref(d), f, 16, f, f, need, None) == S.UNSUPPORTED_SHAPE
     names = (ctypes.c_char_p * 16)()
-    n = lib.moe_ffn_launch_names(ctypes.byref(_desc(group_size=32)), 16, names, 16)
-    assert "tc_gate_up" in [names[i].decode() for i in range(n)]
+    ok = _desc(group_size=64, path=moe.PATH_AUTO)                       # D = 256, F = 512
+    n = lib.moe_ffn_launch_names(ctypes.byref(ok), 16, names, 16)
+    assert "decode_gate_up" in [names[i].decode() for i in range(n)]
+    bad = _desc(group_size=64, D=384, path=moe.PATH_DECODE)            # 384 / 64 = 6 scales a row
+    need = lib.moe_ffn_workspace_size(ctypes.byref(bad), 16)
+    assert need > 0
+    assert lib.moe_ffn_forward(ctypes.byref(bad), f, 16, f, f, need, None) == S.UNSUPPORTED_SHAPE
+    n = lib.moe_ffn_launch_names(ctypes.byref(_desc(group_size=32, F=256)), 16, names, 16)
+    assert "tc_gate_up" in [names[i].decode() for i in range(n)]      # F = 256: 8 < 16 groups a stage
 
 
 def test_rmsnorm_checks_and_layer_prologue(lib):
@@ -164,15 +170,19 @@ def test_rmsnorm_checks_and_layer_prologue(lib):
     assert lib.moe_rmsnorm(f, 4, 256, None, 1e-5, f, None) == S.INVALID_ARG
     assert lib.moe_rmsnorm(f, 4, 256, f, -1.0, f, None) == S.INVALID_ARG
     assert lib.moe_rmsnorm(f, 4, 256, f, float("nan"), f, None) == S.INVALID_ARG
-    # a layer with an RMSNorm: the norm is its first launch and needs T x D x 2 more bytes
+    # a layer with an RMSNorm: the router normalizes x itself (no launch of its
+    # own), and the workspace holds the normalized rows: T x D x 2 more bytes
     plain, normed = _desc(), _desc(rms_weight=f, rms_eps=1e-5)
-    n0 = lib.moe_ffn_workspace_size(ctypes.byref(plain), 16)
-    n1 = lib.moe_ffn_workspace_size(ctypes.byref(normed), 16)
-    assert n1 >= n0 + 16 * 256 * 2
-    names = (ctypes.c_char_p * 16)()
-    n = lib.moe_ffn_launch_names(ctypes.byref(normed), 16, names, 16)
-    assert n == lib.moe_ffn_launch_names(ctypes.byref(plain), 16, None, 0) + 1
-    assert names[0] == b"rmsnorm" and names[1] == b"router"
+    for T in (16, 4096):
+        n0 = lib.moe_ffn_workspace_size(ctypes.byref(plain), T)
+        n1 = lib.moe_ffn_workspace_size(ctypes.byref(normed), T)
+        assert n1 >= n0 + T * 256 * 2
+        names0 = (ctypes.c_char_p * 16)()
+        names1 = (ctypes.c_char_p * 16)()
+        n = lib.moe_ffn_launch_names(ctypes.byref(normed), T, names1, 16)
+        assert n == lib.moe_ffn_launch_names(ctypes.byref(plain), T, names0, 16)
+        assert [names1[i] for i in range(n)] == [names0[i] for i in range(n)]
+        assert names1[0] == b"router" and b"rmsnorm" not in [names1[i] for i in range(n)]
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f, rms_eps=-1.0)), 16) == 0
     assert lib.moe_ffn_workspace_size(ctypes.byref(_desc(rms_weight=f + 4, rms_eps=1e-5)), 16) == 0
 
@@ -249,3 +259,23 @@ def test_noalloc_scratch_covers_scout_decode_batches(lib):
     auto = _scout_decode_desc()
     assert lib.moe_ffn_forward_noalloc(ctypes.byref(auto), f, 65, f, None) == S.WORKSPACE_TOO_SMALL
     assert lib.moe_ffn_forward_noalloc(ctypes.byref(auto), f, 4096, f, None) == S.WORKSPACE_TOO_SMALL
+
+
+def test_expert_parallel_steps_check_arguments(lib):
+    """The compute steps of an expert-parallel layer reject bad arguments
+    before touching the device; their workspaces follow the rows' count."""
+    S = moe.Status
+    f = 1 << 20
+    d = _desc(k=2)
+    n16 = lib.moe_expert_ffn_workspace_size(ctypes.byref(d), 16)
+    n512 = lib.moe_expert_ffn_workspace_size(ctypes.byref(d), 512)
+    assert 0 < n16 < n512 and n16 % 256 == 0
+    assert lib.moe_expert_ffn_workspace_size(ctypes.byref(_desc(D=200)), 16) == 0
+    assert lib.moe_expert_ffn_forward(ctypes.byref(d), f, 16, f, f, f, f, 1024, None) == S.WORKSPACE_TOO_SMALL
+    assert lib.moe_expert_ffn_forward(ctypes.byref(d), f, 16, None, f, f, f, n16, None) == S.INVALID_ARG
+    assert lib.moe_expert_ffn_forward(ctypes.byref(d), f, 16, f, f, f + 8, f, n16, None) == S.INVALID_ARG
+    assert lib.moe_expert_ffn_forward(ctypes.byref(d), f, 0, f, f, f, f, n16, None) == S.UNSUPPORTED_SHAPE
+    s16 = lib.moe_shared_ffn_workspace_size(ctypes.byref(d), 16)
+    assert s16 > 0 and s16 < lib.moe_shared_ffn_workspace_size(ctypes.byref(d), 4096)
+    assert lib.moe_shared_ffn_combine(ctypes.byref(d), f, 16, None, f, f, s16, None) == S.INVALID_ARG
+    assert lib.moe_shared_ffn_combine(ctypes.byref(d), f, 16, f, f, f, 1024, None) == S.WORKSPACE_TOO_SMALL

@@ -123,18 +123,47 @@ def test_skewed_full_size_sampled():
     assert rel_err(got, ref) <= TOL
 
 
+def _decode_takes_groups(D, F, G):
+    """The weight-streaming kernels take groups of 64 / 32 when a stage's
+    scale box fits a row: K / G a multiple of 4 and at least the groups of a
+    stage (256 K for gate/up, 512 K for down)."""
+    return all((K // G) % 4 == 0 and K // G >= kst // G for K, kst in ((D, 256), (F, 512)))
+
+
 @pytest.mark.parametrize("G", [64, 32])
 @pytest.mark.parametrize("T,D,F,Fs,E,k", [(64, 256, 512, 512, 4, 1), (37, 384, 640, 384, 5, 2),
-                                          (300, 256, 256, 128, 3, 2), (1, 256, 512, 512, 4, 1)])
+                                          (300, 256, 256, 128, 3, 2), (1, 256, 512, 512, 4, 1),
+                                          (16, 1024, 1536, 512, 6, 1)])
 def test_small_int4_groups(T, D, F, Fs, E, k, G):
-    """int4 experts quantized in groups of 64 or 32 (AUTO runs them on the
-    tensor-core tiles; the weight-streaming kernels refuse them)."""
+    """int4 experts quantized in groups of 64 or 32 ("a smaller group_size"):
+    AUTO, the tensor-core tiles and -- where the shape allows -- the
+    weight-streaming kernels, whose MMAs then go one 32-K quarter at a time."""
     b = build(synth.LayerShape("g%d" % G, T, D, F, E, k, Fs), group_size=G)
-    got, ref = _run(b, moe.PATH_AUTO)
-    assert rel_err(got, ref) <= TOL
+    for path in (moe.PATH_AUTO, moe.PATH_PREFILL):
+        got, ref = _run(b, path)
+        assert rel_err(got, ref) <= TOL
     b.gpu.set_path(moe.PATH_DECODE)
-    with pytest.raises(moe.MoEError):
-        b.gpu(b.x.cuda())
+    if _decode_takes_groups(D, F, G):
+        got, ref = _run(b, moe.PATH_DECODE)
+        assert rel_err(got, ref) <= TOL
+    else:
+        with pytest.raises(moe.MoEError):
+            b.gpu(b.x.cuda())
+
+
+@pytest.mark.parametrize("G", [64, 32])
+def test_small_int4_groups_wide_range(G):
+    """Groups of 64 / 32 on the weight-streaming path with token rows spanning
+    30 binades (each group of x and h gets its own power of two)."""
+    b = build(synth.LayerShape("wide%d" % G, 24, 512, 1024, 4, 1, 512), margin=False, group_size=G)
+    b.x = _wide_range_tokens(b.shape, b.w_router, b.bias, seed=6)
+    b.gpu.set_path(moe.PATH_DECODE)
+    out = b.gpu(b.x.cuda())
+    assert b.gpu.device_status() == moe.Status.OK
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = offn.moe_forward(b.oracle, b.x)["out"]
+    row_err = np.abs(got - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert row_err.max() <= TOL, row_err.max()
 
 
 FP8_SHAPES = [

@@ -30,9 +30,14 @@ def test_rmsnorm_matches_oracle(T, D, eps):
 
 
 @pytest.mark.parametrize("path", [moe.PATH_DECODE, moe.PATH_PREFILL])
-@pytest.mark.parametrize("shape", [synth.SHAPES["tiny"], synth.LayerShape("r", 37, 384, 640, 5, 2, 384)],
-                         ids=["tiny", "ragged"])
+@pytest.mark.parametrize("shape", [synth.SHAPES["tiny"], synth.LayerShape("r", 37, 384, 640, 5, 2, 384),
+                                   synth.LayerShape("ks4", 16, 1024, 512, 4, 1, 512),
+                                   synth.LayerShape("ks8", 20, 5120, 1024, 8, 2, 512)],
+                         ids=["tiny", "ragged", "split4", "split8"])
 def test_layer_with_rmsnorm(shape, path):
+    """The router normalizes x itself (no launch of its own): with D = 1024
+    and 5120 at decode sizes its K range is split over a cluster of 4 / 8
+    CTAs that exchange the rows' partial sums of squares."""
     b = build(shape, rms=True)
     b.gpu.set_path(path)
     out = b.gpu(b.x.cuda())
@@ -46,3 +51,10 @@ def test_fp8_layer_with_rmsnorm():
     out = b.gpu(b.x.cuda())
     ref = offn.moe_forward(b.oracle, b.x)["out"]
     assert rel_err(out.float().cpu().numpy().astype(np.float64), ref) <= 1e-2
+
+
+def test_layer_norm_is_not_a_launch():
+    b = build(synth.SHAPES["tiny"], rms=True)
+    for path in (moe.PATH_DECODE, moe.PATH_PREFILL):
+        b.gpu.set_path(path)
+        assert "rmsnorm" not in b.gpu.launch_names(64)
