@@ -95,10 +95,10 @@ QUANT_E, QUANT_D, QUANT_F = 16, 5120, 8192
 QUANT_METRIC = "int4_row_quantize GB/s moved (fp32 weights read, int4 codes and fp32 scales written); % of HBM roofline"
 
 
-def quant_matrices():
+def quant_matrices(E: int = QUANT_E):
     """(name, rows, cols) of the quantize workload: each projection of all
-    16 experts as one [E * N, K] matrix."""
-    E, D, F = QUANT_E, QUANT_D, QUANT_F
+    E (16) experts as one [E * N, K] matrix."""
+    D, F = QUANT_D, QUANT_F
     return [("gate", E * F, D), ("up", E * F, D), ("down", E * D, F)]
 
 
@@ -579,7 +579,7 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
     gen = torch.Generator(device=dev)
     gen.manual_seed(args.seed * 1000 + rank)
     mats = []
-    for name, rows, cols in quant_matrices():
+    for name, rows, cols in quant_matrices(args.experts):
         w = torch.randn(rows, cols, generator=gen, device=dev, dtype=torch.float32).mul_(synth.WEIGHT_STD)
         codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
         scales = torch.empty(rows, cols // args.group_size, dtype=torch.float32, device=dev)
@@ -651,10 +651,11 @@ def run_quantize(args, rank: int, world: int, dev: torch.device):
         "dtype": "f32 -> int4 (fp32 scales)",
         "data": "synthetic (N(0, 0.02) fp32 weights from torch's seeded device generator)",
         "config": {
-            "workload": "quantize: int4_row_quantize (group %d) of 16 experts x {gate [8192, 5120], " % args.group_size +
-                        "up [8192, 5120], down [5120, 8192]} fp32 = 2.01 G weights, 3 calls per step",
+            "workload": "quantize: int4_row_quantize (group %d) of %d experts x {gate [8192, 5120], " % (
+                args.group_size, args.experts) + "up [8192, 5120], down [5120, 8192]} fp32 = %.2f G weights, "
+                "3 calls per step" % (args.experts * 3 * 8192 * 5120 / 1e9),
             "parallelism": "replicas" if world > 1 else "single GPU",
-            "l2": "inputs (8.05 GB) larger than L2; no flush",
+            "l2": "inputs (%.2f GB) larger than L2; no flush" % (args.experts * 3 * 8192 * 5120 * 4 / 1e9),
         },
         "roofline": {"bound": "hbm", "kernel": "quantize_int4", "achieved": achieved, "peak": hbm_peak,
                      "peak_source": peak_src + " copy bandwidth", "unit": "GB/s", "frac": achieved / hbm_peak,
@@ -814,6 +815,8 @@ def main(argv=None):
                              "quantize", "dense_decode", "dense_prefill"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=QUANT_E,
+                    help="quantize workload: experts in the weight set (16; fewer for profiling captures)")
     ap.add_argument("--rmsnorm", action="store_true",
                     help="run the layer with its RMSNorm prologue (gamma ~ 1 + N(0, 0.1), eps 1e-5)")
     ap.add_argument("--group-size", type=int, default=128, choices=[128, 64, 32],
