@@ -278,6 +278,8 @@ def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> di
             "rmsnorm": ("bytes", T * D * 2 * 2 + D * 2),
             "router": ("flops", 2 * T * D * E),
             "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
+            "bucket_scan": ("bytes", (E + 1) * 8),
+            "bucket_place": ("bytes", S * 4 * 3),
             "quantize_x": ("bytes", T * D * 2 + S * D),
             "tc_gate_up": ("flops", 2 * S * D * 2 * F),
             "quantize_h": ("bytes", S * F * 2 * 2 + S * F),
@@ -290,6 +292,8 @@ def kernel_work(shape: synth.LayerShape, n_touched: int, group: int = 128) -> di
         "rmsnorm": ("bytes", T * D * 2 * 2 + D * 2),
         "router": ("flops", 2 * T * D * E),
         "bucket": ("bytes", S * 4 * 3 + (E + 1) * 8),
+        "bucket_scan": ("bytes", (E + 1) * 8),
+        "bucket_place": ("bytes", S * 4 * 3),
         "act16_x": ("bytes", T * D * 2 * 2),
         # weights once; x read; h written as bf16 (routed and shared) and as the
         # down pass's fp16 operands (routed)

@@ -52,7 +52,6 @@ struct DecodeParams {
 
 // Extra outputs of the routing step used by the weight-streaming FFN.
 struct RoutePrep {
-    bf16* x_frag;         // x in bf16 fragment order [T, D] (shared expert)
     ChunkEntry* chunks;   // task list
     int32_t* n_chunks;    // [0] all chunks, [1] the shared expert's
     int32_t chunk_tokens;         // tokens per shared-expert chunk (16 weight streaming, 256 tensor cores)
@@ -67,6 +66,7 @@ struct RoutePrep {
     bf16* xn;                   // ... and where the router writes it, bf16 [T, D]
     int32_t* xn_ready;          // ... counted by each router CTA once its part of xn is written (or null)
     int32_t* status;            // device status word: out-of-range given expert ids are reported there
+    int32_t* bucket_hist;       // bucket_blocks(T * k) * E ints for bucketing many slots over several CTAs (or null)
 };
 
 // TMA maps of one weight-streaming launch:
@@ -105,11 +105,15 @@ moe_status launch_decode_ffn(int mode, int G, const DecodeMaps& maps, const Deco
                              cudaStream_t stream);
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
-                        int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between);
+                        int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between,
+                        cudaEvent_t ev_scan = nullptr, cudaEvent_t ev_place = nullptr);
 // The bucketing step alone, from given expert ids [T, k] (counts, offsets,
 // the stable permutation and, with `prep`, the FFN's chunk list).
 moe_status launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream);
+                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t ev_scan = nullptr,
+                         cudaEvent_t ev_place = nullptr);
+// CTAs the bucketing of n slots takes (0: one CTA, bucket_kernel)
+int bucket_blocks(int64_t n_slots);
 moe_status launch_act16(const bf16* in, int64_t rows, int cols, int G, const int32_t* src_perm, int k,
                         __half* out16, float* meta, cudaStream_t stream);
 

@@ -42,6 +42,7 @@ moe_status check_route_shape(int32_t T, int32_t D, int32_t E, int32_t k) {
 // workspace must be large enough for either.
 struct WsLayout {
     size_t status, rt_cnt, dec_cnt, zeros_end, counters, rt_part, ids, gates, counts, offsets, perm, inv_perm, chunks, nchunks;
+    size_t bk_hist;   // per-block expert counts of the multi-CTA bucketing
     size_t xn;   // RMSNorm of x (layers with rms_weight)
     size_t common_end;
     // weight-streaming path
@@ -86,6 +87,7 @@ WsLayout ws_layout(const moe_layer_desc& L, int64_t T, int path) {
     w.offsets = take(size_t(L.E + 1) * 4);
     w.perm = take(S * 4);
     w.inv_perm = take(S * 4);
+    w.bk_hist = take(size_t(bucket_blocks(S)) * L.E * 4);
     w.chunks = take(size_t(decode_max_chunks(int(T), L.k, L.E)) * sizeof(ChunkEntry));
     w.nchunks = take(16);
     w.xn = take(L.rms_weight ? size_t(T) * L.D * 2 : 0);
@@ -181,6 +183,8 @@ struct Marks {
         if (ev && i < n) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
         ++i;
     }
+    // the event j places after the current one (or null)
+    cudaEvent_t event(int j) const { return (ev && i + j < n) ? static_cast<cudaEvent_t>(ev[i + j]) : nullptr; }
 };
 
 const char* const kDecodeLaunches[] = {"router", "bucket", "act16_x", "decode_gate_up", "decode_down"};
@@ -262,13 +266,13 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, const bf16* x
         prep.router_part = at<float>(ws, W.rt_part);
         prep.router_tile_cnt = at<int32_t>(ws, W.rt_cnt);
     }
-    prep.x_frag = nullptr;
     prep.chunks = chunks;
     prep.n_chunks = nch;
     prep.zero_words = nullptr;      // the task counters are cleared with the status word
     prep.n_zero = 0;
     prep.chunk_tokens = 16;
     prep.routed_chunk_tokens = 8;   // one 8-column n-tile per routed chunk
+    prep.bucket_hist = at<int32_t>(ws, W.bk_hist);
     prep.router_after_kernel = false;
     set_rms(prep, L, ws, W);
     moe_status s;
@@ -279,10 +283,11 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, const bf16* x
         gates = const_cast<float*>(pr->gates);
     } else {
         mk.mark(st);
+        const bool multi = bucket_blocks(int64_t(T) * L.k) > 0;
         s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                          at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm,
-                         inv, &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
-        ++mk.i;
+                         inv, &prep, st, mk.event(0), multi ? mk.event(1) : nullptr, multi ? mk.event(2) : nullptr);
+        mk.i += multi ? 3 : 1;
     }
     if (s != MOE_OK) return s;
     mk.mark(st);
@@ -402,12 +407,16 @@ moe_status ffn_decode_path(const moe_layer_desc& L, const bf16* x, const bf16* x
 
 // Kernel launches of the tensor-core path, in order (the combine only when a
 // token has more than one routed slot).
-int prefill_launches(const moe_layer_desc& L, const char** names, int max_names) {
+int prefill_launches(const moe_layer_desc& L, int64_t T, const char** names, int max_names) {
     const bool fp8 = L.format == MOE_WEIGHTS_FP8_ROW;
-    const char* list[9];
+    const char* list[11];
     int n = 0;
     list[n++] = "router";
     list[n++] = "bucket";
+    if (bucket_blocks(T * L.k) > 0) {   // the bucketing's three kernels
+        list[n++] = "bucket_scan";
+        list[n++] = "bucket_place";
+    }
     list[n++] = fp8 ? "quantize_x" : "gather";
     list[n++] = "tc_shared_gate_up";
     list[n++] = "tc_shared_down";
@@ -421,7 +430,7 @@ int prefill_launches(const moe_layer_desc& L, const char** names, int max_names)
 
 // The kernels one forward launches, in order (an RMSNorm runs inside the router).
 int32_t layer_launch_names(const moe_layer_desc& L, int64_t T, const char** names, int32_t max_names) {
-    if (choose_path(L, T) != PATH_SEL_DECODE) return prefill_launches(L, names, max_names);
+    if (choose_path(L, T) != PATH_SEL_DECODE) return prefill_launches(L, T, names, max_names);
     for (int32_t i = 0; i < kDecodeLaunchCount && i < max_names && names; ++i) names[i] = kDecodeLaunches[i];
     return kDecodeLaunchCount;
 }
@@ -448,6 +457,7 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, const bf16* 
     prep.n_chunks = nch;
     prep.chunk_tokens = TC_BLOCK_TOKENS;
     prep.routed_chunk_tokens = TC_BLOCK_TOKENS;
+    prep.bucket_hist = at<int32_t>(ws, W.bk_hist);
     set_rms(prep, L, ws, W);
     moe_status s;
     if (pr) {   // the rows' experts are given: bucketing only
@@ -457,10 +467,11 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, const bf16* 
         gates = const_cast<float*>(pr->gates);
     } else {
         mk.mark(st);
+        const bool multi = bucket_blocks(int64_t(T) * L.k) > 0;
         s = launch_route(x, T, L.D, static_cast<const bf16*>(L.w_router), L.router_bias, L.E, L.k,
                          at<int32_t>(ws, W.ids), gates, at<int32_t>(ws, W.counts), at<int32_t>(ws, W.offsets), perm,
-                         inv, &prep, st, (mk.ev && mk.i < mk.n) ? static_cast<cudaEvent_t>(mk.ev[mk.i]) : nullptr);
-        ++mk.i;
+                         inv, &prep, st, mk.event(0), multi ? mk.event(1) : nullptr, multi ? mk.event(2) : nullptr);
+        mk.i += multi ? 3 : 1;
     }
     if (s != MOE_OK) return s;
     mk.mark(st);

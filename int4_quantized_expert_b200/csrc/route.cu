@@ -13,9 +13,8 @@
 //                  fragments loaded straight from global memory.  Partials are
 //                  summed in a fixed order (deterministic), the bias added, and
 //                  each token's top-k taken by k passes of a warp argmax (ties
-//                  -> lower expert index), then the gate.  For the weight-
-//                  streaming FFN it also writes x in the fragment order its
-//                  shared-expert MMAs read.
+//                  -> lower expert index), then the gate.  With an RMSNorm it
+//                  normalizes the rows first and writes them out.
 //   bucket_kernel  one CTA: per-expert counts, exclusive offsets and the stable
 //                  permutation of slots from warp match ranks and a scan over
 //                  warps; optionally the weight-streaming FFN's task list.
@@ -26,7 +25,6 @@ namespace moe {
 
 constexpr int RT_TOK = 16;      // tokens per CTA (one m16 tile)
 constexpr int RT_MAXW = 12;     // warps splitting K
-constexpr int RT_EPASS = 64;    // experts per accumulator pass (8 n-tiles)
 constexpr size_t RT_SMEM_MAX = 160 * 1024;
 
 // Warps used: the largest divisor of D / 128 that is <= 12 and whose partial
@@ -44,10 +42,14 @@ inline int router_warps(int D, int E) {
 // tile to arrive (counted in tile_cnt, zeroed beforehand) sums them in
 // K-range order -- the same order whichever CTA is last -- and takes the
 // top-k.  No CTA waits for another.
-__global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
+// NT: n-tiles of 8 experts per accumulator pass (1, 2 or 4), the smallest
+// power of two covering E up to 32 -- few experts keep few registers, so more
+// CTAs fit on an SM.
+template <int NT>
+__global__ void __launch_bounds__(RT_MAXW * 32, NT <= 2 ? 2 : 1) router_kernel(
     const bf16* __restrict__ x, int T, int D, const bf16* __restrict__ wr,
     const float* __restrict__ bias, int E, int k, int32_t* __restrict__ ids,
-    float* __restrict__ gates, bf16* __restrict__ x_frag, int ksplit, float* __restrict__ part_g,
+    float* __restrict__ gates, int ksplit, float* __restrict__ part_g,
     int32_t* __restrict__ tile_cnt, const bf16* __restrict__ gamma, float rms_eps, bf16* __restrict__ xn,
     int32_t* __restrict__ xn_ready) {
     extern __shared__ __align__(16) float part[];     // [nw][RT_TOK][E]
@@ -128,21 +130,21 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
         if (xn_ready != nullptr && threadIdx.x == 0) atomicAdd(xn_ready, 1);
     }
 
-    for (int e0 = 0; e0 < E; e0 += RT_EPASS) {
-        float acc[8][4];
+    for (int e0 = 0; e0 < E; e0 += 8 * NT) {
+        float acc[NT][4];
 #pragma unroll
-        for (int n = 0; n < 8; ++n)
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
 
         // operands of the next 32-K chunk are loaded while the current one runs
-        const int n_tiles = min(8, (E - e0 + 7) / 8);
-        uint4 xa, xb, wv[8], nxa, nxb, nwv[8];
-        auto load = [&](int kk, uint4& a, uint4& b, uint4 (&w)[8]) {
+        const int n_tiles = min(NT, (E - e0 + 7) / 8);
+        uint4 xa, xb, wv[NT], nxa, nxb, nwv[NT];
+        auto load = [&](int kk, uint4& a, uint4& b, uint4 (&w)[NT]) {
             a = row_a ? ldg_cached(xa_row + kk + 8 * c) : make_uint4(0, 0, 0, 0);
             b = row_b ? ldg_cached(xb_row + kk + 8 * c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
+            for (int n = 0; n < NT; ++n) {
                 const int e = e0 + n * 8 + g;
                 w[n] = (n < n_tiles && e < E) ? ldg_cached(wr + int64_t(e) * D + kk + 8 * c) : make_uint4(0, 0, 0, 0);
             }
@@ -158,24 +160,8 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
             // thread (g, c) holds K values kk + 8c .. kk + 8c + 7 of rows g and g + 8;
             // the two MMAs below use them as K pairs (0,1)(2,3) and (4,5)(6,7)
             // of A, and the expert rows of W_r in the same order as B.
-            if (x_frag != nullptr && e0 == 0) {
-                // x in the bf16 fragment order the shared expert's weight-
-                // streaming MMAs read (every 8 values stored x0 x4 x1 x5 x2 x6 x3 x7)
-                if (row_a) {
-                    uint4 p;
-                    p.x = prmt(xa.x, xa.z, 0x5410); p.y = prmt(xa.x, xa.z, 0x7632);
-                    p.z = prmt(xa.y, xa.w, 0x5410); p.w = prmt(xa.y, xa.w, 0x7632);
-                    *reinterpret_cast<uint4*>(x_frag + int64_t(t0 + g) * D + kk + 8 * c) = p;
-                }
-                if (row_b) {
-                    uint4 p;
-                    p.x = prmt(xb.x, xb.z, 0x5410); p.y = prmt(xb.x, xb.z, 0x7632);
-                    p.z = prmt(xb.y, xb.w, 0x5410); p.w = prmt(xb.y, xb.w, 0x7632);
-                    *reinterpret_cast<uint4*>(x_frag + int64_t(t0 + g + 8) * D + kk + 8 * c) = p;
-                }
-            }
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
+            for (int n = 0; n < NT; ++n) {
                 if (n >= n_tiles) break;
                 mma_bf16_16816(acc[n], xa.x, xb.x, xa.y, xb.y, wv[n].x, wv[n].y);
                 mma_bf16_16816(acc[n], xa.z, xb.z, xa.w, xb.w, wv[n].z, wv[n].w);
@@ -183,12 +169,12 @@ __global__ void __launch_bounds__(RT_MAXW * 32) router_kernel(
             xa = nxa;
             xb = nxb;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) wv[n] = nwv[n];
+            for (int n = 0; n < NT; ++n) wv[n] = nwv[n];
         }
         // C fragment: rows (tokens) g, g + 8; columns (experts) 2c, 2c + 1 of each n-tile
         float* pw = part + warp * RT_TOK * E;
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
+        for (int n = 0; n < NT; ++n) {
             const int e = e0 + n * 8 + 2 * c;
             if (e < E) { pw[g * E + e] = acc[n][0]; pw[(g + 8) * E + e] = acc[n][2]; }
             if (e + 1 < E) { pw[g * E + e + 1] = acc[n][1]; pw[(g + 8) * E + e + 1] = acc[n][3]; }
@@ -394,6 +380,135 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// Bucketing of many slots over several CTAs (the same results as
+// bucket_kernel): each CTA takes a block of BK_BLOCK consecutive slots.
+//   bucket_hist_kernel   per-block expert counts -> hist[block][E]
+//   bucket_scan_kernel   one CTA: counts, offsets, the chunk list, and each
+//                        (block, expert)'s first position -> hist
+//   bucket_place_kernel  per block: stable positions of its slots (warp match
+//                        ranks and a prefix over warps, block by block in slot
+//                        order) -> perm, inv_perm
+// Three launches chained by programmatic dependent launch; no CTA waits for
+// another.
+// ---------------------------------------------------------------------------
+constexpr int BK_BLOCK = 2 * BK_THREADS;
+
+__device__ __forceinline__ int bucket_expert(const int32_t* ids, int s, int E, int32_t* status) {
+    const int e = ids[s];
+    if (unsigned(e) < unsigned(E)) return e;
+    if (status) atomicExch(status, DEV_BAD_EXPERT);   // given ids out of range count as expert 0
+    return 0;
+}
+
+__global__ void __launch_bounds__(BK_THREADS) bucket_hist_kernel(const int32_t* __restrict__ ids, int n_slots,
+                                                                 int E, int32_t* __restrict__ hist,
+                                                                 int32_t* __restrict__ status) {
+    __shared__ int s_count[BK_MAX_E];
+    griddep_launch_dependents();
+    griddep_wait();   // the router's ids
+    for (int e = threadIdx.x; e < E; e += BK_THREADS) s_count[e] = 0;
+    __syncthreads();
+    const int s_end = min(n_slots, (blockIdx.x + 1) * BK_BLOCK);
+    for (int s = blockIdx.x * BK_BLOCK + threadIdx.x; s < s_end; s += BK_THREADS)
+        atomicAdd(&s_count[bucket_expert(ids, s, E, status)], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += BK_THREADS) hist[blockIdx.x * E + e] = s_count[e];
+}
+
+__global__ void __launch_bounds__(BK_THREADS) bucket_scan_kernel(
+    int32_t* __restrict__ hist, int n_blocks, int n_slots, int T, int E, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks,
+    int chunk_tokens, int routed_chunk_tokens) {
+    __shared__ int s_count[BK_MAX_E];
+    __shared__ int s_base[BK_MAX_E];
+    griddep_launch_dependents();
+    griddep_wait();
+    for (int e = threadIdx.x; e < E; e += BK_THREADS) {
+        int c = 0;
+        for (int b = 0; b < n_blocks; ++b) c += hist[b * E + e];
+        s_count[e] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_count[e]; }
+        offsets[E] = n_slots;
+        if (chunks != nullptr) {   // the FFN kernels' task list, as bucket_kernel writes it
+            int n = 0;
+            for (int t0 = 0; t0 < T; t0 += chunk_tokens) {
+                ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(chunk_tokens, T - t0); ce.pad = 0;
+                chunks[n++] = ce;
+            }
+            n_chunks[1] = n;
+            for (int e = 0; e < E; ++e)
+                for (int s = 0; s < s_count[e]; s += routed_chunk_tokens) {
+                    ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s;
+                    ce.count = min(routed_chunk_tokens, s_count[e] - s);
+                    ce.pad = 0;
+                    chunks[n++] = ce;
+                }
+            n_chunks[0] = n;
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += BK_THREADS) {
+        counts[e] = s_count[e];
+        offsets[e] = s_base[e];
+        int base = s_base[e];
+        for (int b = 0; b < n_blocks; ++b) {   // each block's first position of expert e
+            const int c = hist[b * E + e];
+            hist[b * E + e] = base;
+            base += c;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(BK_THREADS) bucket_place_kernel(const int32_t* __restrict__ ids, int n_slots,
+                                                                  int E, const int32_t* __restrict__ hist,
+                                                                  int32_t* __restrict__ perm,
+                                                                  int32_t* __restrict__ inv_perm) {
+    __shared__ int s_count[BK_MAX_E];
+    __shared__ int s_base[BK_MAX_E];
+    __shared__ int s_warp[BK_WARPS][BK_MAX_E];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_launch_dependents();
+    griddep_wait();   // the bases
+    for (int e = tid; e < E; e += BK_THREADS) s_base[e] = hist[blockIdx.x * E + e];
+    const int s_begin = blockIdx.x * BK_BLOCK, s_end = min(n_slots, s_begin + BK_BLOCK);
+    for (int s0 = s_begin; s0 < s_end; s0 += BK_THREADS) {
+        for (int i = tid; i < BK_WARPS * E; i += BK_THREADS) s_warp[i / E][i % E] = 0;
+        __syncthreads();
+        const int s = s0 + tid;
+        const bool valid = s < s_end;
+        const int e = valid ? bucket_expert(ids, s, E, nullptr) : -1 - lane;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        if (valid && rank == 0) s_warp[warp][e] = __popc(same);
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += BK_THREADS) {
+            int run = 0;
+            for (int w = 0; w < BK_WARPS; ++w) {
+                const int cnt = s_warp[w][ee];
+                s_warp[w][ee] = run;
+                run += cnt;
+            }
+            s_count[ee] = run;
+        }
+        __syncthreads();
+        if (valid) {
+            const int pos = s_base[e] + s_warp[warp][e] + rank;
+            perm[pos] = s;
+            if (inv_perm != nullptr) inv_perm[s] = pos;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += BK_THREADS) s_base[ee] += s_count[ee];
+        __syncthreads();
+    }
+}
+
+int bucket_blocks(int64_t n_slots) { return n_slots >= 2 * BK_BLOCK ? int(ceil_div(n_slots, BK_BLOCK)) : 0; }
+
 size_t router_smem_bytes(int D, int E) { return size_t(router_warps(D, E)) * RT_TOK * E * sizeof(float); }
 
 // K ranges per token tile: with few tiles (a decode batch) the router would
@@ -416,15 +531,18 @@ size_t router_partial_floats(int T, int D, int E, bool rms) {
 
 moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float* bias, int E, int k,
                         int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
-                        int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between) {
+                        int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t between,
+                        cudaEvent_t ev_scan, cudaEvent_t ev_place) {
     // K split only with scratch for the partial logits (the layer's workspace)
     const bool rms = prep && prep->rms_weight;
     const int ks = (prep && prep->router_part) ? router_ksplit(T, D, rms) : 1;
     const int nw = router_warps(D / ks, E);
     const size_t smem = router_smem_bytes(D / ks, E);
-    if (allow_max_smem(router_kernel) != MOE_OK) return MOE_ERR_CUDA;
+    // n-tiles per pass: the smallest power of two covering E, at most 4 (more
+    // experts take several passes over the CTA's K range; 8 n-tiles spilled)
+    auto kern = E <= 8 ? router_kernel<1> : E <= 16 ? router_kernel<2> : router_kernel<4>;
+    if (allow_max_smem(kern) != MOE_OK) return MOE_ERR_CUDA;
     moe_status st;
-    bf16* x_frag = prep ? prep->x_frag : nullptr;
     float* part_g = ks > 1 ? prep->router_part : nullptr;
     int32_t* tile_cnt = ks > 1 ? prep->router_tile_cnt : nullptr;
     const dim3 grid(unsigned(ceil_div(T, RT_TOK)), unsigned(ks));
@@ -456,16 +574,33 @@ moe_status launch_route(const bf16* x, int T, int D, const bf16* wr, const float
         }
         cfg.attrs = attr;
         cfg.numAttrs = na;
-        st = cuda_status(cudaLaunchKernelEx(&cfg, router_kernel, x, T, D, wr, bias, E, k, ids, gates, x_frag, ks,
-                                            part_g, tile_cnt, gamma, eps, xn, xn_ready));
+        st = cuda_status(cudaLaunchKernelEx(&cfg, kern, x, T, D, wr, bias, E, k, ids, gates, ks, part_g, tile_cnt,
+                                            gamma, eps, xn, xn_ready));
     }
     if (st != MOE_OK) return st;
     if (between) cudaEventRecord(between, stream);
-    return launch_bucket(ids, T, k, E, counts, offsets, perm, inv_perm, prep, stream);
+    return launch_bucket(ids, T, k, E, counts, offsets, perm, inv_perm, prep, stream, ev_scan, ev_place);
 }
 
 moe_status launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
-                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream) {
+                         int32_t* inv_perm, const RoutePrep* prep, cudaStream_t stream, cudaEvent_t ev_scan,
+                         cudaEvent_t ev_place) {
+    const int nb = bucket_blocks(int64_t(T) * k);
+    if (prep && prep->bucket_hist && nb > 0 && prep->zero_words == nullptr) {
+        // many slots: three kernels over ceil(slots / BK_BLOCK) CTAs
+        const int n_slots = T * k;
+        int32_t* st = prep->status;
+        moe_status s = launch_pdl(bucket_hist_kernel, dim3(nb), dim3(BK_THREADS), 0, stream, ids, n_slots, E,
+                                  prep->bucket_hist, st);
+        if (s != MOE_OK) return s;
+        if (ev_scan) cudaEventRecord(ev_scan, stream);
+        s = launch_pdl(bucket_scan_kernel, dim3(1), dim3(BK_THREADS), 0, stream, prep->bucket_hist, nb, n_slots, T, E,
+                       counts, offsets, prep->chunks, prep->n_chunks, prep->chunk_tokens, prep->routed_chunk_tokens);
+        if (s != MOE_OK) return s;
+        if (ev_place) cudaEventRecord(ev_place, stream);
+        return launch_pdl(bucket_place_kernel, dim3(nb), dim3(BK_THREADS), 0, stream, ids, n_slots, E,
+                          (const int32_t*)prep->bucket_hist, perm, inv_perm);
+    }
     return launch_pdl(bucket_kernel, dim3(1), dim3(BK_THREADS), 0, stream, ids, T * k, T, E, counts, offsets, perm,
                       inv_perm, prep ? prep->chunks : (ChunkEntry*)nullptr, prep ? prep->n_chunks : (int32_t*)nullptr,
                       prep ? prep->chunk_tokens : 16, prep ? prep->routed_chunk_tokens : 16,

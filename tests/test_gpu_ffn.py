@@ -39,6 +39,7 @@ RAGGED = [
     (50, 256, 384, 256, 6, 3),
     (16, 512, 1024, 768, 16, 1),
     (300, 256, 256, 128, 3, 2),      # more than one 256-token tile per expert
+    (2100, 256, 256, 128, 8, 2),     # 4200 slots: bucketing over several CTAs
 ]
 
 
