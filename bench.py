@@ -209,6 +209,10 @@ class ClockSampler:
     def summary(self, t0: float, t1: float):
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
         if not inside:
+            # a timed region shorter than the sampling period: the samples
+            # taken within one period of it
+            inside = [s for s in self.samples if t0 - 0.03 <= s[0] <= t1 + 0.03]
+        if not inside:
             return None
         reasons = set()
         for s in inside:

@@ -99,7 +99,8 @@ def test_int4_worked_group_on_gpu():
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("rows,cols,nv,ub", [(1, 8, 1, math.inf), (33, 5120, 30, math.inf),
-                                               (64, 8192, 64, 2.0), (5, 40, 3, 0.5)])
+                                               (64, 8192, 64, 2.0), (5, 40, 3, 0.5), (7, 3000, 7, math.inf),
+                                               (3, 8200, 2, math.inf)])
 def test_fp8_rows_bit_exact(dtype, rows, cols, nv, ub):
     g = synth.stream(12, rows * 3 + cols)
     x = g.standard_normal((rows, cols), dtype=np.float32) * np.float32(3.0)
@@ -107,6 +108,39 @@ def test_fp8_rows_bit_exact(dtype, rows, cols, nv, ub):
     xt = torch.from_numpy(x).to(dtype)
     q, s = moe.quantize_fp8_rows(xt.cuda(), num_valid_rows=nv, scale_ub=ub)
     q_ref, s_ref = oq.fp8_row_quantize(xt.float().numpy(), num_valid_rows=nv, scale_ub=ub)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def _fp8_near_ties(rows, cols, seed):
+    """Rows whose quotients x / s sit on or within a few ulps of the midpoint
+    between two e4m3 values (where the rounding decision is taken), across
+    the whole e4m3 range including the subnormals."""
+    g = synth.stream(seed, 77)
+    pos = oq.E4M3_VALUES[:0x7F]
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)     # 4 significant bits: exact in fp32
+    x = np.zeros((rows, cols), np.float32)
+    for r in range(rows):
+        m = np.float32(g.uniform(0.5, 4.0))
+        s = np.float32(m / np.float32(448.0))
+        v = (g.choice(mids, cols - 1) * np.where(g.integers(0, 2, cols - 1) == 1, 1, -1)).astype(np.float32)
+        v = (v * s).astype(np.float32)
+        steps = g.integers(-3, 4, cols - 1)
+        for j in range(cols - 1):
+            for _ in range(abs(int(steps[j]))):
+                v[j] = np.nextafter(v[j], np.float32(np.inf if steps[j] > 0 else -np.inf), dtype=np.float32)
+        x[r, 0] = m                                              # the row maximum
+        x[r, 1:] = np.clip(v, -m, m)
+    return x
+
+
+@pytest.mark.parametrize("cols", [1024, 8192])
+def test_fp8_rows_bit_exact_near_ties(cols):
+    """e4m3 codes of quotients on and around the format's rounding midpoints:
+    the GPU must take the IEEE quotient's rounding decisions, as the oracle."""
+    x = _fp8_near_ties(16, cols, 9)
+    q, s = moe.quantize_fp8_rows(torch.from_numpy(x).cuda())
+    q_ref, s_ref = oq.fp8_row_quantize(x)
     assert np.array_equal(s.cpu().numpy(), s_ref)
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
