@@ -416,50 +416,92 @@ __global__ void __launch_bounds__(BK_THREADS) bucket_hist_kernel(const int32_t* 
     for (int e = threadIdx.x; e < E; e += BK_THREADS) hist[blockIdx.x * E + e] = s_count[e];
 }
 
+// Inclusive prefix sum over the 32 lanes of a warp.
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Exclusive prefix over a[0 .. n) (n <= BK_MAX_E) in shared memory by warp 0;
+// returns the total to every lane of warp 0.
+__device__ __forceinline__ int warp_exclusive_scan_smem(int* a, int n, int lane) {
+    int carry = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int v = i0 + lane < n ? a[i0 + lane] : 0;
+        const int inc = warp_inclusive_scan(v, lane);
+        if (i0 + lane < n) a[i0 + lane] = carry + inc - v;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    return carry;
+}
+
 __global__ void __launch_bounds__(BK_THREADS) bucket_scan_kernel(
     int32_t* __restrict__ hist, int n_blocks, int n_slots, int T, int E, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, ChunkEntry* __restrict__ chunks, int32_t* __restrict__ n_chunks,
     int chunk_tokens, int routed_chunk_tokens) {
     __shared__ int s_count[BK_MAX_E];
     __shared__ int s_base[BK_MAX_E];
+    __shared__ int s_cbase[BK_MAX_E];   // first chunk-list entry of each expert
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     griddep_launch_dependents();
     griddep_wait();
-    for (int e = threadIdx.x; e < E; e += BK_THREADS) {
-        int c = 0;
-        for (int b = 0; b < n_blocks; ++b) c += hist[b * E + e];
-        s_count[e] = c;
+    // a warp per expert: lanes over the blocks, a running carry over groups
+    // of 32 blocks; each (block, expert) entry becomes that block's first
+    // position within the expert (relative; the expert's base is added below)
+    for (int e = warp; e < E; e += BK_WARPS) {
+        int carry = 0;
+        for (int b0 = 0; b0 < n_blocks; b0 += 32) {
+            const int b = b0 + lane;
+            const int c = b < n_blocks ? hist[b * E + e] : 0;
+            const int inc = warp_inclusive_scan(c, lane);
+            if (b < n_blocks) hist[b * E + e] = carry + inc - c;
+            carry += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) s_count[e] = carry;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_count[e]; }
-        offsets[E] = n_slots;
-        if (chunks != nullptr) {   // the FFN kernels' task list, as bucket_kernel writes it
-            int n = 0;
-            for (int t0 = 0; t0 < T; t0 += chunk_tokens) {
-                ChunkEntry ce; ce.expert = -1; ce.start = t0; ce.count = min(chunk_tokens, T - t0); ce.pad = 0;
-                chunks[n++] = ce;
+    const int n_sh = (T + chunk_tokens - 1) / chunk_tokens;
+    if (warp == 0) {
+        for (int e = lane; e < E; e += 32) {
+            s_base[e] = s_count[e];
+            s_cbase[e] = (s_count[e] + routed_chunk_tokens - 1) / routed_chunk_tokens;
+        }
+        __syncwarp();
+        warp_exclusive_scan_smem(s_base, E, lane);
+        const int n_routed = warp_exclusive_scan_smem(s_cbase, E, lane);
+        if (lane == 0) {
+            offsets[E] = n_slots;
+            if (chunks != nullptr) {
+                n_chunks[1] = n_sh;
+                n_chunks[0] = n_sh + n_routed;
             }
-            n_chunks[1] = n;
-            for (int e = 0; e < E; ++e)
-                for (int s = 0; s < s_count[e]; s += routed_chunk_tokens) {
-                    ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + s;
-                    ce.count = min(routed_chunk_tokens, s_count[e] - s);
-                    ce.pad = 0;
-                    chunks[n++] = ce;
-                }
-            n_chunks[0] = n;
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += BK_THREADS) {
+    for (int e = tid; e < E; e += BK_THREADS) {
         counts[e] = s_count[e];
         offsets[e] = s_base[e];
-        int base = s_base[e];
-        for (int b = 0; b < n_blocks; ++b) {   // each block's first position of expert e
-            const int c = hist[b * E + e];
-            hist[b * E + e] = base;
-            base += c;
+    }
+    // absolute first positions: add each expert's base
+    for (int i = tid; i < n_blocks * E; i += BK_THREADS) hist[i] += s_base[i % E];
+    if (chunks != nullptr) {   // the FFN kernels' task list, as bucket_kernel writes it
+        for (int c = tid; c < n_sh; c += BK_THREADS) {
+            ChunkEntry ce; ce.expert = -1; ce.start = c * chunk_tokens;
+            ce.count = min(chunk_tokens, T - c * chunk_tokens); ce.pad = 0;
+            chunks[c] = ce;
+        }
+        // one warp per expert, lanes over its chunks
+        for (int e = warp; e < E; e += BK_WARPS) {
+            const int cnt = s_count[e];
+            for (int j = lane; j * routed_chunk_tokens < cnt; j += 32) {
+                ChunkEntry ce; ce.expert = e; ce.start = s_base[e] + j * routed_chunk_tokens;
+                ce.count = min(routed_chunk_tokens, cnt - j * routed_chunk_tokens); ce.pad = 0;
+                chunks[n_sh + s_cbase[e] + j] = ce;
+            }
         }
     }
 }
