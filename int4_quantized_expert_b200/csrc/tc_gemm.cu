@@ -58,12 +58,13 @@ constexpr int TC_CSTAGES = 2 * TC_STAGES;
 constexpr int TC_TMEM_COLS = 512;
 static_assert(TC_STAGE_BYTES % 1024 == 0, "stage alignment");
 // bf16 / e4m3 modes: the weight tiles (the routed ones read once from DRAM)
-// have a ring of their own, filled by warp 2 up to TC_AST_F8 stages ahead of
+// have a ring of their own, filled by warp 2 up to TC_WSTAGES stages ahead of
 // the MMAs, in the space of the stages' weight halves and the (unused) code
 // ring; the token tiles keep TC_STAGES slots.  Against one ring of four
-// token + weight stages the Maverick-shaped e4m3 GEMMs ran 4 % faster.
-constexpr int TC_AST_F8 = 6;
-static_assert(TC_STAGES * TC_B_BYTES + TC_AST_F8 * TC_A_BYTES == TC_STAGES * TC_STAGE_BYTES + TC_CSTAGES * TC_C_BYTES,
+// token + weight stages the Maverick-shaped e4m3 GEMMs ran 4 % faster and the
+// bf16 ones 2-4 %; three token slots and eight weight slots were slower.
+constexpr int TC_WSTAGES = 6;
+static_assert(TC_STAGES * TC_B_BYTES + TC_WSTAGES * TC_A_BYTES == TC_STAGES * TC_STAGE_BYTES + TC_CSTAGES * TC_C_BYTES,
               "e4m3 rings");
 
 struct TcSmem {
@@ -72,8 +73,8 @@ struct TcSmem {
     uint64_t empty[TC_STAGES];     // the stage's MMAs completed
     uint64_t cfull[TC_CSTAGES];    // int4 codes of a code slot landed
     uint64_t cempty[TC_CSTAGES];   // converter warps read the code slot
-    uint64_t a_full[TC_AST_F8];    // e4m3: the weight slot landed (tx counted)
-    uint64_t a_empty[TC_AST_F8];   // e4m3: the MMAs reading the weight slot completed
+    uint64_t a_full[TC_WSTAGES];    // bf16 / e4m3: the weight slot landed (tx counted)
+    uint64_t a_empty[TC_WSTAGES];   // bf16 / e4m3: the MMAs reading the weight slot completed
     uint64_t acc_full[2];          // accumulator holds a finished tile
     uint64_t acc_empty[2];         // epilogue finished reading the accumulator
     uint32_t tmem_base;
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
             mbar_init(&sm->empty[i], 1);
         }
         for (int i = 0; i < TC_CSTAGES; ++i) { mbar_init(&sm->cfull[i], 1); mbar_init(&sm->cempty[i], 8); }
-        for (int i = 0; i < TC_AST_F8; ++i) { mbar_init(&sm->a_full[i], 1); mbar_init(&sm->a_empty[i], 1); }
+        for (int i = 0; i < TC_WSTAGES; ++i) { mbar_init(&sm->a_full[i], 1); mbar_init(&sm->a_empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&sm->acc_full[i], 1); mbar_init(&sm->acc_empty[i], 4); }
         fence_barrier_init();
     }
@@ -184,8 +185,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 const ChunkEntry ce = p.chunks[c_begin + ci];
                 const int e = ce.expert < 0 ? 0 : ce.expert;
                 for (int kk = 0; kk < nk; ++kk, ++it) {
-                    const uint32_t as = it % TC_AST_F8;
-                    if (!mbar_wait(&sm->a_empty[as], ((it / TC_AST_F8) & 1) ^ 1, p.status)) { ok = false; break; }
+                    const uint32_t as = it % TC_WSTAGES;
+                    if (!mbar_wait(&sm->a_empty[as], ((it / TC_WSTAGES) & 1) ^ 1, p.status)) { ok = false; break; }
                     unsigned char* sa = fring + as * TC_A_BYTES;
                     mbar_arrive_expect_tx(&sm->a_full[as], TC_A_BYTES);
                     // 16-row boxes; gate/up: gate rows, up rows, gate rows, ... (same features)
@@ -203,9 +204,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 }
             }
             // wind down: wait (bounded) for the weight loads still in flight to land
-            for (uint32_t i = 0; i < TC_AST_F8 && i < it; ++i) {
+            for (uint32_t i = 0; i < TC_WSTAGES && i < it; ++i) {
                 const uint32_t j = it - 1 - i;
-                mbar_wait(&sm->a_full[j % TC_AST_F8], (j / TC_AST_F8) & 1, nullptr);
+                mbar_wait(&sm->a_full[j % TC_WSTAGES], (j / TC_WSTAGES) & 1, nullptr);
             }
         }
     } else if (warp == 2 && INT4) {
@@ -256,10 +257,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const uint32_t slot = it % TC_STAGES;
                     const uint32_t par = (it / TC_STAGES) & 1;
-                    const uint32_t as = it % TC_AST_F8;
+                    const uint32_t as = it % TC_WSTAGES;
                     if (!mbar_wait(&sm->full[slot], par, p.status)) { ok = false; break; }
                     if (INT4 && !mbar_wait(&sm->a_ready[slot], par, p.status)) { ok = false; break; }
-                    if (SEPA && !mbar_wait(&sm->a_full[as], (it / TC_AST_F8) & 1, p.status)) { ok = false; break; }
+                    if (SEPA && !mbar_wait(&sm->a_full[as], (it / TC_WSTAGES) & 1, p.status)) { ok = false; break; }
                     tc_fence_after();
                     const unsigned char* st = base + slot * B_PITCH;
                     const uint64_t bd = sw128_desc(st);
