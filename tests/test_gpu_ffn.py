@@ -71,6 +71,23 @@ def test_repeat_calls_identical():
     assert torch.equal(o1, o2)
 
 
+@pytest.mark.parametrize("shape", [synth.LayerShape("k4", 600, 256, 384, 8, 4, 256),
+                                   synth.LayerShape("fp8_k8", 512, 256, 512, 16, 8, 256, "fp8")],
+                         ids=lambda s: s.name)
+def test_repeat_calls_identical_k_slots(shape):
+    """k > 1 on the tensor-core path: the last of a token's k down tiles to
+    finish sums its slots, in slot order -- bit-identical outputs whichever
+    tile is last, call after call."""
+    b = build(shape)
+    b.gpu.set_path(moe.PATH_PREFILL)
+    x = b.x.cuda()
+    o1 = b.gpu(x).clone()
+    for _ in range(3):
+        assert torch.equal(b.gpu(x), o1)
+    got, ref = _run(b, moe.PATH_PREFILL)
+    assert rel_err(got, ref) <= TOL
+
+
 def test_host_buffers_match_device_call():
     b = build(synth.SHAPES["tiny"])
     dev = b.gpu(b.x.cuda()).cpu()

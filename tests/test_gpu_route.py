@@ -56,6 +56,14 @@ def test_route_ragged(T, D, E, k):
     _check(synth.LayerShape("r", T, D, 128, E, k, 128))
 
 
+@pytest.mark.parametrize("T,D,E,k", [(16384, 128, 256, 8), (40000, 128, 7, 2)])
+def test_route_many_bucket_blocks(T, D, E, k):
+    """More than 32 blocks of 2048 slots (131072 and 80000 slots): the
+    multi-CTA bucketing's per-expert scans carry across groups of 32 blocks,
+    and with 256 experts the expert scans span eight warp passes."""
+    _check(synth.LayerShape("r", T, D, 128, E, k, 128))
+
+
 def test_route_all_tokens_on_one_expert():
     T, D, E = 300, 256, 8
     wr = torch.zeros(E, D, dtype=torch.bfloat16)
