@@ -553,7 +553,8 @@ def run_dense(args, rank: int, world: int, dev: torch.device):
         "roofline": roof,
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2, "ms_per_step": e2e_ms},
-        "gpu_launches": (4 + (1 if args.rmsnorm else 0)) * args.steps,   # [rmsnorm,] prep, gate/up, down, combine
+        # [rmsnorm,] prep, gate/up, down; the tensor-core path adds the combine
+        "gpu_launches": ((3 if T <= 64 else 4) + (1 if args.rmsnorm else 0)) * args.steps,
         "clocks": clocks,
     }
 
