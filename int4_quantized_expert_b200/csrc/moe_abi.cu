@@ -493,22 +493,28 @@ moe_status ffn_prefill_path(const moe_layer_desc& L, const bf16* x, const bf16* 
         bool ok;
         if (fp8)
             ok = make_tmap_2d(&m_gu.b, at<uint8_t>(ws, W.xq), 1, L.D, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_gu.b_small, at<uint8_t>(ws, W.xq), 1, L.D, S_pad, 128, TC_SMALL_TOKENS, true) &&
                  make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D, E * L.F, 128, 16, true) &&
                  make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D, E * L.F, 128, 16, true) &&
                  make_tmap_2d(&m_dn.b, at<uint8_t>(ws, W.hq), 1, L.F, S_pad, 128, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_dn.b_small, at<uint8_t>(ws, W.hq), 1, L.F, S_pad, 128, TC_SMALL_TOKENS, true) &&
                  make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F, E * L.D, 128, 16, true);
         else
             ok = make_tmap_2d(&m_gu.b, x_sorted, 2, L.D, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_gu.b_small, x_sorted, 2, L.D, S_pad, 64, TC_SMALL_TOKENS, true) &&
                  make_tmap_2d(&m_gu.a0, L.w_gate, 1, L.D / 2, E * L.F, 32, 64, false) &&
                  make_tmap_2d(&m_gu.a1, L.w_up, 1, L.D / 2, E * L.F, 32, 64, false) &&
                  make_tmap_2d(&m_dn.b, h_sorted, 2, L.F, S_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_dn.b_small, h_sorted, 2, L.F, S_pad, 64, TC_SMALL_TOKENS, true) &&
                  make_tmap_2d(&m_dn.a0, L.w_down, 1, L.F / 2, E * L.D, 32, 64, false);
         // the shared expert's token tiles come straight from x: a 256-row box that
         // runs past row T - 1 reads zeros there
         ok = ok && make_tmap_2d(&m_sgu.b, xin, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_sgu.b_small, xin, 2, L.D, uint64_t(T), 64, TC_SMALL_TOKENS, true) &&
                   make_tmap_2d(&m_sgu.a0, L.ws_gate, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sgu.a1, L.ws_up, 2, L.D, L.F_shared, 64, 16, true) &&
                   make_tmap_2d(&m_sdn.b, h_s, 2, L.F_shared, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&m_sdn.b_small, h_s, 2, L.F_shared, T_pad, 64, TC_SMALL_TOKENS, true) &&
                   make_tmap_2d(&m_sdn.a0, L.ws_down, 2, L.F_shared, L.D, 64, 16, true);
         if (!ok) return false;
         m_dn.a1 = m_dn.a0;
@@ -993,9 +999,11 @@ moe_status dense_forward_impl(const moe_dense_desc* layer, const void* x, int32_
     if (!same_dense_key(key, key_p)) {
         key_p.valid = false;
         bool ok = make_tmap_2d(&mg.b, xin, 2, L.D, uint64_t(T), 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&mg.b_small, xin, 2, L.D, uint64_t(T), 64, TC_SMALL_TOKENS, true) &&
                   make_tmap_2d(&mg.a0, L.w_gate, 2, L.D, L.F, 64, 16, true) &&
                   make_tmap_2d(&mg.a1, L.w_up, 2, L.D, L.F, 64, 16, true) &&
                   make_tmap_2d(&md.b, h, 2, L.F, T_pad, 64, TC_BLOCK_TOKENS, true) &&
+                 make_tmap_2d(&md.b_small, h, 2, L.F, T_pad, 64, TC_SMALL_TOKENS, true) &&
                   make_tmap_2d(&md.a0, L.w_down, 2, L.F, L.D, 64, 16, true);
         if (!ok) return MOE_ERR_CUDA;
         md.a1 = md.a0;

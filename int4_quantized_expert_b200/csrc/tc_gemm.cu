@@ -105,7 +105,8 @@ __device__ __forceinline__ int tile_n(int count) { return min(TC_BLOCK_TOKENS, (
 // ---------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
-    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_a0,
+    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_bs,
+    const __grid_constant__ CUtensorMap tm_a0,
     const __grid_constant__ CUtensorMap tm_a1, TcParams p) {
     constexpr bool INT4 = MODE == TC_GATEUP_INT4 || MODE == TC_DOWN_INT4;
     constexpr bool FP8 = MODE == TC_GATEUP_FP8 || MODE == TC_DOWN_FP8;
@@ -154,18 +155,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(
         // ------------------------- TMA producer of the token tiles -------------------------
         // (int4 codes and the bf16 / e4m3 weights come through their own rings, warp 2)
         if (lane == 0) {
-            prefetch_tmap(&tm_b); prefetch_tmap(&tm_a0); prefetch_tmap(&tm_a1);
+            prefetch_tmap(&tm_b); prefetch_tmap(&tm_bs); prefetch_tmap(&tm_a0); prefetch_tmap(&tm_a1);
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
                 int ci, fb;
                 tile_coords(tile, c_end - c_begin, p.n_fblocks, ci, fb);
                 const ChunkEntry ce = p.chunks[c_begin + ci];
+                // a chunk of a few tokens (an expert's tail) loads a box of only
+                // TC_SMALL_TOKENS rows: with the full box it moved as many bytes
+                // per stage as a full tile for a sliver of its MMA work
+                const bool small = tile_n(ce.count) <= TC_SMALL_TOKENS;
+                const CUtensorMap* mb = small ? &tm_bs : &tm_b;
+                const uint32_t bbytes = small ? uint32_t(TC_SMALL_TOKENS * 128) : uint32_t(TC_B_BYTES);
                 for (int kk = 0; kk < nk; ++kk, ++it) {
                     const uint32_t slot = it % TC_STAGES;
                     if (!mbar_wait(&sm->empty[slot], ((it / TC_STAGES) & 1) ^ 1, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sm->full[slot], TC_B_BYTES);
-                    tma_load_2d(base + slot * B_PITCH, &tm_b, &sm->full[slot], kk * KSTEP, ce.start);
+                    mbar_arrive_expect_tx(&sm->full[slot], bbytes);
+                    tma_load_2d(base + slot * B_PITCH, mb, &sm->full[slot], kk * KSTEP, ce.start);
                 }
             }
             // wind down: wait (bounded) for the stages still in flight to land
@@ -577,7 +584,7 @@ moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cud
 #define TC_LAUNCH(M)                                                                                     \
     do {                                                                                                 \
         if (allow_max_smem(tc_gemm_kernel<M>) != MOE_OK) return MOE_ERR_CUDA;                         \
-        tc_gemm_kernel<M><<<sms, TC_THREADS, smem, stream>>>(maps.b, maps.a0, maps.a1, prm);           \
+        tc_gemm_kernel<M><<<sms, TC_THREADS, smem, stream>>>(maps.b, maps.b_small, maps.a0, maps.a1, prm); \
     } while (0)
     switch (mode) {
         case TC_GATEUP_INT4: TC_LAUNCH(TC_GATEUP_INT4); break;

@@ -43,11 +43,15 @@ struct TcParams {
 
 struct TcMaps {
     CUtensorMap b;       // tokens: bf16 [rows, K], box 64 x 256, 128-byte swizzle
+    CUtensorMap b_small; // the same tensor, box 64 x TC_SMALL_TOKENS (e4m3: 128 x ...)
     CUtensorMap a0, a1;  // int4 codes uint8 [E * rows, K / 2], box 32 x 64; bf16 weights, box 64 x 16;
                          // or e4m3 weights uint8 [E * rows, K], box 128 x 16
 };
 
 constexpr int TC_BLOCK_TOKENS = 256;
+// Chunks of at most this many tokens load their token tiles with a box of
+// this many rows (the MMAs read only the chunk's rows).
+constexpr int TC_SMALL_TOKENS = 64;
 
 size_t tc_smem_bytes();
 moe_status launch_tc_gemm(int mode, const TcMaps& maps, const TcParams& prm, cudaStream_t stream);
